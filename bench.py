@@ -1,0 +1,308 @@
+"""Benchmark of one Orthrus decoding round on B200 (Qwen3-8B attention shape).
+
+A step = one full round (both attention views over 36 layers, argmax of both
+views' logits, consensus, KV commit of the accepted rows), replayed from CUDA
+graphs with every input resident in HBM.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the round on its own
+GPU (independent sequences; no data-path collective): weak scaling, value =
+rounds completed by all ranks / max-over-ranks device time.
+
+--impl reference times the CPU oracle (the only reference that exists for this
+method: its pages carry no code) on this host's cores, on a bounded sample of
+the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-attn HBM GB/s (% of peak) and consensus rounds/s, Qwen3-8B shape"
+WORKLOAD = dict(name="qwen3_8b_round", layers=36, B=1, Hq=32, Hkv=8, D=128, ctx=8192,
+                blk=32, vocab=151936, dtype="bf16", logits_dtype="f32", accept_mean=5.4)
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def config_dict():
+    w = WORKLOAD
+    return {"workload": w["name"], "layers": w["layers"], "B": w["B"], "Hq": w["Hq"],
+            "Hkv": w["Hkv"], "D": w["D"], "ctx": w["ctx"], "blk": w["blk"],
+            "vocab": w["vocab"], "kv_dtype": w["dtype"], "logits_dtype": w["logits_dtype"],
+            "accept_len": f"Geometric(mean {w['accept_mean']}) planted",
+            "l2": "inputs larger than L2: 1.21 GB KV cache, 2.46 GB of K/V streamed per round"}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid, self.proc, self.path = uuid, None, None
+
+    def start(self):
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.uuid:
+                cmd[1:1] = ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 10:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        smax = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
+        load = [s for s in sm if s > 0.5 * max(smax or [1])] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def oracle_round_sample(heads=1, layers_timed=1):
+    """Time the oracle on a bounded sample of one round and extrapolate to the
+    whole round: `layers_timed` layer(s) per view restricted to `heads` kv-head
+    group(s) (x 36 layers x 8/heads groups), plus the full argmax of both
+    views' 32 x 151936 logits, consensus and one layer's commit (x 36)."""
+    import oracle
+    from block_attention_b200 import synth
+    w = WORKLOAD
+    G = w["Hq"] // w["Hkv"]
+    cap = w["ctx"] + w["blk"]
+    nthreads = os.cpu_count() or 1
+    t_attn = 0.0
+    for v in (0, 1):
+        for l in range(layers_timed):
+            inp = synth.attn_inputs(1, G * heads, heads, w["D"], w["blk"], [w["ctx"]], cap,
+                                    w["dtype"], seed=7, layer=2 * l + v)
+            t0 = time.perf_counter()
+            oracle.block_attn(inp["q"], inp["k_blk"], inp["v_blk"], inp["k_cache"],
+                              inp["v_cache"], inp["ctx_lens"], v, nthreads=nthreads)
+            t_attn += time.perf_counter() - t0
+    t_attn *= (w["layers"] / layers_timed) * (w["Hkv"] / heads)
+    g = synth.rng(8)
+    acc = synth.geometric_accept(g, 1)
+    d, a = synth.planted_tokens(g, 1, w["blk"], w["vocab"], acc)
+    ld = synth.planted_logits(g, d, w["vocab"])
+    la = synth.planted_logits(g, a, w["vocab"])
+    t0 = time.perf_counter()
+    di, ai = oracle.vocab_argmax(ld), oracle.vocab_argmax(la)
+    L, ne, em, na = oracle.consensus(di[None], ai[None])
+    t_mid = time.perf_counter()
+    kc = np.zeros((1, w["Hkv"], cap, w["D"]), np.uint16)
+    vc = np.zeros_like(kc)
+    kb = np.zeros((1, w["blk"], w["Hkv"], w["D"]), np.uint16)
+    oracle.kv_commit(kc, vc, kb, kb.copy(), [w["ctx"]], ne)
+    t_end = time.perf_counter()
+    t_round = t_attn + (t_mid - t0) + w["layers"] * (t_end - t_mid)
+    sample = (f"{layers_timed} layer(s) per view x {heads} of {w['Hkv']} kv-head groups timed, "
+              f"extrapolated x{w['layers'] // layers_timed * w['Hkv'] // heads}; "
+              "full argmax (2 x 32 x 151936), consensus, 1-layer commit x36")
+    return 1.0 / t_round, nthreads, sample
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_round_sample()
+    vals, t0 = [], time.perf_counter()
+    for _ in range(args.steps):
+        v, cores, sample = oracle_round_sample()
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rounds/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(),
+            "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "rounds/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": wall}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    import block_attention_b200 as ba
+    from block_attention_b200.round import DecodeRound
+    ba.lib()
+    w = WORKLOAD
+    rnd = DecodeRound(layers=w["layers"], B=w["B"], Hq=w["Hq"], Hkv=w["Hkv"], D=w["D"],
+                      blk=w["blk"], vocab=w["vocab"], ctx_lens=[w["ctx"]] * w["B"],
+                      dtype=w["dtype"], logits_dtype=w["logits_dtype"],
+                      accept_mean=w["accept_mean"], seed=1000 + 3 + rank, device=dev)
+    rnd.capture()
+
+    for _ in range(args.warmup):
+        rnd.replay()
+    torch.cuda.synchronize()
+    expect_ne = np.minimum(rnd.accept + 1, w["blk"])
+    assert np.array_equal(rnd.n_emit.cpu().numpy(), expect_ne), "round result mismatch"
+    assert int(rnd.err.item()) == 0
+
+    # ---- timed region: K rounds from the graphs, inputs resident in HBM
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    clocks = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        rnd.replay(ev[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    clk = clocks.stop()
+
+    step_ms = [e[0].elapsed_time(e[4]) for e in ev]
+    attn_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = ev[0][0].elapsed_time(ev[-1][4])
+    t = torch.tensor([total_ms, sum(attn_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, attn_total_ms = float(t[0]), float(t[1])
+
+    launches_attn = 2 * w["layers"] * args.steps
+    attn_launch_us = attn_total_ms * 1e3 / launches_attn
+    bytes_per_launch = rnd.attn_bytes_per_launch()
+    hbm, src = peaks()
+    achieved = bytes_per_launch / (attn_launch_us * 1e-6) / 1e9
+    rounds_per_s = world * args.steps / (total_ms * 1e-3)
+    gpu_launches = rnd.kernels_per_round() * args.steps
+
+    # ---- end to end: per-round inputs from pinned host memory, results back
+    h_in, h_out = rnd.pinned_inputs(), rnd.pinned_outputs()
+    for _ in range(2):
+        rnd.h2d(h_in); rnd.replay(); rnd.d2h(h_out)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        bi = rnd.h2d(h_in)
+        rnd.replay()
+        bo = rnd.d2h(h_out)
+    e1.record()
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_rounds = world * args.steps / (float(te[0]) * 1e-3)
+    assert np.array_equal(h_out["n_emit"].numpy(), expect_ne)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_round_sample(heads=WORKLOAD["Hkv"], layers_timed=4)
+        cpu = {"value": v, "unit": "rounds/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    if world > 1:
+        dist.barrier()
+        rnd.graphs = None
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    rb = rnd.round_bytes()
+    line = {
+        "metric": METRIC, "value": rounds_per_s, "unit": "rounds/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_dict(),
+        "block_attn": {"gbs": achieved, "pct_of_peak": 100.0 * achieved / hbm,
+                       "us_per_launch": attn_launch_us, "bytes_per_launch": bytes_per_launch,
+                       "launches_per_round": 2 * w["layers"]},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": src, "traffic": None,
+                     "kernel": "block_attn (both views, per-layer launches)"},
+        "round_bytes": rb,
+        "round_hbm_gbs": sum(rb.values()) / (total_ms / args.steps * 1e-3) / 1e9,
+        "step_ms_median": statistics.median(step_ms),
+        "e2e": {"value": e2e_rounds, "unit": "rounds/s", "h2d_bytes_per_step": bi,
+                "d2h_bytes_per_step": bo},
+        "gpu_launches": gpu_launches,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

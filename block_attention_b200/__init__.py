@@ -1,0 +1,248 @@
+"""block_attention_b200 -- B200 (sm_100a) hot path of one Orthrus decoding round.
+
+Thin Python binding over the C ABI in ``include/orthrus.h`` (``liborthrus.so``,
+built in-tree by ``block_attention_b200.build``).  Every function here only
+marshals torch tensors into pointers and sizes; all arithmetic runs in the
+CUDA kernels.  There is no CPU fallback: if the library is missing or a
+tensor is not on a CUDA device, the call raises.
+
+Entry points (same names as the C ABI, minus the ``orthrus_`` prefix):
+    block_attn      both views' attention over the shared GQA KV cache
+    vocab_argmax    per-row argmax, lowest index on ties
+    consensus       accepted prefix, tokens to emit, next anchor
+    kv_commit       copy accepted block K/V rows into every layer's cache
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liborthrus.so")
+
+F32, BF16 = 0, 1
+BIDIR_BLOCK, CAUSAL_VERIFY = 0, 1
+STATUS = {0: "ok", -1: "EINVAL", -2: "EUNSUPPORTED", -3: "EWORKSPACE", -4: "ECAPACITY",
+          -5: "ECUDA"}
+
+
+class OrthrusError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({code})")
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
+                ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("blk", ctypes.c_int32), ("cap", ctypes.c_int32),
+                ("max_ctx", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("q", ctypes.c_void_p), ("k_blk", ctypes.c_void_p),
+                ("v_blk", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
+                ("v_cache", ctypes.c_void_p), ("ctx_lens", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("err", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class CommitArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("layers", ctypes.c_int32),
+                ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("blk", ctypes.c_int32), ("cap", ctypes.c_int32),
+                ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("cache_layer_stride", ctypes.c_int64),
+                ("k_blk", ctypes.c_void_p), ("v_blk", ctypes.c_void_p),
+                ("blk_layer_stride", ctypes.c_int64),
+                ("ctx_lens", ctypes.c_void_p), ("n_emit", ctypes.c_void_p),
+                ("err", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
+           "orthrus_block_attn_launches", "orthrus_vocab_argmax",
+           "orthrus_vocab_argmax_workspace", "orthrus_consensus", "orthrus_kv_commit",
+           "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version")
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load liborthrus.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        vp, i32, i64, sz = c.c_void_p, c.c_int32, c.c_int64, c.c_size_t
+        L.orthrus_block_attn.argtypes = [c.POINTER(AttnArgs), vp]
+        L.orthrus_block_attn_workspace.argtypes = [c.POINTER(AttnArgs)]
+        L.orthrus_block_attn_workspace.restype = sz
+        L.orthrus_block_attn_launches.argtypes = [c.POINTER(AttnArgs)]
+        L.orthrus_block_attn_launches.restype = c.c_int
+        L.orthrus_vocab_argmax.argtypes = [i32, vp, i32, i32, i64, vp, vp, vp, sz, vp]
+        L.orthrus_vocab_argmax_workspace.argtypes = [i32]
+        L.orthrus_vocab_argmax_workspace.restype = sz
+        L.orthrus_consensus.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, vp]
+        L.orthrus_kv_commit.argtypes = [c.POINTER(CommitArgs), vp]
+        L.orthrus_kv_commit_workspace.argtypes = [c.POINTER(CommitArgs)]
+        L.orthrus_kv_commit_workspace.restype = sz
+        L.orthrus_status_str.argtypes = [c.c_int]
+        L.orthrus_status_str.restype = c.c_char_p
+        L.orthrus_version.restype = c.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise OrthrusError(fn, rc)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be on a CUDA device (no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Workspace:
+    """Zero-initialised device scratch, grown on demand and reused.
+
+    The kernels return their ticket counters to zero, so one workspace serves
+    every later call issued on the same stream."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(ws, device, op):
+    """Caller's workspace, else a per-(device, op) default: ops must not share
+    one, since argmax/commit keep zeroed ticket counters in theirs."""
+    if ws is None:
+        dev = device.index if device.index is not None else torch.cuda.current_device()
+        ws = _default_ws.setdefault((dev, op), Workspace(torch.device("cuda", dev)))
+    return ws
+
+
+def attn_args(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, out=None,
+              scale=None, max_ctx=None, err=None) -> AttnArgs:
+    B, blk, Hq, D = q.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    return AttnArgs(_dtype(q), int(mask_mode), B, Hq, Hkv, D, blk, cap,
+                    cap if max_ctx is None else int(max_ctx),
+                    float(D ** -0.5 if scale is None else scale),
+                    q.data_ptr(), k_blk.data_ptr(), v_blk.data_ptr(), k_cache.data_ptr(),
+                    v_cache.data_ptr(), ctx_lens.data_ptr(),
+                    out.data_ptr() if out is not None else None,
+                    err.data_ptr() if err is not None else None, None, 0)
+
+
+def block_attn_workspace_bytes(args: AttnArgs) -> int:
+    return lib().orthrus_block_attn_workspace(ctypes.byref(args))
+
+
+def block_attn(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, *, out=None,
+               scale=None, max_ctx=None, err=None, workspace=None, stream=None):
+    """Attention of one layer for one round (see orthrus.h for the definition).
+
+    q [B, blk, Hq, D]; k_blk/v_blk [B, blk, Hkv, D]; k_cache/v_cache
+    [B, Hkv, cap, D]; ctx_lens int32 [B] on the device.  max_ctx bounds every
+    ctx_lens entry (default: cap).  Returns out [B, blk, Hq, D] (q's dtype)."""
+    _dev(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, out, err)
+    if ctx_lens.dtype != torch.int32:
+        raise TypeError("ctx_lens must be int32")
+    if out is None:
+        out = torch.empty_like(q)
+    a = attn_args(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, out, scale,
+                  max_ctx, err)
+    need = block_attn_workspace_bytes(a)
+    if need:
+        buf = _ws(workspace, q.device, "attn").get(need)
+        a.workspace, a.workspace_bytes = buf.data_ptr(), buf.numel()
+    _check("orthrus_block_attn", lib().orthrus_block_attn(ctypes.byref(a), _stream(stream)))
+    return out
+
+
+def vocab_argmax(logits, *, idx=None, maxval=None, workspace=None, stream=None):
+    """Row argmax of logits [rows, vocab] (row stride may exceed vocab)."""
+    _dev(idx, maxval)
+    if not logits.is_cuda or logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits must be a 2-D CUDA tensor with unit column stride")
+    rows, vocab = logits.shape
+    if idx is None:
+        idx = torch.empty(rows, dtype=torch.int32, device=logits.device)
+    need = lib().orthrus_vocab_argmax_workspace(rows)
+    buf = _ws(workspace, logits.device, "argmax").get(need)
+    _check("orthrus_vocab_argmax", lib().orthrus_vocab_argmax(
+        _dtype(logits), _ptr(logits), rows, vocab, logits.stride(0), _ptr(idx), _ptr(maxval),
+        _ptr(buf), buf.numel(), _stream(stream)))
+    return idx
+
+
+def consensus(draft, verify, *, accept_len=None, n_emit=None, emitted=None,
+              next_anchor=None, stream=None):
+    """Returns (accept_len [B], n_emit [B], emitted [B, blk], next_anchor [B])."""
+    _dev(draft, verify)
+    B, blk = draft.shape
+    dev = draft.device
+    mk = lambda t, shp: t if t is not None else torch.empty(shp, dtype=torch.int32, device=dev)
+    accept_len, n_emit, next_anchor = mk(accept_len, B), mk(n_emit, B), mk(next_anchor, B)
+    emitted = mk(emitted, (B, blk))
+    _check("orthrus_consensus", lib().orthrus_consensus(
+        _ptr(draft), _ptr(verify), B, blk, _ptr(accept_len), _ptr(n_emit), _ptr(emitted),
+        _ptr(next_anchor), _stream(stream)))
+    return accept_len, n_emit, emitted, next_anchor
+
+
+def kv_commit(k_cache, v_cache, k_blk, v_blk, ctx_lens, n_emit, *, err=None,
+              workspace=None, stream=None):
+    """Commit accepted rows for all layers and advance ctx_lens in place.
+
+    k_cache/v_cache [layers, B, Hkv, cap, D] (or [B, Hkv, cap, D] for one
+    layer); k_blk/v_blk [layers, B, blk, Hkv, D] (or [B, blk, Hkv, D])."""
+    _dev(k_cache, v_cache, k_blk, v_blk, ctx_lens, n_emit, err)
+    if k_cache.dim() == 4:
+        k_cache, v_cache = k_cache[None], v_cache[None]
+        k_blk, v_blk = k_blk[None], v_blk[None]
+    layers, B, Hkv, cap, D = k_cache.shape
+    blk = k_blk.shape[2]
+    a = CommitArgs(_dtype(k_cache), layers, B, Hkv, D, blk, cap, k_cache.data_ptr(),
+                   v_cache.data_ptr(), k_cache.stride(0), k_blk.data_ptr(), v_blk.data_ptr(),
+                   k_blk.stride(0), ctx_lens.data_ptr(), n_emit.data_ptr(),
+                   err.data_ptr() if err is not None else None, None, 0)
+    need = lib().orthrus_kv_commit_workspace(ctypes.byref(a))
+    buf = _ws(workspace, k_cache.device, "commit").get(need)
+    a.workspace, a.workspace_bytes = buf.data_ptr(), buf.numel()
+    _check("orthrus_kv_commit", lib().orthrus_kv_commit(ctypes.byref(a), _stream(stream)))
+    return ctx_lens

@@ -1,0 +1,133 @@
+// argmax.cu -- vocab-row argmax with lowest-index tie-break (the per-position
+// "most likely token" of both views, Orthrus explainer §四 steps 1-2).
+//
+// One pass over the logits, split across many CTAs per row so a 32 x 151936
+// matrix spreads over every SM.  Each element maps to a 64-bit key
+//     (order-preserving bits of the value) << 32 | (0xFFFFFFFF - index)
+// so the unsigned maximum of the keys is the largest value and, among equal
+// values, the smallest index.  NaN maps to key 0 and never wins; -0.0 is
+// canonicalised to +0.0 so the two zeros tie.  Because max is associative
+// and commutative, the result does not depend on how the row is split or in
+// which order CTAs finish.  Each CTA folds its key into the row's slot with
+// atomicMax; the last CTA of the row (ticket counter) decodes the key, writes
+// idx/maxval and returns the slot and the ticket to zero for the next call.
+#include "common.cuh"
+
+namespace orthrus {
+
+constexpr int kArgmaxThreads = 256;
+constexpr int kArgmaxChunk = 16384;  // elements per CTA (multiple of 8)
+
+__device__ __forceinline__ unsigned long long argmax_key(float v, int j) {
+  if (v != v) return 0ull;  // NaN
+  if (v == 0.f) v = 0.f;    // -0.0 -> +0.0
+  unsigned u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (unsigned)j);
+}
+
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  unsigned u = (unsigned)(k >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+  return __uint_as_float(u);
+}
+
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a,
+                                                     unsigned long long b) {
+  return a > b ? a : b;
+}
+
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kArgmaxThreads)
+argmax_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
+              int nchunks, unsigned long long* keys, unsigned* tickets,
+              int32_t* idx, float* maxval) {
+  const int c = blockIdx.x, r = blockIdx.y;
+  const T* row = logits + (int64_t)r * stride;
+  const int beg = c * kArgmaxChunk;
+  const int end = min(beg + kArgmaxChunk, vocab);
+  unsigned long long best = 0ull;
+  if (kVec) {
+    // 4 elements per vector load for f32 (16 B), 8 for bf16 (16 B)
+    constexpr int kV = 16 / sizeof(T);
+    constexpr int kIters = kArgmaxChunk / (kV * kArgmaxThreads);
+    uint4 buf[kIters];
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int j = beg + (it * kArgmaxThreads + threadIdx.x) * kV;
+      if (j + kV <= end) buf[it] = __ldcs(reinterpret_cast<const uint4*>(row + j));
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int j = beg + (it * kArgmaxThreads + threadIdx.x) * kV;
+      if (j + kV <= end) {
+        const T* e = reinterpret_cast<const T*>(&buf[it]);
+#pragma unroll
+        for (int u = 0; u < kV; ++u) best = umax64(best, argmax_key(to_f32(e[u]), j + u));
+      } else {
+        for (int u = 0; u < kV && j + u < end; ++u)
+          best = umax64(best, argmax_key(to_f32(row[j + u]), j + u));
+      }
+    }
+  } else {
+    for (int j = beg + threadIdx.x; j < end; j += kArgmaxThreads)
+      best = umax64(best, argmax_key(to_f32(row[j]), j));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    best = umax64(best, __shfl_xor_sync(0xffffffffu, best, off));
+  __shared__ unsigned long long warp_best[kArgmaxThreads / 32];
+  __shared__ bool last;
+  if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kArgmaxThreads / 32; ++w) best = umax64(best, warp_best[w]);
+    atomicMax(&keys[r], best);
+    __threadfence();
+    last = atomicAdd(&tickets[r], 1u) == (unsigned)nchunks - 1u;
+    if (last) {
+      const unsigned long long k = atomicExch(&keys[r], 0ull);
+      tickets[r] = 0u;
+      if (k == 0ull) {  // every element was NaN
+        idx[r] = 0;
+        if (maxval) maxval[r] = to_f32(row[0]);
+      } else {
+        idx[r] = (int32_t)(0xFFFFFFFFu - (unsigned)(k & 0xFFFFFFFFull));
+        if (maxval) maxval[r] = key_value(k);
+      }
+    }
+  }
+}
+
+size_t argmax_workspace_bytes(int rows) {
+  return (size_t)(((int64_t)rows * 12 + 255) / 256 * 256);
+}
+
+cudaError_t launch_argmax(int dtype, const void* logits, int rows, int vocab,
+                          int64_t stride, int32_t* idx, float* maxval, void* ws,
+                          cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  unsigned long long* keys = static_cast<unsigned long long*>(ws);
+  unsigned* tickets = reinterpret_cast<unsigned*>(keys + rows);
+  const int nchunks = ceil_div(vocab, kArgmaxChunk);
+  dim3 grid(nchunks, rows);
+  const size_t es = dtype == ORTHRUS_F32 ? 4 : 2;
+  const bool vec = (reinterpret_cast<uintptr_t>(logits) % 16 == 0) &&
+                   ((stride * (int64_t)es) % 16 == 0);
+  if (dtype == ORTHRUS_F32) {
+    auto p = static_cast<const float*>(logits);
+    if (vec)
+      argmax_kernel<float, true><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
+    else
+      argmax_kernel<float, false><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
+  } else {
+    auto p = static_cast<const __nv_bfloat16*>(logits);
+    if (vec)
+      argmax_kernel<__nv_bfloat16, true><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
+    else
+      argmax_kernel<__nv_bfloat16, false><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace orthrus

@@ -1,0 +1,15 @@
+// attn_tc.cuh -- tensor-core (tcgen05) block attention for bf16 tensors.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "orthrus.h"
+
+namespace orthrus {
+
+bool tc_supported(const orthrus_attn_args& a);
+size_t tc_workspace_bytes(const orthrus_attn_args& a);
+int tc_launch(const orthrus_attn_args& a, cudaStream_t st);
+int tc_launches(const orthrus_attn_args& a);
+
+}  // namespace orthrus

@@ -66,7 +66,7 @@ def cast(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def attn_inputs(B, Hq, Hkv, D, blk, ctx_lens, cap, dtype="f32", seed=0, layer=0,
-                std=1.0):
+                std=1.0, with_cache=True):
     """Q/K/V for one layer of one round: all entries ~ N(0, std).
 
     Returns q [B, blk, Hq, D], k_blk/v_blk [B, blk, Hkv, D],
@@ -78,7 +78,10 @@ def attn_inputs(B, Hq, Hkv, D, blk, ctx_lens, cap, dtype="f32", seed=0, layer=0,
         "q": cast(normal(rng(seed, S_Q, layer), (B, blk, Hq, D), std), dtype),
         "k_blk": cast(normal(rng(seed, S_KBLK, layer), (B, blk, Hkv, D), std), dtype),
         "v_blk": cast(normal(rng(seed, S_VBLK, layer), (B, blk, Hkv, D), std), dtype),
+        "ctx_lens": ctx_lens,
     }
+    if not with_cache:
+        return out
     kc = np.zeros((B, Hkv, cap, D), np.float32)
     vc = np.zeros((B, Hkv, cap, D), np.float32)
     gk, gv = rng(seed, S_KC, layer), rng(seed, S_VC, layer)
@@ -88,7 +91,6 @@ def attn_inputs(B, Hq, Hkv, D, blk, ctx_lens, cap, dtype="f32", seed=0, layer=0,
         vc[b, :, :n] = normal(gv, (Hkv, n, D), std)
     out["k_cache"] = cast(kc, dtype)
     out["v_cache"] = cast(vc, dtype)
-    out["ctx_lens"] = ctx_lens
     return out
 
 

@@ -1,0 +1,183 @@
+/*
+ * orthrus.h -- C ABI of the B200 (sm_100a) hot path of one Orthrus
+ * self-speculative decoding round.
+ *
+ * One round (Orthrus explainer, cjcn.com.cn, on arXiv:2605.12825, §四):
+ *   1. diffusion view: the block [anchor, MASK x (blk-1)] attends to the frozen
+ *      AR model's KV cache and, bidirectionally, to its own block K/V
+ *      (orthrus_block_attn, ORTHRUS_BIDIR_BLOCK), per layer;
+ *      LM-head logits -> orthrus_vocab_argmax -> drafts d[0..blk)
+ *   2. AR view: [anchor, d0..d_{blk-2}] verified causally over the same cache
+ *      (orthrus_block_attn, ORTHRUS_CAUSAL_VERIFY), per layer;
+ *      logits -> orthrus_vocab_argmax -> a[0..blk)
+ *   3. orthrus_consensus: accept the agreeing prefix plus one correction token
+ *   4. orthrus_kv_commit: only the accepted rows' AR K/V enter the cache
+ *
+ * Conventions (all entry points):
+ *   - Every pointer is caller-owned device memory unless stated otherwise; the
+ *     library allocates nothing and keeps no state between calls other than
+ *     the zero-initialised workspaces the caller passes in.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *     never synchronise it.  Lengths (ctx_lens, n_emit) stay on the device, so
+ *     a whole round can be captured in one CUDA graph.
+ *   - Arguments the host can check are checked before any launch; a bad one
+ *     returns a negative status and launches nothing.  Conditions only the
+ *     device can see (a device-resident length out of range) set the optional
+ *     device error word `err` (first error code wins) and skip the affected
+ *     sequence's writes; kernels never trap.
+ *   - Workspaces: query the size, allocate it once, zero it once
+ *     (cudaMemset 0).  Kernels leave their ticket counters at zero again, so
+ *     the same workspace serves every later call on the same stream.  After a
+ *     call that reported an error, zero it again.
+ *   - Tensors are dense, row-major, with the layouts written next to each
+ *     field.  dtype applies to every floating-point tensor of a call.
+ */
+#ifndef ORTHRUS_H
+#define ORTHRUS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ORTHRUS_VERSION 10000 /* major*10000 + minor*100 + patch */
+
+typedef struct CUstream_st* orthrus_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  ORTHRUS_OK = 0,
+  ORTHRUS_EINVAL = -1,       /* null pointer, negative size, bad enum */
+  ORTHRUS_EUNSUPPORTED = -2, /* valid but not implemented (D, G*blk, ...) */
+  ORTHRUS_EWORKSPACE = -3,   /* workspace missing or too small */
+  ORTHRUS_ECAPACITY = -4,    /* a length exceeds the cache capacity */
+  ORTHRUS_ECUDA = -5         /* a CUDA launch or attribute call failed */
+} orthrus_status;
+
+typedef enum { ORTHRUS_F32 = 0, ORTHRUS_BF16 = 1 } orthrus_dtype;
+
+typedef enum {
+  /* Diffusion view (explainer §二 and §三): every block row sees the cache
+   * rows [0, n) -- the context before the anchor -- and all blk block rows. */
+  ORTHRUS_BIDIR_BLOCK = 0,
+  /* AR verify view (explainer §四 step 2): block row i sees cache rows
+   * [0, n) and block rows [0, i]; row i equals a single-token decode at
+   * absolute position n + i. */
+  ORTHRUS_CAUSAL_VERIFY = 1
+} orthrus_mask_mode;
+
+/* ------------------------------------------------------------------------
+ * Block attention (both views), one layer.
+ *
+ * For sequence b (context n = ctx_lens[b]), block row i in [0, blk) and query
+ * head h, with kv-head g = h / (Hq / Hkv):
+ *   out[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k_j) v_j
+ * over the visible keys j of the mask mode, where key positions [0, n) come
+ * from k_cache/v_cache[b,g,0:n,:] and positions n + r from k_blk/v_blk[b,r,g,:].
+ *
+ * Arithmetic: F32 tensors -> FP32 FMA on CUDA cores, split-KV by absolute key
+ * position (fixed 256-key chunks) with a fixed-order combine, so a causal row
+ * reproduces single-token decoding bit for bit.  BF16 tensors -> tcgen05
+ * tensor-core tiles (bf16 products, FP32 accumulation, bf16 softmax weights),
+ * FP32 online softmax, bf16 output.
+ * ---------------------------------------------------------------------- */
+typedef struct orthrus_attn_args {
+  int32_t dtype;     /* orthrus_dtype of q, k_blk, v_blk, caches and out */
+  int32_t mask_mode; /* orthrus_mask_mode */
+  int32_t B;         /* sequences (0 = nothing to do) */
+  int32_t Hq, Hkv;   /* query heads, kv heads; Hq % Hkv == 0 */
+  int32_t D;         /* head dim: 64 or 128 */
+  int32_t blk;       /* block rows, 1..32; (Hq/Hkv)*blk <= 128 */
+  int32_t cap;       /* cache rows per (sequence, kv-head) */
+  int32_t max_ctx;   /* host bound on every ctx_lens[b]; 0 <= max_ctx <= cap.
+                        Sizes the grid; a device length above it is an error. */
+  float scale;       /* softmax scale, usually 1/sqrt(D) */
+  const void* q;       /* [B, blk, Hq, D] */
+  const void* k_blk;   /* [B, blk, Hkv, D] block K (bidir: diffusion K_diff; causal: AR K) */
+  const void* v_blk;   /* [B, blk, Hkv, D] */
+  const void* k_cache; /* [B, Hkv, cap, D] frozen AR K cache, rows [0, n) valid */
+  const void* v_cache; /* [B, Hkv, cap, D] */
+  const int32_t* ctx_lens; /* [B] device, committed context length n per sequence */
+  void* out;           /* [B, blk, Hq, D], same dtype as q */
+  int32_t* err;        /* optional device int32 error word (NULL = none) */
+  void* workspace;     /* zero-initialised, orthrus_block_attn_workspace() bytes */
+  size_t workspace_bytes;
+} orthrus_attn_args;
+
+/* Bytes of workspace orthrus_block_attn needs for these arguments (0 if none).
+ * Pointers in `a` are not read.  Returns 0 for invalid shapes as well. */
+size_t orthrus_block_attn_workspace(const orthrus_attn_args* a);
+
+int orthrus_block_attn(const orthrus_attn_args* a, orthrus_stream_t stream);
+
+/* Number of kernel launches one orthrus_block_attn call with these arguments
+ * issues (for launch accounting); 0 for invalid shapes or B == 0. */
+int orthrus_block_attn_launches(const orthrus_attn_args* a);
+
+/* ------------------------------------------------------------------------
+ * Vocab-row argmax (explainer §四: "the token that should most appear here").
+ * idx[r] = smallest j with logits[r*row_stride + j] == max_k logits[r*row_stride + k];
+ * NaN never wins; an all-NaN row gives 0; -0.0 and +0.0 are equal.
+ * maxval (nullable) receives the winning value as float (bf16 widened exactly).
+ * dtype: ORTHRUS_F32 or ORTHRUS_BF16; rows >= 0, vocab >= 1, row_stride >= vocab.
+ * ---------------------------------------------------------------------- */
+size_t orthrus_vocab_argmax_workspace(int32_t rows);
+
+int orthrus_vocab_argmax(int32_t dtype, const void* logits, int32_t rows,
+                         int32_t vocab, int64_t row_stride, int32_t* idx,
+                         float* maxval, void* workspace, size_t workspace_bytes,
+                         orthrus_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Prefix consensus (explainer §四 step 3), per sequence b:
+ *   accept_len[b]  = first j with draft[b,j] != verify[b,j], else blk
+ *   n_emit[b]      = min(accept_len[b] + 1, blk)        (always >= 1)
+ *   emitted[b,j]   = verify[b,j] for j < n_emit[b], else -1
+ *   next_anchor[b] = verify[b, n_emit[b] - 1]
+ * draft/verify [B, blk] int32 device; 1 <= blk <= 32.  Any output pointer
+ * except n_emit may be NULL.
+ * ---------------------------------------------------------------------- */
+int orthrus_consensus(const int32_t* draft, const int32_t* verify, int32_t B,
+                      int32_t blk, int32_t* accept_len, int32_t* n_emit,
+                      int32_t* emitted, int32_t* next_anchor,
+                      orthrus_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * KV commit / rollback for all layers in one launch (explainer §四 step 3
+ * "update the notebook"; §七: the block is the only extra state).  For every
+ * layer l, sequence b (n = ctx_lens[b], e = n_emit[b]) and kv-head g:
+ *   cache_l[b, g, n + r, :] = blk_l[b, r, g, :]   for r in [0, e)
+ * then ctx_lens[b] = n + e.  Rows r >= e are never written (that is the
+ * rollback); e == 0 changes nothing.  If n + e > cap or e is outside
+ * [0, blk], sequence b is skipped and `err` gets ORTHRUS_ECAPACITY.
+ * ---------------------------------------------------------------------- */
+typedef struct orthrus_commit_args {
+  int32_t dtype;   /* element type of caches and blocks */
+  int32_t layers;  /* >= 1 */
+  int32_t B, Hkv, D, blk, cap;
+  void* k_cache;   /* layer l at k_cache + l*cache_layer_stride: [B, Hkv, cap, D] */
+  void* v_cache;
+  int64_t cache_layer_stride; /* elements; >= B*Hkv*cap*D */
+  const void* k_blk; /* layer l at k_blk + l*blk_layer_stride: [B, blk, Hkv, D] */
+  const void* v_blk;
+  int64_t blk_layer_stride;   /* elements; >= B*blk*Hkv*D */
+  int32_t* ctx_lens;          /* [B] device, in/out */
+  const int32_t* n_emit;      /* [B] device */
+  int32_t* err;               /* optional device error word */
+  void* workspace;            /* zero-initialised, orthrus_kv_commit_workspace() bytes */
+  size_t workspace_bytes;
+} orthrus_commit_args;
+
+size_t orthrus_kv_commit_workspace(const orthrus_commit_args* a);
+
+int orthrus_kv_commit(const orthrus_commit_args* a, orthrus_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+const char* orthrus_status_str(int status);
+int orthrus_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ORTHRUS_H */

@@ -1,0 +1,142 @@
+"""CPU-only checks of the C ABI: the library loads, exports every function
+include/orthrus.h declares, the ctypes structs match the C layout, and
+host-side argument checks return their status codes without launching
+anything (no GPU is touched by these calls)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_attention_b200 as ba
+from block_attention_b200 import build as ba_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "orthrus.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    ba_build.build()
+    return ba.lib()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(orthrus_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert set(names) >= set(ba.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", ba.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L, n)
+
+
+def test_version_and_status_strings(L):
+    assert L.orthrus_version() == 10000
+    assert L.orthrus_status_str(0) == b"ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert L.orthrus_status_str(code) not in (b"ok", b"unknown status")
+
+
+def test_struct_layout_matches_c(tmp_path):
+    prog = tmp_path / "layout.c"
+    prog.write_text(r'''
+#include <stddef.h>
+#include <stdio.h>
+#include "orthrus.h"
+#define F(T, m) printf(#T " " #m " %zu\n", offsetof(T, m))
+int main(void) {
+  printf("orthrus_attn_args size %zu\n", sizeof(orthrus_attn_args));
+  F(orthrus_attn_args, scale); F(orthrus_attn_args, q); F(orthrus_attn_args, ctx_lens);
+  F(orthrus_attn_args, err); F(orthrus_attn_args, workspace_bytes);
+  printf("orthrus_commit_args size %zu\n", sizeof(orthrus_commit_args));
+  F(orthrus_commit_args, k_cache); F(orthrus_commit_args, cache_layer_stride);
+  F(orthrus_commit_args, blk_layer_stride); F(orthrus_commit_args, n_emit);
+  F(orthrus_commit_args, workspace_bytes);
+  return 0;
+}''')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)],
+                   check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines():
+        t, m, v = line.split()
+        got[(t, m)] = int(v)
+    cls = {"orthrus_attn_args": ba.AttnArgs, "orthrus_commit_args": ba.CommitArgs}
+    for (t, m), v in got.items():
+        c = cls[t]
+        assert (ctypes.sizeof(c) if m == "size" else getattr(c, m).offset) == v, (t, m)
+
+
+def _args(**kw):
+    base = dict(dtype=0, mask_mode=0, B=1, Hq=4, Hkv=2, D=64, blk=32, cap=300, max_ctx=256,
+                scale=0.125)
+    base.update(kw)
+    a = ba.AttnArgs()
+    for k, v in base.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), -1), (dict(mask_mode=2), -1), (dict(Hq=5), -1), (dict(blk=0), -1),
+    (dict(D=96), -2), (dict(blk=33), -2), (dict(Hq=16, Hkv=2, blk=32), -2),
+    (dict(max_ctx=301), -4), (dict(scale=float("inf")), -1),
+])
+def test_block_attn_rejects_bad_shapes_without_launch(L, kw, code):
+    a = _args(**kw)
+    assert L.orthrus_block_attn(ctypes.byref(a), None) == code
+    assert L.orthrus_block_attn_workspace(ctypes.byref(a)) == 0
+
+
+def test_block_attn_null_pointers_and_workspace(L):
+    a = _args()
+    assert L.orthrus_block_attn(ctypes.byref(a), None) == -1  # null tensors
+    for f in ("q", "k_blk", "v_blk", "k_cache", "v_cache", "out", "ctx_lens"):
+        setattr(a, f, 4096)  # aligned fake addresses: never dereferenced
+    need = L.orthrus_block_attn_workspace(ctypes.byref(a))
+    assert need > 0
+    assert L.orthrus_block_attn(ctypes.byref(a), None) == -3  # no workspace
+    a.workspace, a.workspace_bytes = 8192, need - 1
+    assert L.orthrus_block_attn(ctypes.byref(a), None) == -3
+    a.q = 4100  # misaligned
+    assert L.orthrus_block_attn(ctypes.byref(a), None) == -1
+    b = _args(B=0)
+    assert L.orthrus_block_attn(ctypes.byref(b), None) == 0  # nothing to do
+
+
+def test_argmax_consensus_commit_host_checks(L):
+    assert L.orthrus_vocab_argmax(0, None, 4, 0, 0, None, None, None, 0, None) == -1
+    assert L.orthrus_vocab_argmax(0, None, 4, 10, 5, None, None, None, 0, None) == -1
+    assert L.orthrus_vocab_argmax(3, None, 4, 10, 10, None, None, None, 0, None) == -1
+    assert L.orthrus_vocab_argmax(0, None, 0, 10, 10, None, None, None, 0, None) == 0
+    assert L.orthrus_vocab_argmax(0, 4096, 4, 10, 10, 4096, None, None, 0, None) == -3
+    assert L.orthrus_vocab_argmax_workspace(32) >= 32 * 12
+    assert L.orthrus_consensus(None, None, 1, 0, None, None, None, None, None) == -1
+    assert L.orthrus_consensus(None, None, 1, 33, None, None, None, None, None) == -2
+    assert L.orthrus_consensus(None, None, 0, 32, None, None, None, None, None) == 0
+    assert L.orthrus_consensus(None, None, 2, 32, None, None, None, None, None) == -1
+    c = ba.CommitArgs(dtype=1, layers=2, B=1, Hkv=8, D=128, blk=32, cap=100,
+                      cache_layer_stride=10, blk_layer_stride=10)
+    assert L.orthrus_kv_commit(ctypes.byref(c), None) == -1  # strides too small
+    c.cache_layer_stride, c.blk_layer_stride = 8 * 100 * 128, 32 * 8 * 128
+    for f in ("k_cache", "v_cache", "k_blk", "v_blk", "ctx_lens", "n_emit"):
+        setattr(c, f, 4096)
+    assert L.orthrus_kv_commit(ctypes.byref(c), None) == -3  # no workspace
+    assert L.orthrus_kv_commit_workspace(ctypes.byref(c)) >= 4
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(2, 8)
+    with pytest.raises(ValueError):
+        ba.vocab_argmax(x)
