@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "liborthrus.so")
 F32, BF16 = 0, 1
 BIDIR_BLOCK, CAUSAL_VERIFY = 0, 1
 STATUS = {0: "ok", -1: "EINVAL", -2: "EUNSUPPORTED", -3: "EWORKSPACE", -4: "ECAPACITY",
-          -5: "ECUDA"}
+          -5: "ECUDA", -6: "ETIMEOUT"}
 
 
 class OrthrusError(RuntimeError):

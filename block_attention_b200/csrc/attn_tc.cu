@@ -1,11 +1,550 @@
-// attn_tc.cu -- tensor-core block attention (bf16); not enabled yet.
+// attn_tc.cu -- bf16 block attention on the 5th-generation tensor cores.
+//
+// What it computes is the Orthrus round's attention (explainer on
+// arXiv:2605.12825, §二: the block's queries attend to the frozen AR model's
+// KV cache concatenated with the block's own K/V; §三: bidirectional inside
+// the block for the diffusion view, causal for the AR verify view).
+//
+// Shape of the work.  Decoding reads every cached K/V row once per layer and
+// view, so the kernel is bound by HBM bandwidth; the G = Hq/Hkv query heads
+// that share a kv-head and the blk block rows form one M = G*blk <= 128 row
+// tile, so each K/V tile fetched from HBM feeds a full 128-row tcgen05 MMA
+// (128 FLOP per KV byte at the Qwen3-8B shape -- beyond CUDA cores, so the
+// QK^T and PV products run on the tensor pipe).
+//
+// Grid: (S splits, Hkv, B) launched as clusters of S CTAs; one cluster covers
+// one (sequence, kv-head).  The keys cache[0, n) are cut into 64-key tiles,
+// followed by one tile holding the blk block rows; the tiles are dealt out
+// contiguously over the S CTAs (split-KV).  Each CTA:
+//   warp 0      TMA producer: Q once, then K/V tiles into a 4-stage ring
+//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered
+//               TMEM tile, then O += P V with P read from TMEM
+//   warps 2..5  softmax, one query row per thread: online softmax with lazy
+//               rescaling (O in TMEM is rescaled only when a row's running
+//               maximum grows by more than 2^8), P written back to TMEM as
+//               bf16; then the split combine.
+// Split combine: every CTA parks its unnormalised O, running max and sum in
+// its shared memory, the cluster synchronises, and CTA s reduces rows
+// [s*128/S, (s+1)*128/S) over the S splits through distributed shared memory,
+// in split order, and writes them out -- one launch, no global scratch.
+//
+// Every mbarrier wait is bounded: on a timeout the kernel records
+// ORTHRUS_ETIMEOUT in the error word, stops issuing work, drains what it
+// issued and still reaches the cluster barriers, so it always terminates.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
 #include "attn_tc.cuh"
+#include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace orthrus {
+namespace {
 
-bool tc_supported(const orthrus_attn_args&) { return false; }
+constexpr int kRows = 128;      // UMMA M
+constexpr int kTile = 64;       // keys per tile
+constexpr int kStages = 4;      // K/V ring depth
+constexpr int kThreads = 192;   // 6 warps
+constexpr int kTmemCols = 256;  // S0 [0,64) S1 [64,128) O [128,256)
+constexpr int kOCol = 128;
+constexpr float kLazyThresh = 8.f;  // log2 units
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int kQBytes = 2 * kRows * 128;        // two 64-dim halves, 128 B rows
+constexpr int kHalfTile = kTile * 128;          // one 64-dim half of a K or V tile
+constexpr int kStageBytes = 4 * kHalfTile;      // K (2 halves) + V (2 halves)
+constexpr int kRingOff = kQBytes;
+constexpr int kBarOff = kRingOff + kStages * kStageBytes;
+constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+constexpr int kMiscOff = kBarOff + kNumBars * 8;
+constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
+// combine staging (aliases the ring once every MMA has finished)
+constexpr int kStageStride = 128 + 4;  // floats per O row (bank-conflict-free float4 stores)
+constexpr int kStageO = kRingOff;
+constexpr int kStageM = kStageO + kRows * kStageStride * 4;
+constexpr int kStageL = kStageM + kRows * 4;
+static_assert(kStageL + kRows * 4 <= kBarOff, "staging must fit in the ring");
+
+struct __align__(64) TcParams {
+  CUtensorMap tm_q;   // 3D (D, Hq, B*blk), box (64, G, blk)
+  CUtensorMap tm_kc;  // 2D (D, B*Hkv*cap), box (64, 64)
+  CUtensorMap tm_vc;
+  CUtensorMap tm_kb;  // 3D (D, Hkv, B*blk), box (64, 1, blk)
+  CUtensorMap tm_vb;
+  const int32_t* ctx_lens;
+  __nv_bfloat16* out;
+  int32_t* err;
+  int B, Hq, Hkv, D, blk, cap, max_ctx, mask_mode, G, S;
+  float scale_log2;
+};
+
+struct Bars {
+  uint32_t q_full, full[kStages], empty[kStages], s_full[2], p_full[2], pv_done[2], mma_done;
+};
+
+__device__ __forceinline__ void record_timeout(const TcParams& p, volatile int* abort_flag) {
+  *abort_flag = 1;
+  set_err(p.err, ORTHRUS_ETIMEOUT);
+}
+
+template <int kD>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr int halves = kD / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const uint32_t rank = ptx::cluster_rank();
+  const int S = p.S;
+
+  Bars bars;
+  {
+    uint32_t a = sbase + kBarOff;
+    bars.q_full = a; a += 8;
+    for (int s = 0; s < kStages; ++s) { bars.full[s] = a; a += 8; }
+    for (int s = 0; s < kStages; ++s) { bars.empty[s] = a; a += 8; }
+    for (int s = 0; s < 2; ++s) { bars.s_full[s] = a; a += 8; }
+    for (int s = 0; s < 2; ++s) { bars.p_full[s] = a; a += 8; }
+    for (int s = 0; s < 2; ++s) { bars.pv_done[s] = a; a += 8; }
+    bars.mma_done = a;
+  }
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 8);
+
+  // ---- sequence geometry (every CTA of the cluster reads the same n)
+  const int n = p.ctx_lens[b];
+  const bool bad = n < 0 || n > p.max_ctx;
+  const int Tc = bad ? 0 : ceil_div(n, kTile);  // cache tiles
+  const int T = bad ? 0 : Tc + 1;               // + the block tile
+  const int t0 = (int)(((int64_t)rank * T) / S);
+  const int t1 = (int)(((int64_t)(rank + 1) * T) / S);
+  const int U = t1 - t0;
+  const int rows = p.G * p.blk;
+
+  // ---- setup: barriers, TMEM, zero the Q padding rows
+  if (threadIdx.x == 0) {
+    if (bad && rank == 0 && g == 0) set_err(p.err, ORTHRUS_ECAPACITY);
+    *abort_flag = 0;
+    ptx::mbar_init(bars.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(bars.full[s], 1);
+      ptx::mbar_init(bars.empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(bars.s_full[s], 1);
+      ptx::mbar_init(bars.p_full[s], 128);
+      ptx::mbar_init(bars.pv_done[s], 1);
+    }
+    ptx::mbar_init(bars.mma_done, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::tma_prefetch_desc(&p.tm_q);
+    ptx::tma_prefetch_desc(&p.tm_kc);
+    ptx::tma_prefetch_desc(&p.tm_vc);
+    ptx::tma_prefetch_desc(&p.tm_kb);
+    ptx::tma_prefetch_desc(&p.tm_vb);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  for (int e = threadIdx.x; e < (kRows - rows) * 8 * halves; e += kThreads) {
+    const int h = e / ((kRows - rows) * 8), rem = e % ((kRows - rows) * 8);
+    const int r = rows + rem / 8, c = rem % 8;
+    *reinterpret_cast<uint4*>(smem + h * (kRows * 128) + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+  }
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const uint32_t q_s = sbase;
+  auto k_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes; };
+  auto v_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes + 2 * kHalfTile; };
+
+  if (warp == 0) {
+    // ================================================== TMA producer
+    if (lane == 0 && U > 0) {
+      int issued = 0;
+      ptx::mbar_expect_tx(bars.q_full, (uint32_t)(halves * rows * 128));
+      for (int h = 0; h < halves; ++h)
+        ptx::tma_load_3d(q_s + h * (kRows * 128), &p.tm_q, bars.q_full, 64 * h, g * p.G,
+                         b * p.blk);
+      const int slab = (b * p.Hkv + g) * p.cap;
+      for (int u = 0; u < U && !*abort_flag; ++u) {
+        const int t = t0 + u, st = u % kStages;
+        if (!ptx::mbar_wait(bars.empty[st], ((u / kStages) & 1) ^ 1)) {
+          record_timeout(p, abort_flag);
+          break;
+        }
+        const bool blk_tile = t == Tc;
+        const int rows_ld = blk_tile ? p.blk : kTile;
+        ptx::mbar_expect_tx(bars.full[st], (uint32_t)(2 * halves * rows_ld * 128));
+        for (int h = 0; h < halves; ++h) {
+          if (blk_tile) {
+            ptx::tma_load_3d(k_s(st) + h * kHalfTile, &p.tm_kb, bars.full[st], 64 * h, g,
+                             b * p.blk);
+            ptx::tma_load_3d(v_s(st) + h * kHalfTile, &p.tm_vb, bars.full[st], 64 * h, g,
+                             b * p.blk);
+          } else {
+            ptx::tma_load_2d(k_s(st) + h * kHalfTile, &p.tm_kc, bars.full[st], 64 * h,
+                             slab + t * kTile);
+            ptx::tma_load_2d(v_s(st) + h * kHalfTile, &p.tm_vc, bars.full[st], 64 * h,
+                             slab + t * kTile);
+          }
+        }
+        issued = u + 1;
+      }
+      // drain: the last (up to) kStages loads must have landed before exit
+      for (int u = max(0, issued - kStages); u < issued; ++u)
+        if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1)) record_timeout(p, abort_flag);
+      if (!ptx::mbar_wait(bars.q_full, 0)) record_timeout(p, abort_flag);
+    }
+  } else if (warp == 1) {
+    // ================================================== MMA issuer
+    if (lane == 0 && U > 0) {
+      const uint32_t id_s = ptx::idesc_bf16(kRows, kTile, false, false);
+      const uint32_t id_pv = ptx::idesc_bf16(kRows, kD, false, true);
+      bool ok = ptx::mbar_wait(bars.q_full, 0);
+      auto pv = [&](int u) -> bool {
+        const int buf = u & 1, st = u % kStages;
+        if (!ptx::mbar_wait(bars.p_full[buf], (u >> 1) & 1)) return false;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k) {
+          const uint64_t bd = ptx::sdesc_sw128(v_s(st) + k * 2048, kHalfTile, 1024);
+          ptx::mma_ts(tmem + kOCol, tmem + buf * 64 + k * 8, bd, id_pv, (u > 0 || k > 0) ? 1u : 0u);
+        }
+        ptx::tc_commit(bars.pv_done[buf]);
+        ptx::tc_commit(bars.empty[st]);
+        return true;
+      };
+      for (int u = 0; ok && u < U && !*abort_flag; ++u) {
+        const int buf = u & 1, st = u % kStages;
+        if (!ptx::mbar_wait(bars.full[st], (u / kStages) & 1)) { ok = false; break; }
+        if (u >= 2 && !ptx::mbar_wait(bars.pv_done[buf], ((u - 2) >> 1) & 1)) { ok = false; break; }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k) {
+          const uint32_t h = k >> 2, kk = k & 3;  // 64-dim half, 16-dim step in it
+          const uint64_t ad = ptx::sdesc_sw128(q_s + h * (kRows * 128) + kk * 32, 16, 1024);
+          const uint64_t bd = ptx::sdesc_sw128(k_s(st) + h * kHalfTile + kk * 32, 16, 1024);
+          ptx::mma_ss(tmem + buf * 64, ad, bd, id_s, k > 0 ? 1u : 0u);
+        }
+        ptx::tc_commit(bars.s_full[buf]);
+        if (u >= 1 && !pv(u - 1)) { ok = false; break; }
+      }
+      if (ok && !*abort_flag) ok = pv(U - 1);
+      if (!ok) record_timeout(p, abort_flag);
+      // every MMA issued so far has finished before TMEM is released
+      ptx::tc_commit(bars.mma_done);
+      if (!ptx::mbar_wait(bars.mma_done, 0)) record_timeout(p, abort_flag);
+    }
+  } else {
+    // ================================================== softmax + epilogue
+    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;            // query row of this thread
+    const int i_blk = r < rows ? r / p.G : p.blk;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int sm_tid = threadIdx.x - 64;       // 0..127
+    float m_ref = -INFINITY, l = 0.f;
+    bool alive = true;
+    const unsigned full = 0xffffffffu;
+    for (int u = 0; u < U; ++u) {
+      if (__any_sync(full, *abort_flag != 0)) { alive = false; break; }
+      const int t = t0 + u, buf = u & 1, st = u % kStages;
+      if (!__all_sync(full, ptx::mbar_wait(bars.s_full[buf], (u >> 1) & 1))) {
+        record_timeout(p, abort_flag); alive = false; break;
+      }
+      ptx::tc_fence_after();
+      uint32_t sa[32], sb[32];
+      ptx::tmem_ld32(lane_addr + buf * 64, sa);
+      ptx::tmem_ld32(lane_addr + buf * 64 + 32, sb);
+      ptx::tmem_wait_ld();
+      const bool blk_tile = t == Tc;
+      const int nv_tile = blk_tile ? p.blk : min(kTile, n - t * kTile);
+      int nv = nv_tile;
+      if (blk_tile && p.mask_mode == ORTHRUS_CAUSAL_VERIFY) nv = min(i_blk + 1, p.blk);
+      float mt = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < nv) mt = fmaxf(mt, __uint_as_float(sa[j]));
+        if (j + 32 < nv) mt = fmaxf(mt, __uint_as_float(sb[j]));
+      }
+      const float ms = mt * p.scale_log2;
+      const bool need = ms > m_ref + kLazyThresh;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? ms : m_ref;
+        const float f = ptx::ex2(m_ref - m_new);  // 0 for the first tile, 1 if unchanged
+        if (u > 0) {
+          if (!__all_sync(full, ptx::mbar_wait(bars.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1))) {
+            record_timeout(p, abort_flag); alive = false; break;
+          }
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int cb = 0; cb < kD / 32; ++cb) {
+            uint32_t o[32];
+            ptx::tmem_ld32(lane_addr + kOCol + cb * 32, o);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+            ptx::tmem_st32(lane_addr + kOCol + cb * 32, o);
+          }
+          ptx::tmem_wait_st();
+        }
+        l *= f;
+        m_ref = m_new;
+      }
+      // P = 2^(s*c - m_ref) as bf16 pairs; the row sum uses the rounded values
+      uint32_t pk[32];
+      float lsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float p0 = (2 * j < nv) ? ptx::ex2(__uint_as_float(sa[2 * j]) * p.scale_log2 - m_ref) : 0.f;
+        const float p1 = (2 * j + 1 < nv) ? ptx::ex2(__uint_as_float(sa[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
+        pk[j] = ptx::pack_bf16x2(p0, p1);
+        lsum += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float p0 = (2 * j + 32 < nv) ? ptx::ex2(__uint_as_float(sb[2 * j]) * p.scale_log2 - m_ref) : 0.f;
+        const float p1 = (2 * j + 33 < nv) ? ptx::ex2(__uint_as_float(sb[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
+        pk[16 + j] = ptx::pack_bf16x2(p0, p1);
+        lsum += __uint_as_float(pk[16 + j] << 16) + __uint_as_float(pk[16 + j] & 0xffff0000u);
+      }
+      l += lsum;
+      ptx::tmem_st32(lane_addr + buf * 64, pk);
+      ptx::tmem_wait_st();
+      if (nv_tile < kTile) {
+        // rows past the valid keys hold stale or foreign data: zero them in V
+        // so 0 * garbage cannot reach O
+        if (!__all_sync(full, ptx::mbar_wait(bars.full[st], (u / kStages) & 1))) {
+          record_timeout(p, abort_flag); alive = false; break;
+        }
+        const int nz = (kTile - nv_tile) * 8 * halves;  // 16-byte chunks
+        for (int e = sm_tid; e < nz; e += 128) {
+          const int h = e / ((kTile - nv_tile) * 8), rem = e % ((kTile - nv_tile) * 8);
+          const int row = nv_tile + rem / 8, c = rem % 8;
+          *reinterpret_cast<uint4*>(smem + kRingOff + st * kStageBytes + 2 * kHalfTile +
+                                    h * kHalfTile + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+        ptx::fence_proxy_async_smem();
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bars.p_full[buf]);
+    }
+    // ---- epilogue: park this split's (O, m, l) in shared memory
+    float* stO = reinterpret_cast<float*>(smem + kStageO);
+    float* stM = reinterpret_cast<float*>(smem + kStageM);
+    float* stL = reinterpret_cast<float*>(smem + kStageL);
+    uint32_t o[kD / 32][32];
+    bool have = alive && U > 0 && !__any_sync(full, *abort_flag != 0);
+    if (have) {
+      if (!__all_sync(full, ptx::mbar_wait(bars.pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1))) {
+        record_timeout(p, abort_flag);
+        have = false;
+      } else {
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int cb = 0; cb < kD / 32; ++cb) ptx::tmem_ld32(lane_addr + kOCol + cb * 32, o[cb]);
+        ptx::tmem_wait_ld();
+      }
+    }
+    ptx::named_bar_sync(1, 128);  // all softmax threads are done with the ring
+    const bool have2 = have && *abort_flag == 0;
+#pragma unroll
+    for (int cb = 0; cb < kD / 32; ++cb)
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(stO + r * kStageStride + cb * 32 + j) =
+            have2 ? make_float4(__uint_as_float(o[cb][j]), __uint_as_float(o[cb][j + 1]),
+                                __uint_as_float(o[cb][j + 2]), __uint_as_float(o[cb][j + 3]))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    stM[r] = have2 ? m_ref : -INFINITY;
+    stL[r] = have2 ? l : 0.f;
+  }
+  __syncwarp();
+  ptx::tc_fence_before();
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+
+  // ---- split combine through distributed shared memory
+  if (warp >= 2) {
+    const int sm_tid = threadIdx.x - 64;
+    const int R = kRows / S;
+    const int per_row = kD / 4;
+    bool any_abort = false;
+    for (int s = 0; s < S; ++s)
+      any_abort |= ptx::ld_cluster_s32(ptx::map_rank(sbase + kMiscOff + 8, s)) != 0;
+    for (int it = sm_tid; it < R * per_row && !bad && !any_abort; it += 128) {
+      const int rr = (int)rank * R + it / per_row;
+      const int d4 = (it % per_row) * 4;
+      if (rr >= rows) continue;
+      float M = -INFINITY;
+      for (int s = 0; s < S; ++s)
+        M = fmaxf(M, ptx::ld_cluster_f32(ptx::map_rank(sbase + kStageM + rr * 4, s)));
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < S; ++s) {
+        const float ms = ptx::ld_cluster_f32(ptx::map_rank(sbase + kStageM + rr * 4, s));
+        const float w = ptx::ex2(ms - M);
+        const float ls = ptx::ld_cluster_f32(ptx::map_rank(sbase + kStageL + rr * 4, s));
+        const float4 os = ptx::ld_cluster_f32x4(
+            ptx::map_rank(sbase + kStageO + (rr * kStageStride + d4) * 4, s));
+        L = fmaf(w, ls, L);
+        O.x = fmaf(w, os.x, O.x);
+        O.y = fmaf(w, os.y, O.y);
+        O.z = fmaf(w, os.z, O.z);
+        O.w = fmaf(w, os.w, O.w);
+      }
+      const float inv = 1.f / L;
+      const int i = rr / p.G, h = g * p.G + rr % p.G;
+      uint2 pkd;
+      pkd.x = ptx::pack_bf16x2(O.x * inv, O.y * inv);
+      pkd.y = ptx::pack_bf16x2(O.z * inv, O.w * inv);
+      *reinterpret_cast<uint2*>(p.out + ((int64_t)(b * p.blk + i) * p.Hq + h) * kD + d4) = pkd;
+    }
+  }
+  __syncwarp();
+  ptx::tc_fence_before();
+  ptx::cluster_sync();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+            strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Largest supported cluster size whose clusters can be resident (16, else 8).
+template <int kD>
+int cluster_size(int device) {
+  static int cached[64] = {0};
+  if (device >= 0 && device < 64 && cached[device]) return cached[device];
+  int best = 0;
+  if (cudaFuncSetAttribute(attn_tc_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes) != cudaSuccess)
+    return 0;
+  cudaFuncSetAttribute(attn_tc_kernel<kD>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  for (int s : {16, 8}) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(s, 8, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = s;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, attn_tc_kernel<kD>, &cfg) == cudaSuccess &&
+        nclusters > 0) {
+      best = s;
+      break;
+    }
+    cudaGetLastError();
+  }
+  if (device >= 0 && device < 64) cached[device] = best;
+  return best;
+}
+
+}  // namespace
+
+bool tc_supported(const orthrus_attn_args& a) {
+  return a.dtype == ORTHRUS_BF16 && (a.D == 64 || a.D == 128) &&
+         (a.Hq / a.Hkv) * a.blk <= kRows && a.blk <= 32 && a.Hq / a.Hkv <= 256;
+}
+
 size_t tc_workspace_bytes(const orthrus_attn_args&) { return 0; }
-int tc_launch(const orthrus_attn_args&, cudaStream_t) { return ORTHRUS_EUNSUPPORTED; }
+
 int tc_launches(const orthrus_attn_args&) { return 1; }
+
+int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ECUDA;
+  const int S = a.D == 64 ? cluster_size<64>(dev) : cluster_size<128>(dev);
+  if (S == 0) return ORTHRUS_ECUDA;
+  TcParams p;
+  const int G = a.Hq / a.Hkv;
+  const cuuint64_t es = 2;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)a.D, (cuuint64_t)a.Hq, (cuuint64_t)a.B * a.blk};
+    cuuint64_t str[2] = {a.D * es, (cuuint64_t)a.Hq * a.D * es};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)a.blk};
+    if (!encode(&p.tm_q, a.q, 3, dims, str, box)) return ORTHRUS_ECUDA;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)a.D, (cuuint64_t)a.B * a.Hkv * a.cap};
+    cuuint64_t str[1] = {a.D * es};
+    cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    if (!encode(&p.tm_kc, a.k_cache, 2, dims, str, box)) return ORTHRUS_ECUDA;
+    if (!encode(&p.tm_vc, a.v_cache, 2, dims, str, box)) return ORTHRUS_ECUDA;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)a.D, (cuuint64_t)a.Hkv, (cuuint64_t)a.B * a.blk};
+    cuuint64_t str[2] = {a.D * es, (cuuint64_t)a.Hkv * a.D * es};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)a.blk};
+    if (!encode(&p.tm_kb, a.k_blk, 3, dims, str, box)) return ORTHRUS_ECUDA;
+    if (!encode(&p.tm_vb, a.v_blk, 3, dims, str, box)) return ORTHRUS_ECUDA;
+  }
+  p.ctx_lens = a.ctx_lens;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.err = a.err;
+  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.blk = a.blk; p.cap = a.cap;
+  p.max_ctx = a.max_ctx; p.mask_mode = a.mask_mode; p.G = G; p.S = S;
+  p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, a.Hkv, a.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_kernel<64>, p)
+                                  : cudaLaunchKernelEx(&cfg, attn_tc_kernel<128>, p);
+  if (e != cudaSuccess) return ORTHRUS_ECUDA;
+  return ORTHRUS_OK;
+}
 
 }  // namespace orthrus

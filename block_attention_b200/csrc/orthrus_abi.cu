@@ -62,6 +62,7 @@ const char* orthrus_status_str(int s) {
     case ORTHRUS_EWORKSPACE: return "workspace missing or too small";
     case ORTHRUS_ECAPACITY: return "length exceeds cache capacity";
     case ORTHRUS_ECUDA: return "CUDA launch failed";
+    case ORTHRUS_ETIMEOUT: return "bounded device wait timed out";
     default: return "unknown status";
   }
 }

@@ -52,7 +52,9 @@ typedef enum {
   ORTHRUS_EUNSUPPORTED = -2, /* valid but not implemented (D, G*blk, ...) */
   ORTHRUS_EWORKSPACE = -3,   /* workspace missing or too small */
   ORTHRUS_ECAPACITY = -4,    /* a length exceeds the cache capacity */
-  ORTHRUS_ECUDA = -5         /* a CUDA launch or attribute call failed */
+  ORTHRUS_ECUDA = -5,        /* a CUDA launch or attribute call failed */
+  ORTHRUS_ETIMEOUT = -6      /* device error word only: a bounded wait inside a
+                                kernel gave up; that call's outputs are not valid */
 } orthrus_status;
 
 typedef enum { ORTHRUS_F32 = 0, ORTHRUS_BF16 = 1 } orthrus_dtype;
