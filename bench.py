@@ -166,6 +166,50 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- one kernel alone
+
+def kernel_alone(args):
+    """Block attention alone at the Qwen3-8B layer shape, B=8 sequences of
+    context 8192 (269 MB of K/V, over twice the L2), bidirectional view:
+    W warm-up launches, then K launches captured in one CUDA graph."""
+    import torch
+    import block_attention_b200 as ba
+    from block_attention_b200.round import _dev
+    from block_attention_b200 import synth
+    w = WORKLOAD
+    B, ctx = 8, w["ctx"]
+    cap = ctx + w["blk"]
+    dev = torch.device("cuda", 0)
+    inp = synth.attn_inputs(B, w["Hq"], w["Hkv"], w["D"], w["blk"], [ctx] * B, cap, "bf16",
+                            seed=11)
+    t = {k: _dev(v, dev) for k, v in inp.items()}
+    out = torch.empty_like(t["q"])
+    call = lambda: ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                                 t["ctx_lens"], ba.BIDIR_BLOCK, out=out, max_ctx=ctx)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(args.steps):
+            call()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    nbytes = 2 * B * ctx * w["Hkv"] * w["D"] * 2 + 2 * B * w["blk"] * w["Hq"] * w["D"] * 2 \
+        + 2 * B * w["blk"] * w["Hkv"] * w["D"] * 2
+    hbm, src = peaks()
+    print(json.dumps({"kernel": "block_attn", "case": f"B={B} ctx={ctx} Hq=32 Hkv=8 D=128 blk=32 bf16 bidir",
+                      "us_per_launch": us, "bytes_per_launch": nbytes,
+                      "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / hbm,
+                      "peak": hbm, "peak_source": src}), flush=True)
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def main():
@@ -175,8 +219,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["attn"], default=None,
+                    help="time one kernel alone on a case larger than L2 (for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.kernel:
+        return kernel_alone(args)
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

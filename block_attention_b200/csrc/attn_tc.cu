@@ -16,21 +16,25 @@
 // one (sequence, kv-head).  The keys cache[0, n) are cut into 64-key tiles,
 // followed by one tile holding the blk block rows; the tiles are dealt out
 // contiguously over the S CTAs (split-KV).  Each CTA:
-//   warp 0      TMA producer: Q once, then K/V tiles into a 4-stage ring
+//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
 //   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered
 //               TMEM tile, then O += P V with P read from TMEM
 //   warps 2..5  softmax, one query row per thread: online softmax with lazy
 //               rescaling (O in TMEM is rescaled only when a row's running
 //               maximum grows by more than 2^8), P written back to TMEM as
 //               bf16; then the split combine.
-// Split combine: every CTA parks its unnormalised O, running max and sum in
-// its shared memory, the cluster synchronises, and CTA s reduces rows
-// [s*128/S, (s+1)*128/S) over the S splits through distributed shared memory,
-// in split order, and writes them out -- one launch, no global scratch.
+// A CTA needs ~97 KB of shared memory and 256 TMEM columns, so two fit on an
+// SM: every cluster of a launch is resident at once, and under programmatic
+// dependent launch the next kernel's CTAs can start while this one drains.
+//
+// Split combine: each CTA writes its unnormalised O (fp32) with its row maxima
+// and sums to an L2-resident workspace, the cluster synchronises, and CTA s
+// reduces rows [s*128/S, (s+1)*128/S) over the S splits in split order
+// (deterministic) and writes them out -- one launch.
 //
 // Every mbarrier wait is bounded: on a timeout the kernel records
 // ORTHRUS_ETIMEOUT in the error word, stops issuing work, drains what it
-// issued and still reaches the cluster barriers, so it always terminates.
+// issued and still reaches the cluster barrier, so it always terminates.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -44,29 +48,28 @@
 namespace orthrus {
 namespace {
 
-constexpr int kRows = 128;      // UMMA M
-constexpr int kTile = 64;       // keys per tile
-constexpr int kStages = 4;      // K/V ring depth
-constexpr int kThreads = 192;   // 6 warps
-constexpr int kTmemCols = 256;  // S0 [0,64) S1 [64,128) O [128,256)
+constexpr int kRows = 128;          // UMMA M
+constexpr int kTile = 64;           // keys per tile
+constexpr int kStages = 2;          // K/V ring depth
+constexpr int kThreads = 192;       // 6 warps
+constexpr int kTmemCols = 256;      // S0 [0,64) S1 [64,128) O [128,256)
 constexpr int kOCol = 128;
 constexpr float kLazyThresh = 8.f;  // log2 units
+constexpr int kMaxSplits = 16;      // largest cluster (non-portable size)
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kQBytes = 2 * kRows * 128;        // two 64-dim halves, 128 B rows
-constexpr int kHalfTile = kTile * 128;          // one 64-dim half of a K or V tile
-constexpr int kStageBytes = 4 * kHalfTile;      // K (2 halves) + V (2 halves)
+constexpr int kHalfTile = kTile * 128;      // one 64-dim half of a K or V tile
+constexpr int kQBytes = 2 * kRows * 128;    // two 64-dim halves, 128 B rows
+constexpr int kStageBytes = 4 * kHalfTile;  // K (2 halves) + V (2 halves)
 constexpr int kRingOff = kQBytes;
 constexpr int kBarOff = kRingOff + kStages * kStageBytes;
 constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
-constexpr int kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
-// combine staging (aliases the ring once every MMA has finished)
-constexpr int kStageStride = 128 + 4;  // floats per O row (bank-conflict-free float4 stores)
-constexpr int kStageO = kRingOff;
-constexpr int kStageM = kStageO + kRows * kStageStride * 4;
-constexpr int kStageL = kStageM + kRows * 4;
-static_assert(kStageL + kRows * 4 <= kBarOff, "staging must fit in the ring");
+constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+
+// workspace per (b, g, split): O as [D/4][128 rows] float4, then m[128], l[128]
+template <int kD>
+__host__ __device__ constexpr int part_floats() { return kRows * kD + 2 * kRows; }
 
 struct __align__(64) TcParams {
   CUtensorMap tm_q;   // 3D (D, Hq, B*blk), box (64, G, blk)
@@ -77,7 +80,8 @@ struct __align__(64) TcParams {
   const int32_t* ctx_lens;
   __nv_bfloat16* out;
   int32_t* err;
-  int B, Hq, Hkv, D, blk, cap, max_ctx, mask_mode, G, S;
+  float* part;  // split partials
+  int B, Hq, Hkv, blk, cap, max_ctx, mask_mode, G, S;
   float scale_log2;
 };
 
@@ -91,7 +95,7 @@ __device__ __forceinline__ void record_timeout(const TcParams& p, volatile int* 
 }
 
 template <int kD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr int halves = kD / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -102,6 +106,7 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   const int g = blockIdx.y, b = blockIdx.z;
   const uint32_t rank = ptx::cluster_rank();
   const int S = p.S;
+  const unsigned full_mask = 0xffffffffu;
 
   Bars bars;
   {
@@ -116,20 +121,10 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   }
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 8);
-
-  // ---- sequence geometry (every CTA of the cluster reads the same n)
-  const int n = p.ctx_lens[b];
-  const bool bad = n < 0 || n > p.max_ctx;
-  const int Tc = bad ? 0 : ceil_div(n, kTile);  // cache tiles
-  const int T = bad ? 0 : Tc + 1;               // + the block tile
-  const int t0 = (int)(((int64_t)rank * T) / S);
-  const int t1 = (int)(((int64_t)(rank + 1) * T) / S);
-  const int U = t1 - t0;
   const int rows = p.G * p.blk;
 
-  // ---- setup: barriers, TMEM, zero the Q padding rows
+  // ---- setup that reads nothing a preceding kernel writes
   if (threadIdx.x == 0) {
-    if (bad && rank == 0 && g == 0) set_err(p.err, ORTHRUS_ECAPACITY);
     *abort_flag = 0;
     ptx::mbar_init(bars.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -165,10 +160,25 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // Programmatic dependent launch: the next kernel in the stream may start
+  // its own setup now; everything below may read what earlier kernels wrote.
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
+
+  // ---- sequence geometry (every CTA of the cluster reads the same n)
+  const int n = p.ctx_lens[b];
+  const bool bad = n < 0 || n > p.max_ctx;
+  if (bad && rank == 0 && g == 0 && threadIdx.x == 0) set_err(p.err, ORTHRUS_ECAPACITY);
+  const int Tc = bad ? 0 : ceil_div(n, kTile);  // cache tiles
+  const int T = bad ? 0 : Tc + 1;               // + the block tile
+  const int t0 = (int)(((int64_t)rank * T) / S);
+  const int t1 = (int)(((int64_t)(rank + 1) * T) / S);
+  const int U = t1 - t0;
 
   const uint32_t q_s = sbase;
   auto k_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes; };
   auto v_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes + 2 * kHalfTile; };
+  float* part = p.part + ((int64_t)(b * p.Hkv + g) * S + rank) * part_floats<kD>();
 
   if (warp == 0) {
     // ================================================== TMA producer
@@ -203,7 +213,7 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
         }
         issued = u + 1;
       }
-      // drain: the last (up to) kStages loads must have landed before exit
+      // drain: every issued load must have landed before the CTA exits
       for (int u = max(0, issued - kStages); u < issued; ++u)
         if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1)) record_timeout(p, abort_flag);
       if (!ptx::mbar_wait(bars.q_full, 0)) record_timeout(p, abort_flag);
@@ -220,8 +230,11 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
         ptx::tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
+          // V tile as the MN-major B operand: 8-key groups 1024 B apart,
+          // 64-dim halves kHalfTile apart
           const uint64_t bd = ptx::sdesc_sw128(v_s(st) + k * 2048, kHalfTile, 1024);
-          ptx::mma_ts(tmem + kOCol, tmem + buf * 64 + k * 8, bd, id_pv, (u > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_ts(tmem + kOCol, tmem + buf * 64 + k * 8, bd, id_pv,
+                      (u > 0 || k > 0) ? 1u : 0u);
         }
         ptx::tc_commit(bars.pv_done[buf]);
         ptx::tc_commit(bars.empty[st]);
@@ -249,51 +262,57 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       if (!ptx::mbar_wait(bars.mma_done, 0)) record_timeout(p, abort_flag);
     }
   } else {
-    // ================================================== softmax + epilogue
-    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-    const int r = quad * 32 + lane;            // query row of this thread
+    // ================================================== softmax + partial
+    const int quad = warp & 3;            // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;       // query row of this thread
     const int i_blk = r < rows ? r / p.G : p.blk;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const int sm_tid = threadIdx.x - 64;       // 0..127
+    const int sm_tid = threadIdx.x - 64;  // 0..127
+    const float c = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool alive = true;
-    const unsigned full = 0xffffffffu;
     for (int u = 0; u < U; ++u) {
-      if (__any_sync(full, *abort_flag != 0)) { alive = false; break; }
+      if (__any_sync(full_mask, *abort_flag != 0)) { alive = false; break; }
       const int t = t0 + u, buf = u & 1, st = u % kStages;
-      if (!__all_sync(full, ptx::mbar_wait(bars.s_full[buf], (u >> 1) & 1))) {
+      if (!__all_sync(full_mask, ptx::mbar_wait(bars.s_full[buf], (u >> 1) & 1))) {
         record_timeout(p, abort_flag); alive = false; break;
       }
       ptx::tc_fence_after();
       uint32_t sa[32], sb[32];
-      ptx::tmem_ld32(lane_addr + buf * 64, sa);
-      ptx::tmem_ld32(lane_addr + buf * 64 + 32, sb);
-      ptx::tmem_wait_ld();
+      ptx::tmem_ld32_sync(lane_addr + buf * 64, sa);
+      ptx::tmem_ld32_sync(lane_addr + buf * 64 + 32, sb);
       const bool blk_tile = t == Tc;
       const int nv_tile = blk_tile ? p.blk : min(kTile, n - t * kTile);
       int nv = nv_tile;
       if (blk_tile && p.mask_mode == ORTHRUS_CAUSAL_VERIFY) nv = min(i_blk + 1, p.blk);
-      float mt = -INFINITY;
+      // masked keys -> -inf before the max and the exponent (exactly 0 in P)
+      if (nv < kTile) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j >= nv) sa[j] = __float_as_uint(-INFINITY);
+          if (j + 32 >= nv) sb[j] = __float_as_uint(-INFINITY);
+        }
+      }
+      float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        if (j < nv) mt = fmaxf(mt, __uint_as_float(sa[j]));
-        if (j + 32 < nv) mt = fmaxf(mt, __uint_as_float(sb[j]));
+        mt0 = fmaxf(mt0, __uint_as_float(sa[j]));
+        mt1 = fmaxf(mt1, __uint_as_float(sb[j]));
       }
-      const float ms = mt * p.scale_log2;
+      const float ms = fmaxf(mt0, mt1) * c;
       const bool need = ms > m_ref + kLazyThresh;
-      if (__any_sync(0xffffffffu, need)) {
+      if (__any_sync(full_mask, need)) {
         const float m_new = need ? ms : m_ref;
         const float f = ptx::ex2(m_ref - m_new);  // 0 for the first tile, 1 if unchanged
         if (u > 0) {
-          if (!__all_sync(full, ptx::mbar_wait(bars.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1))) {
+          if (!__all_sync(full_mask, ptx::mbar_wait(bars.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1))) {
             record_timeout(p, abort_flag); alive = false; break;
           }
           ptx::tc_fence_after();
 #pragma unroll
           for (int cb = 0; cb < kD / 32; ++cb) {
             uint32_t o[32];
-            ptx::tmem_ld32(lane_addr + kOCol + cb * 32, o);
-            ptx::tmem_wait_ld();
+            ptx::tmem_ld32_sync(lane_addr + kOCol + cb * 32, o);
 #pragma unroll
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
             ptx::tmem_st32(lane_addr + kOCol + cb * 32, o);
@@ -303,108 +322,106 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
         l *= f;
         m_ref = m_new;
       }
-      // P = 2^(s*c - m_ref) as bf16 pairs; the row sum uses the rounded values
+      // P = 2^(s*c - m_ref) as bf16 pairs into the first 32 columns of this S
+      // buffer; ex2(-inf) = 0 for masked keys
+      const float nm = -m_ref;
       uint32_t pk[32];
-      float lsum = 0.f;
+      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float p0 = (2 * j < nv) ? ptx::ex2(__uint_as_float(sa[2 * j]) * p.scale_log2 - m_ref) : 0.f;
-        const float p1 = (2 * j + 1 < nv) ? ptx::ex2(__uint_as_float(sa[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
+        const float p0 = ptx::ex2(fmaf(__uint_as_float(sa[2 * j]), c, nm));
+        const float p1 = ptx::ex2(fmaf(__uint_as_float(sa[2 * j + 1]), c, nm));
+        const float p2 = ptx::ex2(fmaf(__uint_as_float(sb[2 * j]), c, nm));
+        const float p3 = ptx::ex2(fmaf(__uint_as_float(sb[2 * j + 1]), c, nm));
+        ls0 += p0; ls1 += p1; ls2 += p2; ls3 += p3;
         pk[j] = ptx::pack_bf16x2(p0, p1);
-        lsum += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+        pk[16 + j] = ptx::pack_bf16x2(p2, p3);
       }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float p0 = (2 * j + 32 < nv) ? ptx::ex2(__uint_as_float(sb[2 * j]) * p.scale_log2 - m_ref) : 0.f;
-        const float p1 = (2 * j + 33 < nv) ? ptx::ex2(__uint_as_float(sb[2 * j + 1]) * p.scale_log2 - m_ref) : 0.f;
-        pk[16 + j] = ptx::pack_bf16x2(p0, p1);
-        lsum += __uint_as_float(pk[16 + j] << 16) + __uint_as_float(pk[16 + j] & 0xffff0000u);
-      }
-      l += lsum;
+      l += (ls0 + ls1) + (ls2 + ls3);
       ptx::tmem_st32(lane_addr + buf * 64, pk);
       ptx::tmem_wait_st();
       if (nv_tile < kTile) {
         // rows past the valid keys hold stale or foreign data: zero them in V
         // so 0 * garbage cannot reach O
-        if (!__all_sync(full, ptx::mbar_wait(bars.full[st], (u / kStages) & 1))) {
+        if (!__all_sync(full_mask, ptx::mbar_wait(bars.full[st], (u / kStages) & 1))) {
           record_timeout(p, abort_flag); alive = false; break;
         }
         const int nz = (kTile - nv_tile) * 8 * halves;  // 16-byte chunks
         for (int e = sm_tid; e < nz; e += 128) {
           const int h = e / ((kTile - nv_tile) * 8), rem = e % ((kTile - nv_tile) * 8);
-          const int row = nv_tile + rem / 8, c = rem % 8;
+          const int row = nv_tile + rem / 8, cc = rem % 8;
           *reinterpret_cast<uint4*>(smem + kRingOff + st * kStageBytes + 2 * kHalfTile +
-                                    h * kHalfTile + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                                    h * kHalfTile + row * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
         }
         ptx::fence_proxy_async_smem();
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(bars.p_full[buf]);
     }
-    // ---- epilogue: park this split's (O, m, l) in shared memory
-    float* stO = reinterpret_cast<float*>(smem + kStageO);
-    float* stM = reinterpret_cast<float*>(smem + kStageM);
-    float* stL = reinterpret_cast<float*>(smem + kStageL);
-    uint32_t o[kD / 32][32];
-    bool have = alive && U > 0 && !__any_sync(full, *abort_flag != 0);
-    if (have) {
-      if (!__all_sync(full, ptx::mbar_wait(bars.pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1))) {
-        record_timeout(p, abort_flag);
-        have = false;
-      } else {
-        ptx::tc_fence_after();
+    // ---- this split's unnormalised O, row max and row sum -> workspace
+    bool have = alive && U > 0 && !__any_sync(full_mask, *abort_flag != 0);
+    if (have && !__all_sync(full_mask, ptx::mbar_wait(bars.pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1))) {
+      record_timeout(p, abort_flag);
+      have = false;
+    }
+    if (have) ptx::tc_fence_after();
+    float4* po = reinterpret_cast<float4*>(part);
 #pragma unroll
-        for (int cb = 0; cb < kD / 32; ++cb) ptx::tmem_ld32(lane_addr + kOCol + cb * 32, o[cb]);
-        ptx::tmem_wait_ld();
+    for (int cb = 0; cb < kD / 32; ++cb) {
+      uint32_t o[32];
+      if (have) ptx::tmem_ld32_sync(lane_addr + kOCol + cb * 32, o);
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 v = have ? make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]),
+                                            __uint_as_float(o[j + 2]), __uint_as_float(o[j + 3]))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        __stcg(po + (cb * 8 + j / 4) * kRows + r, v);  // [d4][row]: coalesced over rows
       }
     }
-    ptx::named_bar_sync(1, 128);  // all softmax threads are done with the ring
-    const bool have2 = have && *abort_flag == 0;
-#pragma unroll
-    for (int cb = 0; cb < kD / 32; ++cb)
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(stO + r * kStageStride + cb * 32 + j) =
-            have2 ? make_float4(__uint_as_float(o[cb][j]), __uint_as_float(o[cb][j + 1]),
-                                __uint_as_float(o[cb][j + 2]), __uint_as_float(o[cb][j + 3]))
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    stM[r] = have2 ? m_ref : -INFINITY;
-    stL[r] = have2 ? l : 0.f;
+    __stcg(part + kRows * kD + r, have ? m_ref : -INFINITY);
+    __stcg(part + kRows * kD + kRows + r, have ? l : 0.f);
+    __threadfence();
   }
   __syncwarp();
   ptx::tc_fence_before();
   ptx::cluster_sync();
   ptx::tc_fence_after();
 
-  // ---- split combine through distributed shared memory
-  if (warp >= 2) {
+  // ---- split combine: CTA `rank` owns rows [rank*R, (rank+1)*R)
+  if (warp >= 2 && !bad) {
     const int sm_tid = threadIdx.x - 64;
     const int R = kRows / S;
-    const int per_row = kD / 4;
-    bool any_abort = false;
-    for (int s = 0; s < S; ++s)
-      any_abort |= ptx::ld_cluster_s32(ptx::map_rank(sbase + kMiscOff + 8, s)) != 0;
-    for (int it = sm_tid; it < R * per_row && !bad && !any_abort; it += 128) {
-      const int rr = (int)rank * R + it / per_row;
-      const int d4 = (it % per_row) * 4;
+    constexpr int per_row = kD / 4;
+    const float* base = p.part + (int64_t)(b * p.Hkv + g) * S * part_floats<kD>();
+    const int any_abort = *abort_flag;
+    for (int it = sm_tid; it < R * per_row; it += 128) {
+      const int rr = (int)rank * R + it % R;  // consecutive threads: consecutive rows
+      const int d4 = (it / R) * 4;
       if (rr >= rows) continue;
+      float ms[kMaxSplits];
+#pragma unroll
+      for (int s = 0; s < kMaxSplits; ++s)
+        ms[s] = s < S ? __ldcg(base + (int64_t)s * part_floats<kD>() + kRows * kD + rr) : -INFINITY;
       float M = -INFINITY;
-      for (int s = 0; s < S; ++s)
-        M = fmaxf(M, ptx::ld_cluster_f32(ptx::map_rank(sbase + kStageM + rr * 4, s)));
+#pragma unroll
+      for (int s = 0; s < kMaxSplits; ++s) M = fmaxf(M, ms[s]);
       float L = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s = 0; s < S; ++s) {
-        const float ms = ptx::ld_cluster_f32(ptx::map_rank(sbase + kStageM + rr * 4, s));
-        const float w = ptx::ex2(ms - M);
-        const float ls = ptx::ld_cluster_f32(ptx::map_rank(sbase + kStageL + rr * 4, s));
-        const float4 os = ptx::ld_cluster_f32x4(
-            ptx::map_rank(sbase + kStageO + (rr * kStageStride + d4) * 4, s));
-        L = fmaf(w, ls, L);
-        O.x = fmaf(w, os.x, O.x);
-        O.y = fmaf(w, os.y, O.y);
-        O.z = fmaf(w, os.z, O.z);
-        O.w = fmaf(w, os.w, O.w);
+#pragma unroll
+      for (int s = 0; s < kMaxSplits; ++s) {
+        if (s < S) {
+          const float* ps = base + (int64_t)s * part_floats<kD>();
+          const float ls = __ldcg(ps + kRows * kD + kRows + rr);
+          const float4 os = __ldcg(reinterpret_cast<const float4*>(ps) + (d4 / 4) * kRows + rr);
+          const float w = ptx::ex2(ms[s] - M);
+          L = fmaf(w, ls, L);
+          O.x = fmaf(w, os.x, O.x);
+          O.y = fmaf(w, os.y, O.y);
+          O.z = fmaf(w, os.z, O.z);
+          O.w = fmaf(w, os.w, O.w);
+        }
       }
+      if (any_abort) continue;
       const float inv = 1.f / L;
       const int i = rr / p.G, h = g * p.G + rr % p.G;
       uint2 pkd;
@@ -413,11 +430,8 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       *reinterpret_cast<uint2*>(p.out + ((int64_t)(b * p.blk + i) * p.Hq + h) * kD + d4) = pkd;
     }
   }
-  __syncwarp();
-  ptx::tc_fence_before();
-  ptx::cluster_sync();
   if (warp == 1) {
-    ptx::tc_fence_after();
+    __syncwarp();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
 }
@@ -449,7 +463,7 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
          CUDA_SUCCESS;
 }
 
-// Largest supported cluster size whose clusters can be resident (16, else 8).
+// Largest cluster size (16, else 8) whose clusters can be resident; 0 if none.
 template <int kD>
 int cluster_size(int device) {
   static int cached[64] = {0};
@@ -490,7 +504,10 @@ bool tc_supported(const orthrus_attn_args& a) {
          (a.Hq / a.Hkv) * a.blk <= kRows && a.blk <= 32 && a.Hq / a.Hkv <= 256;
 }
 
-size_t tc_workspace_bytes(const orthrus_attn_args&) { return 0; }
+size_t tc_workspace_bytes(const orthrus_attn_args& a) {
+  const int64_t per = a.D == 64 ? part_floats<64>() : part_floats<128>();
+  return (size_t)((int64_t)a.B * a.Hkv * kMaxSplits * per * 4);
+}
 
 int tc_launches(const orthrus_attn_args&) { return 1; }
 
@@ -525,7 +542,8 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   p.ctx_lens = a.ctx_lens;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = a.err;
-  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.blk = a.blk; p.cap = a.cap;
+  p.part = static_cast<float*>(a.workspace);
+  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.blk = a.blk; p.cap = a.cap;
   p.max_ctx = a.max_ctx; p.mask_mode = a.mask_mode; p.G = G; p.S = S;
   p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
 
@@ -534,13 +552,15 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_kernel<64>, p)
                                   : cudaLaunchKernelEx(&cfg, attn_tc_kernel<128>, p);
   if (e != cudaSuccess) return ORTHRUS_ECUDA;
