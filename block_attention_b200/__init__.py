@@ -39,6 +39,7 @@ class AttnArgs(ctypes.Structure):
                 ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("blk", ctypes.c_int32), ("cap", ctypes.c_int32),
                 ("max_ctx", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_int32),
                 ("q", ctypes.c_void_p), ("k_blk", ctypes.c_void_p),
                 ("v_blk", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
                 ("v_cache", ctypes.c_void_p), ("ctx_lens", ctypes.c_void_p),
@@ -155,13 +156,16 @@ def _ws(ws, device, op):
     return ws
 
 
+ATTN_EARLY_KV = 1
+
+
 def attn_args(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, out=None,
-              scale=None, max_ctx=None, err=None) -> AttnArgs:
+              scale=None, max_ctx=None, err=None, flags=0) -> AttnArgs:
     B, blk, Hq, D = q.shape
     Hkv, cap = k_cache.shape[1], k_cache.shape[2]
     return AttnArgs(_dtype(q), int(mask_mode), B, Hq, Hkv, D, blk, cap,
                     cap if max_ctx is None else int(max_ctx),
-                    float(D ** -0.5 if scale is None else scale),
+                    float(D ** -0.5 if scale is None else scale), int(flags),
                     q.data_ptr(), k_blk.data_ptr(), v_blk.data_ptr(), k_cache.data_ptr(),
                     v_cache.data_ptr(), ctx_lens.data_ptr(),
                     out.data_ptr() if out is not None else None,
@@ -173,7 +177,7 @@ def block_attn_workspace_bytes(args: AttnArgs) -> int:
 
 
 def block_attn(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, *, out=None,
-               scale=None, max_ctx=None, err=None, workspace=None, stream=None):
+               scale=None, max_ctx=None, err=None, workspace=None, stream=None, flags=0):
     """Attention of one layer for one round (see orthrus.h for the definition).
 
     q [B, blk, Hq, D]; k_blk/v_blk [B, blk, Hkv, D]; k_cache/v_cache
@@ -185,10 +189,12 @@ def block_attn(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, *, out=No
     if out is None:
         out = torch.empty_like(q)
     a = attn_args(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, out, scale,
-                  max_ctx, err)
+                  max_ctx, err, flags)
     need = block_attn_workspace_bytes(a)
     if need:
-        buf = _ws(workspace, q.device, "attn").get(need)
+        # fp32 calls use the buffer as scratch; bf16 calls also keep zeroed
+        # ticket counters at its end: separate default buffers per dtype
+        buf = _ws(workspace, q.device, f"attn_{q.dtype}").get(need)
         a.workspace, a.workspace_bytes = buf.data_ptr(), buf.numel()
     _check("orthrus_block_attn", lib().orthrus_block_attn(ctypes.byref(a), _stream(stream)))
     return out

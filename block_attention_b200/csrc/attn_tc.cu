@@ -6,35 +6,42 @@
 // the block for the diffusion view, causal for the AR verify view).
 //
 // Shape of the work.  Decoding reads every cached K/V row once per layer and
-// view, so the kernel is bound by HBM bandwidth; the G = Hq/Hkv query heads
+// view, so the path is bound by HBM bandwidth; the G = Hq/Hkv query heads
 // that share a kv-head and the blk block rows form one M = G*blk <= 128 row
 // tile, so each K/V tile fetched from HBM feeds a full 128-row tcgen05 MMA
 // (128 FLOP per KV byte at the Qwen3-8B shape -- beyond CUDA cores, so the
 // QK^T and PV products run on the tensor pipe).
 //
-// Grid: (S splits, Hkv, B) launched as clusters of S CTAs; one cluster covers
-// one (sequence, kv-head).  The keys cache[0, n) are cut into 64-key tiles,
-// followed by one tile holding the blk block rows; the tiles are dealt out
-// contiguously over the S CTAs (split-KV).  Each CTA:
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
-//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered
-//               TMEM tile, then O += P V with P read from TMEM
+// Two kernels per call, chained by programmatic dependent launch:
+//
+// attn_tc_partial, grid (S splits, Hkv, B), one CTA per SM.  The keys
+// cache[0, n) of a (sequence, kv-head) are cut into 128-key tiles, followed by
+// one tile holding the blk block rows; the tiles are dealt out contiguously
+// over the S splits.  Per CTA:
+//   warp 0      TMA producer: Q once, then K/V tiles through a 3 x 64 KB ring
+//   warp 1      MMA issuer (one thread): S = Q K^T (M=128, N=128 per
+//               instruction) into a double-buffered TMEM tile, then O += P V
+//               with P read from TMEM
 //   warps 2..5  softmax, one query row per thread: online softmax with lazy
 //               rescaling (O in TMEM is rescaled only when a row's running
 //               maximum grows by more than 2^8), P written back to TMEM as
-//               bf16; then the split combine.
-// A CTA needs ~97 KB of shared memory and 256 TMEM columns, so two fit on an
-// SM: every cluster of a launch is resident at once, and under programmatic
-// dependent launch the next kernel's CTAs can start while this one drains.
+//               bf16; finally the split's unnormalised O, row max and row sum
+//               go to an L2-resident workspace.
+// 128-key S tiles: a tcgen05.mma with N = 64 costs the issuing thread as much
+// as one with N = 128, so the wider tile halves the MMA issue time per key.
 //
-// Split combine: each CTA writes its unnormalised O (fp32) with its row maxima
-// and sums to an L2-resident workspace, the cluster synchronises, and CTA s
-// reduces rows [s*128/S, (s+1)*128/S) over the S splits in split order
-// (deterministic) and writes them out -- one launch.
+// attn_tc_combine, grid (16 row groups, Hkv, B): merges the S partials of 8
+// query rows in split order (deterministic) and writes bf16 output.  Its CTAs
+// are small, so they start while the partial kernel drains, and the next
+// kernel in the stream can take the SMs the partial kernel frees.
+//
+// With ORTHRUS_ATTN_EARLY_KV the partial kernel reads ctx_lens and starts
+// streaming K/V tiles before waiting on the preceding kernel; Q and the block
+// K/V are read only after that wait.
 //
 // Every mbarrier wait is bounded: on a timeout the kernel records
-// ORTHRUS_ETIMEOUT in the error word, stops issuing work, drains what it
-// issued and still reaches the cluster barrier, so it always terminates.
+// ORTHRUS_ETIMEOUT in the error word, stops issuing work and drains what it
+// issued, so it always terminates.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -49,16 +56,18 @@ namespace orthrus {
 namespace {
 
 constexpr int kRows = 128;          // UMMA M
-constexpr int kTile = 64;           // keys per tile
-constexpr int kStages = 2;          // K/V ring depth
+constexpr int kTile = 128;          // keys per tile (UMMA N of S = Q K^T)
+constexpr int kStages = 3;          // K/V ring depth
 constexpr int kThreads = 192;       // 6 warps
-constexpr int kTmemCols = 256;      // S0 [0,64) S1 [64,128) O [128,256)
-constexpr int kOCol = 128;
+constexpr int kTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256, 256+D)
+constexpr int kOCol = 256;
 constexpr float kLazyThresh = 8.f;  // log2 units
-constexpr int kMaxSplits = 16;      // largest cluster (non-portable size)
+constexpr int kMaxSplits = 32;
+constexpr int kGroupRows = 8;       // rows per combine CTA
+constexpr int kCombineThreads = 256;
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kHalfTile = kTile * 128;      // one 64-dim half of a K or V tile
+constexpr int kHalfTile = kTile * 128;      // one 64-dim half of a K or V tile (16 KB)
 constexpr int kQBytes = 2 * kRows * 128;    // two 64-dim halves, 128 B rows
 constexpr int kStageBytes = 4 * kHalfTile;  // K (2 halves) + V (2 halves)
 constexpr int kRingOff = kQBytes;
@@ -67,21 +76,21 @@ constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 
-// workspace per (b, g, split): O as [D/4][128 rows] float4, then m[128], l[128]
+// One split's partial: O as [16 row groups][D/4][8 rows] float4, then m[128], l[128].
 template <int kD>
 __host__ __device__ constexpr int part_floats() { return kRows * kD + 2 * kRows; }
 
 struct __align__(64) TcParams {
   CUtensorMap tm_q;   // 3D (D, Hq, B*blk), box (64, G, blk)
-  CUtensorMap tm_kc;  // 2D (D, B*Hkv*cap), box (64, 64)
+  CUtensorMap tm_kc;  // 2D (D, B*Hkv*cap), box (64, 128)
   CUtensorMap tm_vc;
   CUtensorMap tm_kb;  // 3D (D, Hkv, B*blk), box (64, 1, blk)
   CUtensorMap tm_vb;
   const int32_t* ctx_lens;
   __nv_bfloat16* out;
   int32_t* err;
-  float* part;  // split partials
-  int B, Hq, Hkv, blk, cap, max_ctx, mask_mode, G, S;
+  float* part;  // [B][Hkv][S] partials
+  int B, Hq, Hkv, blk, cap, max_ctx, mask_mode, G, S, early;
   float scale_log2;
 };
 
@@ -89,22 +98,21 @@ struct Bars {
   uint32_t q_full, full[kStages], empty[kStages], s_full[2], p_full[2], pv_done[2], mma_done;
 };
 
-__device__ __forceinline__ void record_timeout(const TcParams& p, volatile int* abort_flag) {
+__device__ __forceinline__ void record_timeout(int32_t* err, volatile int* abort_flag) {
   *abort_flag = 1;
-  set_err(p.err, ORTHRUS_ETIMEOUT);
+  set_err(err, ORTHRUS_ETIMEOUT);
 }
 
 template <int kD>
-__global__ void __launch_bounds__(kThreads, 2)
-attn_tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_partial(const __grid_constant__ TcParams p) {
   constexpr int halves = kD / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.y, b = blockIdx.z;
-  const uint32_t rank = ptx::cluster_rank();
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int S = p.S;
   const unsigned full_mask = 0xffffffffu;
 
@@ -160,63 +168,92 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // Programmatic dependent launch: the next kernel in the stream may start
-  // its own setup now; everything below may read what earlier kernels wrote.
   ptx::griddep_launch_dependents();
-  ptx::griddep_wait();
-
-  // ---- sequence geometry (every CTA of the cluster reads the same n)
-  const int n = p.ctx_lens[b];
-  const bool bad = n < 0 || n > p.max_ctx;
-  if (bad && rank == 0 && g == 0 && threadIdx.x == 0) set_err(p.err, ORTHRUS_ECAPACITY);
-  const int Tc = bad ? 0 : ceil_div(n, kTile);  // cache tiles
-  const int T = bad ? 0 : Tc + 1;               // + the block tile
-  const int t0 = (int)(((int64_t)rank * T) / S);
-  const int t1 = (int)(((int64_t)(rank + 1) * T) / S);
-  const int U = t1 - t0;
 
   const uint32_t q_s = sbase;
   auto k_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes; };
   auto v_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes + 2 * kHalfTile; };
-  float* part = p.part + ((int64_t)(b * p.Hkv + g) * S + rank) * part_floats<kD>();
+  const int slab = (b * p.Hkv + g) * p.cap;
+  // tiles of this split: cache tiles [0, Tc) then the block tile Tc
+  auto geometry = [&](int n, int& Tc, int& t0, int& U) {
+    const bool bad = n < 0 || n > p.max_ctx;
+    Tc = bad ? 0 : ceil_div(n, kTile);
+    const int T = bad ? 0 : Tc + 1;
+    t0 = (int)(((int64_t)split * T) / S);
+    U = (int)(((int64_t)(split + 1) * T) / S) - t0;
+  };
+  auto issue_tile = [&](int u, int t, int Tc) {
+    const int st = u % kStages;
+    const bool blk_tile = t == Tc;
+    const int rows_ld = blk_tile ? p.blk : kTile;
+    ptx::mbar_expect_tx(bars.full[st], (uint32_t)(2 * halves * rows_ld * 128));
+    for (int h = 0; h < halves; ++h) {
+      if (blk_tile) {
+        ptx::tma_load_3d(k_s(st) + h * kHalfTile, &p.tm_kb, bars.full[st], 64 * h, g, b * p.blk);
+        ptx::tma_load_3d(v_s(st) + h * kHalfTile, &p.tm_vb, bars.full[st], 64 * h, g, b * p.blk);
+      } else {
+        ptx::tma_load_2d(k_s(st) + h * kHalfTile, &p.tm_kc, bars.full[st], 64 * h, slab + t * kTile);
+        ptx::tma_load_2d(v_s(st) + h * kHalfTile, &p.tm_vc, bars.full[st], 64 * h, slab + t * kTile);
+      }
+    }
+  };
+
+  // Early cache streaming: the first ring's worth of cache tiles (never the
+  // block tile, which the preceding kernel may still be writing).
+  int early_issued = 0;
+  int early_n = 0;
+  if (p.early && warp == 0 && lane == 0) {
+    early_n = p.ctx_lens[b];
+    int Tc, t0, U;
+    geometry(early_n, Tc, t0, U);
+    while (early_issued < min(U, kStages) && t0 + early_issued < Tc) {
+      issue_tile(early_issued, t0 + early_issued, Tc);
+      ++early_issued;
+    }
+  }
+  ptx::griddep_wait();
+
+  const int n = p.ctx_lens[b];
+  const bool bad = n < 0 || n > p.max_ctx;
+  if (bad && split == 0 && g == 0 && threadIdx.x == 0) set_err(p.err, ORTHRUS_ECAPACITY);
+  int Tc, t0, U;
+  geometry(n, Tc, t0, U);
+  if (warp == 0 && lane == 0 && early_issued > 0 && early_n != n) {
+    // the EARLY_KV contract was broken (the length changed under us): drain
+    // the early loads and produce nothing for this split
+    for (int u = 0; u < early_issued; ++u)
+      if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1))
+        record_timeout(p.err, abort_flag);
+    set_err(p.err, ORTHRUS_EINVAL);
+    *abort_flag = 1;
+    early_issued = 0;
+  }
+  __syncthreads();
+  if (*abort_flag) U = 0;
+  float* part = p.part + ((int64_t)(b * p.Hkv + g) * S + split) * part_floats<kD>();
 
   if (warp == 0) {
     // ================================================== TMA producer
     if (lane == 0 && U > 0) {
-      int issued = 0;
+      int issued = early_issued;
       ptx::mbar_expect_tx(bars.q_full, (uint32_t)(halves * rows * 128));
       for (int h = 0; h < halves; ++h)
         ptx::tma_load_3d(q_s + h * (kRows * 128), &p.tm_q, bars.q_full, 64 * h, g * p.G,
                          b * p.blk);
-      const int slab = (b * p.Hkv + g) * p.cap;
-      for (int u = 0; u < U && !*abort_flag; ++u) {
-        const int t = t0 + u, st = u % kStages;
+      for (int u = early_issued; u < U && !*abort_flag; ++u) {
+        const int st = u % kStages;
         if (!ptx::mbar_wait(bars.empty[st], ((u / kStages) & 1) ^ 1)) {
-          record_timeout(p, abort_flag);
+          record_timeout(p.err, abort_flag);
           break;
         }
-        const bool blk_tile = t == Tc;
-        const int rows_ld = blk_tile ? p.blk : kTile;
-        ptx::mbar_expect_tx(bars.full[st], (uint32_t)(2 * halves * rows_ld * 128));
-        for (int h = 0; h < halves; ++h) {
-          if (blk_tile) {
-            ptx::tma_load_3d(k_s(st) + h * kHalfTile, &p.tm_kb, bars.full[st], 64 * h, g,
-                             b * p.blk);
-            ptx::tma_load_3d(v_s(st) + h * kHalfTile, &p.tm_vb, bars.full[st], 64 * h, g,
-                             b * p.blk);
-          } else {
-            ptx::tma_load_2d(k_s(st) + h * kHalfTile, &p.tm_kc, bars.full[st], 64 * h,
-                             slab + t * kTile);
-            ptx::tma_load_2d(v_s(st) + h * kHalfTile, &p.tm_vc, bars.full[st], 64 * h,
-                             slab + t * kTile);
-          }
-        }
+        issue_tile(u, t0 + u, Tc);
         issued = u + 1;
       }
       // drain: every issued load must have landed before the CTA exits
       for (int u = max(0, issued - kStages); u < issued; ++u)
-        if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1)) record_timeout(p, abort_flag);
-      if (!ptx::mbar_wait(bars.q_full, 0)) record_timeout(p, abort_flag);
+        if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1))
+          record_timeout(p.err, abort_flag);
+      if (!ptx::mbar_wait(bars.q_full, 0)) record_timeout(p.err, abort_flag);
     }
   } else if (warp == 1) {
     // ================================================== MMA issuer
@@ -233,7 +270,7 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
           // V tile as the MN-major B operand: 8-key groups 1024 B apart,
           // 64-dim halves kHalfTile apart
           const uint64_t bd = ptx::sdesc_sw128(v_s(st) + k * 2048, kHalfTile, 1024);
-          ptx::mma_ts(tmem + kOCol, tmem + buf * 64 + k * 8, bd, id_pv,
+          ptx::mma_ts(tmem + kOCol, tmem + buf * kTile + k * 8, bd, id_pv,
                       (u > 0 || k > 0) ? 1u : 0u);
         }
         ptx::tc_commit(bars.pv_done[buf]);
@@ -250,19 +287,19 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
           const uint32_t h = k >> 2, kk = k & 3;  // 64-dim half, 16-dim step in it
           const uint64_t ad = ptx::sdesc_sw128(q_s + h * (kRows * 128) + kk * 32, 16, 1024);
           const uint64_t bd = ptx::sdesc_sw128(k_s(st) + h * kHalfTile + kk * 32, 16, 1024);
-          ptx::mma_ss(tmem + buf * 64, ad, bd, id_s, k > 0 ? 1u : 0u);
+          ptx::mma_ss(tmem + buf * kTile, ad, bd, id_s, k > 0 ? 1u : 0u);
         }
         ptx::tc_commit(bars.s_full[buf]);
         if (u >= 1 && !pv(u - 1)) { ok = false; break; }
       }
       if (ok && !*abort_flag) ok = pv(U - 1);
-      if (!ok) record_timeout(p, abort_flag);
+      if (!ok) record_timeout(p.err, abort_flag);
       // every MMA issued so far has finished before TMEM is released
       ptx::tc_commit(bars.mma_done);
-      if (!ptx::mbar_wait(bars.mma_done, 0)) record_timeout(p, abort_flag);
+      if (!ptx::mbar_wait(bars.mma_done, 0)) record_timeout(p.err, abort_flag);
     }
   } else {
-    // ================================================== softmax + partial
+    // ================================================== softmax
     const int quad = warp & 3;            // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;       // query row of this thread
     const int i_blk = r < rows ? r / p.G : p.blk;
@@ -275,12 +312,12 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       if (__any_sync(full_mask, *abort_flag != 0)) { alive = false; break; }
       const int t = t0 + u, buf = u & 1, st = u % kStages;
       if (!__all_sync(full_mask, ptx::mbar_wait(bars.s_full[buf], (u >> 1) & 1))) {
-        record_timeout(p, abort_flag); alive = false; break;
+        record_timeout(p.err, abort_flag); alive = false; break;
       }
       ptx::tc_fence_after();
-      uint32_t sa[32], sb[32];
-      ptx::tmem_ld32_sync(lane_addr + buf * 64, sa);
-      ptx::tmem_ld32_sync(lane_addr + buf * 64 + 32, sb);
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) ptx::tmem_ld32_sync(lane_addr + buf * kTile + cb * 32, sv[cb]);
       const bool blk_tile = t == Tc;
       const int nv_tile = blk_tile ? p.blk : min(kTile, n - t * kTile);
       int nv = nv_tile;
@@ -288,25 +325,24 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       // masked keys -> -inf before the max and the exponent (exactly 0 in P)
       if (nv < kTile) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j >= nv) sa[j] = __float_as_uint(-INFINITY);
-          if (j + 32 >= nv) sb[j] = __float_as_uint(-INFINITY);
-        }
-      }
-      float mt0 = -INFINITY, mt1 = -INFINITY;
+        for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        mt0 = fmaxf(mt0, __uint_as_float(sa[j]));
-        mt1 = fmaxf(mt1, __uint_as_float(sb[j]));
+          for (int j = 0; j < 32; ++j)
+            if (cb * 32 + j >= nv) sv[cb][j] = __float_as_uint(-INFINITY);
       }
-      const float ms = fmaxf(mt0, mt1) * c;
+      float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mt[cb] = fmaxf(mt[cb], __uint_as_float(sv[cb][j]));
+      const float ms = fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3])) * c;
       const bool need = ms > m_ref + kLazyThresh;
       if (__any_sync(full_mask, need)) {
         const float m_new = need ? ms : m_ref;
         const float f = ptx::ex2(m_ref - m_new);  // 0 for the first tile, 1 if unchanged
         if (u > 0) {
           if (!__all_sync(full_mask, ptx::mbar_wait(bars.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1))) {
-            record_timeout(p, abort_flag); alive = false; break;
+            record_timeout(p.err, abort_flag); alive = false; break;
           }
           ptx::tc_fence_after();
 #pragma unroll
@@ -322,29 +358,32 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
         l *= f;
         m_ref = m_new;
       }
-      // P = 2^(s*c - m_ref) as bf16 pairs into the first 32 columns of this S
+      // P = 2^(s*c - m_ref) as bf16 pairs into the first 64 columns of this S
       // buffer; ex2(-inf) = 0 for masked keys
       const float nm = -m_ref;
-      uint32_t pk[32];
-      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float p0 = ptx::ex2(fmaf(__uint_as_float(sa[2 * j]), c, nm));
-        const float p1 = ptx::ex2(fmaf(__uint_as_float(sa[2 * j + 1]), c, nm));
-        const float p2 = ptx::ex2(fmaf(__uint_as_float(sb[2 * j]), c, nm));
-        const float p3 = ptx::ex2(fmaf(__uint_as_float(sb[2 * j + 1]), c, nm));
-        ls0 += p0; ls1 += p1; ls2 += p2; ls3 += p3;
-        pk[j] = ptx::pack_bf16x2(p0, p1);
-        pk[16 + j] = ptx::pack_bf16x2(p2, p3);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half][2 * j]), c, nm));
+          const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half][2 * j + 1]), c, nm));
+          const float p2 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half + 1][2 * j]), c, nm));
+          const float p3 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half + 1][2 * j + 1]), c, nm));
+          ls[0] += p0; ls[1] += p1; ls[2] += p2; ls[3] += p3;
+          pk[j] = ptx::pack_bf16x2(p0, p1);
+          pk[16 + j] = ptx::pack_bf16x2(p2, p3);
+        }
+        ptx::tmem_st32(lane_addr + buf * kTile + half * 32, pk);
       }
-      l += (ls0 + ls1) + (ls2 + ls3);
-      ptx::tmem_st32(lane_addr + buf * 64, pk);
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       ptx::tmem_wait_st();
       if (nv_tile < kTile) {
         // rows past the valid keys hold stale or foreign data: zero them in V
         // so 0 * garbage cannot reach O
         if (!__all_sync(full_mask, ptx::mbar_wait(bars.full[st], (u / kStages) & 1))) {
-          record_timeout(p, abort_flag); alive = false; break;
+          record_timeout(p.err, abort_flag); alive = false; break;
         }
         const int nz = (kTile - nv_tile) * 8 * halves;  // 16-byte chunks
         for (int e = sm_tid; e < nz; e += 128) {
@@ -361,11 +400,12 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
     // ---- this split's unnormalised O, row max and row sum -> workspace
     bool have = alive && U > 0 && !__any_sync(full_mask, *abort_flag != 0);
     if (have && !__all_sync(full_mask, ptx::mbar_wait(bars.pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1))) {
-      record_timeout(p, abort_flag);
+      record_timeout(p.err, abort_flag);
       have = false;
     }
     if (have) ptx::tc_fence_after();
-    float4* po = reinterpret_cast<float4*>(part);
+    const int rg = r / kGroupRows, ri = r % kGroupRows;
+    float4* po = reinterpret_cast<float4*>(part) + (int64_t)rg * (kD / 4) * kGroupRows + ri;
 #pragma unroll
     for (int cb = 0; cb < kD / 32; ++cb) {
       uint32_t o[32];
@@ -375,65 +415,80 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
         const float4 v = have ? make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]),
                                             __uint_as_float(o[j + 2]), __uint_as_float(o[j + 3]))
                               : make_float4(0.f, 0.f, 0.f, 0.f);
-        __stcg(po + (cb * 8 + j / 4) * kRows + r, v);  // [d4][row]: coalesced over rows
+        __stcg(po + (cb * 8 + j / 4) * kGroupRows, v);
       }
     }
     __stcg(part + kRows * kD + r, have ? m_ref : -INFINITY);
     __stcg(part + kRows * kD + kRows + r, have ? l : 0.f);
-    __threadfence();
   }
   __syncwarp();
   ptx::tc_fence_before();
-  ptx::cluster_sync();
-  ptx::tc_fence_after();
-
-  // ---- split combine: CTA `rank` owns rows [rank*R, (rank+1)*R)
-  if (warp >= 2 && !bad) {
-    const int sm_tid = threadIdx.x - 64;
-    const int R = kRows / S;
-    constexpr int per_row = kD / 4;
-    const float* base = p.part + (int64_t)(b * p.Hkv + g) * S * part_floats<kD>();
-    const int any_abort = *abort_flag;
-    for (int it = sm_tid; it < R * per_row; it += 128) {
-      const int rr = (int)rank * R + it % R;  // consecutive threads: consecutive rows
-      const int d4 = (it / R) * 4;
-      if (rr >= rows) continue;
-      float ms[kMaxSplits];
-#pragma unroll
-      for (int s = 0; s < kMaxSplits; ++s)
-        ms[s] = s < S ? __ldcg(base + (int64_t)s * part_floats<kD>() + kRows * kD + rr) : -INFINITY;
-      float M = -INFINITY;
-#pragma unroll
-      for (int s = 0; s < kMaxSplits; ++s) M = fmaxf(M, ms[s]);
-      float L = 0.f;
-      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int s = 0; s < kMaxSplits; ++s) {
-        if (s < S) {
-          const float* ps = base + (int64_t)s * part_floats<kD>();
-          const float ls = __ldcg(ps + kRows * kD + kRows + rr);
-          const float4 os = __ldcg(reinterpret_cast<const float4*>(ps) + (d4 / 4) * kRows + rr);
-          const float w = ptx::ex2(ms[s] - M);
-          L = fmaf(w, ls, L);
-          O.x = fmaf(w, os.x, O.x);
-          O.y = fmaf(w, os.y, O.y);
-          O.z = fmaf(w, os.z, O.z);
-          O.w = fmaf(w, os.w, O.w);
-        }
-      }
-      if (any_abort) continue;
-      const float inv = 1.f / L;
-      const int i = rr / p.G, h = g * p.G + rr % p.G;
-      uint2 pkd;
-      pkd.x = ptx::pack_bf16x2(O.x * inv, O.y * inv);
-      pkd.y = ptx::pack_bf16x2(O.z * inv, O.w * inv);
-      *reinterpret_cast<uint2*>(p.out + ((int64_t)(b * p.blk + i) * p.Hq + h) * kD + d4) = pkd;
-    }
-  }
+  __syncthreads();
   if (warp == 1) {
-    __syncwarp();
+    ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Merge the S split partials of 8 query rows, in split order, and write bf16.
+template <int kD>
+__global__ void __launch_bounds__(kCombineThreads)
+attn_tc_combine(const __grid_constant__ TcParams p) {
+  const int rg = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int it = threadIdx.x;  // item: (d4, row in group)
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
+  const int n = p.ctx_lens[b];
+  if (n < 0 || n > p.max_ctx) return;  // reported by the partial kernel
+  if (it >= (kD / 4) * kGroupRows) return;
+  const int d4 = it / kGroupRows, ri = it % kGroupRows;
+  const int r = rg * kGroupRows + ri;
+  if (r >= p.G * p.blk) return;
+  const int S = p.S;
+  const float* base = p.part + (int64_t)(b * p.Hkv + g) * S * part_floats<kD>();
+  const int64_t o_off = ((int64_t)rg * (kD / 4) + d4) * kGroupRows + ri;  // float4 index
+  float M = -INFINITY;
+  for (int s0 = 0; s0 < S; s0 += 8) {
+    float m8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      m8[k] = s0 + k < S ? __ldcg(base + (int64_t)(s0 + k) * part_floats<kD>() + kRows * kD + r)
+                         : -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) M = fmaxf(M, m8[k]);
+  }
+  float L = 0.f;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < S; s0 += 8) {
+    float m8[8], l8[8];
+    float4 o8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (s0 + k < S) {
+        const float* ps = base + (int64_t)(s0 + k) * part_floats<kD>();
+        m8[k] = __ldcg(ps + kRows * kD + r);
+        l8[k] = __ldcg(ps + kRows * kD + kRows + r);
+        o8[k] = __ldcg(reinterpret_cast<const float4*>(ps) + o_off);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (s0 + k < S) {
+        const float w = M == -INFINITY ? 0.f : ptx::ex2(m8[k] - M);
+        L = fmaf(w, l8[k], L);
+        O.x = fmaf(w, o8[k].x, O.x);
+        O.y = fmaf(w, o8[k].y, O.y);
+        O.z = fmaf(w, o8[k].z, O.z);
+        O.w = fmaf(w, o8[k].w, O.w);
+      }
+    }
+  }
+  const float inv = 1.f / L;
+  const int i = r / p.G, h = g * p.G + r % p.G;
+  uint2 pkd;
+  pkd.x = ptx::pack_bf16x2(O.x * inv, O.y * inv);
+  pkd.y = ptx::pack_bf16x2(O.z * inv, O.w * inv);
+  *reinterpret_cast<uint2*>(p.out + ((int64_t)(b * p.blk + i) * p.Hq + h) * kD + 4 * d4) = pkd;
 }
 
 // ------------------------------------------------------------------ host
@@ -463,59 +518,47 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
          CUDA_SUCCESS;
 }
 
-// Largest cluster size (16, else 8) whose clusters can be resident; 0 if none.
 template <int kD>
-int cluster_size(int device) {
-  static int cached[64] = {0};
-  if (device >= 0 && device < 64 && cached[device]) return cached[device];
-  int best = 0;
-  if (cudaFuncSetAttribute(attn_tc_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+bool prepare(int device) {
+  static bool done[64] = {false};
+  if (device >= 0 && device < 64 && done[device]) return true;
+  if (cudaFuncSetAttribute(attn_tc_partial<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kSmemBytes) != cudaSuccess)
-    return 0;
-  cudaFuncSetAttribute(attn_tc_kernel<kD>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  for (int s : {16, 8}) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(s, 8, 1);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = s;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, attn_tc_kernel<kD>, &cfg) == cudaSuccess &&
-        nclusters > 0) {
-      best = s;
-      break;
-    }
-    cudaGetLastError();
-  }
-  if (device >= 0 && device < 64) cached[device] = best;
-  return best;
+    return false;
+  if (device >= 0 && device < 64) done[device] = true;
+  return true;
+}
+
+// Splits per (sequence, kv-head): one wave of CTAs (one per SM) when the
+// batch is small, else 4 per head so ragged lengths still balance; never more
+// splits than the longest sequence has tiles.
+int choose_splits(const orthrus_attn_args& a) {
+  const int heads = a.B * a.Hkv;
+  int S = heads >= 148 ? 4 : 148 / heads;
+  S = min(S, ceil_div(a.max_ctx, kTile) + 1);
+  return max(1, min(S, kMaxSplits));
 }
 
 }  // namespace
 
 bool tc_supported(const orthrus_attn_args& a) {
   return a.dtype == ORTHRUS_BF16 && (a.D == 64 || a.D == 128) &&
-         (a.Hq / a.Hkv) * a.blk <= kRows && a.blk <= 32 && a.Hq / a.Hkv <= 256;
+         (a.Hq / a.Hkv) * a.blk <= kRows && a.blk <= 32 && a.Hq / a.Hkv <= 256 &&
+         a.B <= 65535 && a.Hkv <= 65535;
 }
 
 size_t tc_workspace_bytes(const orthrus_attn_args& a) {
   const int64_t per = a.D == 64 ? part_floats<64>() : part_floats<128>();
-  return (size_t)((int64_t)a.B * a.Hkv * kMaxSplits * per * 4);
+  return (size_t)((int64_t)a.B * a.Hkv * choose_splits(a) * per * 4);
 }
 
-int tc_launches(const orthrus_attn_args&) { return 1; }
+int tc_launches(const orthrus_attn_args&) { return 2; }
 
 int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ECUDA;
-  const int S = a.D == 64 ? cluster_size<64>(dev) : cluster_size<128>(dev);
-  if (S == 0) return ORTHRUS_ECUDA;
+  if (!(a.D == 64 ? prepare<64>(dev) : prepare<128>(dev))) return ORTHRUS_ECUDA;
+  const int S = choose_splits(a);
   TcParams p;
   const int G = a.Hq / a.Hkv;
   const cuuint64_t es = 2;
@@ -545,26 +588,28 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   p.part = static_cast<float*>(a.workspace);
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.blk = a.blk; p.cap = a.cap;
   p.max_ctx = a.max_ctx; p.mask_mode = a.mask_mode; p.G = G; p.S = S;
+  p.early = (a.flags & ORTHRUS_ATTN_EARLY_KV) ? 1 : 0;
   p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
 
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S, a.Hkv, a.B);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  const cudaError_t e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_kernel<64>, p)
-                                  : cudaLaunchKernelEx(&cfg, attn_tc_kernel<128>, p);
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_partial<64>, p)
+                            : cudaLaunchKernelEx(&cfg, attn_tc_partial<128>, p);
   if (e != cudaSuccess) return ORTHRUS_ECUDA;
-  return ORTHRUS_OK;
+  cfg.gridDim = dim3(kRows / kGroupRows, a.Hkv, a.B);
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = 0;
+  e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_combine<64>, p)
+                : cudaLaunchKernelEx(&cfg, attn_tc_combine<128>, p);
+  return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
 }
 
 }  // namespace orthrus

@@ -247,6 +247,16 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
                : "memory");
   return v;
 }
+// Bulk copy (TMA engine) from this CTA's shared memory to a cluster peer's;
+// completion is signalled on the peer's mbarrier.  Addresses 16-byte aligned,
+// size a multiple of 16.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta,
+                                                  uint32_t bytes, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst_cluster), "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

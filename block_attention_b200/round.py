@@ -21,7 +21,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import BIDIR_BLOCK, CAUSAL_VERIFY
+from . import ATTN_EARLY_KV, BIDIR_BLOCK, CAUSAL_VERIFY
 from . import attn_args, block_attn, consensus, kv_commit, lib, vocab_argmax, Workspace
 from . import synth
 
@@ -86,12 +86,16 @@ class DecodeRound:
 
     # ------------------------------------------------------------ segments
     def _attn(self, view):
+        # Within a view the kernel before each attention call is the previous
+        # layer's attention (or, for layer 0, the length reset copy / the
+        # diffusion argmax): none of them writes a cache or the lengths, so the
+        # cache may start streaming before that kernel has finished.
         mode = BIDIR_BLOCK if view == 0 else CAUSAL_VERIFY
         for l in range(self.L):
             block_attn(self.q[view, l], self.k_blk[view, l], self.v_blk[view, l],
                        self.k_cache[l], self.v_cache[l], self.ctx_lens, mode,
                        out=self.out[view, l], max_ctx=self.max_ctx, err=self.err,
-                       workspace=self.ws[f"attn{view}"])
+                       workspace=self.ws[f"attn{view}"], flags=ATTN_EARLY_KV)
 
     def seg_a(self):
         self.ctx_lens.copy_(self.ctx_base)  # same round every step

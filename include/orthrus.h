@@ -69,6 +69,15 @@ typedef enum {
   ORTHRUS_CAUSAL_VERIFY = 1
 } orthrus_mask_mode;
 
+typedef enum {
+  /* The kernel that immediately precedes this call on the stream does not
+   * write k_cache, v_cache or ctx_lens.  BF16 calls then start streaming the
+   * cache while that kernel is still finishing (programmatic dependent
+   * launch); q, k_blk and v_blk are still read only after it has completed.
+   * Without the flag every input is read after the preceding work finishes. */
+  ORTHRUS_ATTN_EARLY_KV = 1
+} orthrus_attn_flags;
+
 /* ------------------------------------------------------------------------
  * Block attention (both views), one layer.
  *
@@ -95,6 +104,7 @@ typedef struct orthrus_attn_args {
   int32_t max_ctx;   /* host bound on every ctx_lens[b]; 0 <= max_ctx <= cap.
                         Sizes the grid; a device length above it is an error. */
   float scale;       /* softmax scale, usually 1/sqrt(D) */
+  int32_t flags;     /* bitwise OR of orthrus_attn_flags (0 = none) */
   const void* q;       /* [B, blk, Hq, D] */
   const void* k_blk;   /* [B, blk, Hkv, D] block K (bidir: diffusion K_diff; causal: AR K) */
   const void* v_blk;   /* [B, blk, Hkv, D] */
@@ -103,9 +113,17 @@ typedef struct orthrus_attn_args {
   const int32_t* ctx_lens; /* [B] device, committed context length n per sequence */
   void* out;           /* [B, blk, Hq, D], same dtype as q */
   int32_t* err;        /* optional device int32 error word (NULL = none) */
-  void* workspace;     /* zero-initialised, orthrus_block_attn_workspace() bytes */
-  size_t workspace_bytes;
+  void* workspace;     /* >= orthrus_block_attn_workspace() bytes, 256-byte aligned,
+                          zero-initialised once (see below) */
+  size_t workspace_bytes; /* size of the caller's buffer */
 } orthrus_attn_args;
+
+/* Workspace of orthrus_block_attn.  BF16 calls keep 16*B*Hkv bytes of ticket
+ * counters at the END of the buffer (last workspace_bytes) and use the front
+ * as scratch; every call leaves its counters at zero.  One buffer, zeroed
+ * once, may serve any sequence of BF16 calls on one stream whose sizes fit it.
+ * FP32 calls use the buffer as scratch only: give FP32 and BF16 calls
+ * separate buffers. */
 
 /* Bytes of workspace orthrus_block_attn needs for these arguments (0 if none).
  * Pointers in `a` are not read.  Returns 0 for invalid shapes as well. */

@@ -56,7 +56,8 @@ def test_struct_layout_matches_c(tmp_path):
 #define F(T, m) printf(#T " " #m " %zu\n", offsetof(T, m))
 int main(void) {
   printf("orthrus_attn_args size %zu\n", sizeof(orthrus_attn_args));
-  F(orthrus_attn_args, scale); F(orthrus_attn_args, q); F(orthrus_attn_args, ctx_lens);
+  F(orthrus_attn_args, scale); F(orthrus_attn_args, flags); F(orthrus_attn_args, q);
+  F(orthrus_attn_args, ctx_lens);
   F(orthrus_attn_args, err); F(orthrus_attn_args, workspace_bytes);
   printf("orthrus_commit_args size %zu\n", sizeof(orthrus_commit_args));
   F(orthrus_commit_args, k_cache); F(orthrus_commit_args, cache_layer_stride);

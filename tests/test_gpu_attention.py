@@ -138,3 +138,36 @@ def test_device_length_over_bound_sets_error_word(oracle_mod, dtype):
                                 sub["v_cache"], sub["ctx_lens"], 0)
     assert rel_err_rows(got[:1], ref).max() <= TOL[dtype]
     assert np.all(got[1] == 7.0)  # skipped sequence left untouched
+
+
+def test_one_workspace_reused_across_shapes(oracle_mod):
+    """One bf16 workspace serves calls of different shapes in any order: its
+    ticket counters (kept at the end of the buffer) stay valid."""
+    ws = ba.Workspace("cuda")
+    shapes = [(2, 32, 8, 128, 32, [3000, 500]), (1, 4, 1, 64, 32, [100]),
+              (1, 16, 8, 128, 32, [2048]), (1, 8, 8, 128, 4, [0]),
+              (3, 32, 8, 128, 32, [900, 10, 4000]), (1, 16, 8, 128, 32, [2048])]
+    for k, (B, Hq, Hkv, D, blk, lens) in enumerate(shapes):
+        inp = synth.attn_inputs(B, Hq, Hkv, D, blk, lens, max(lens) + 8, "bf16", seed=300 + k)
+        t = {kk: to_dev(v) for kk, v in inp.items()}
+        for mode in (0, 1):
+            out = ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                                t["ctx_lens"], mode, workspace=ws)
+            torch.cuda.synchronize()
+            ref = oracle_mod.block_attn(inp["q"], inp["k_blk"], inp["v_blk"], inp["k_cache"],
+                                        inp["v_cache"], inp["ctx_lens"], mode)
+            e = rel_err_rows(to_host(out), ref)
+            assert e.max() <= TOL["bf16"], (k, mode, e.max())
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_early_kv_flag_same_result(oracle_mod, mode):
+    """ORTHRUS_ATTN_EARLY_KV only moves when the cache is read: same output."""
+    inp = synth.attn_inputs(2, 32, 8, 128, 32, [4000, 1500], 4100, "bf16", seed=109)
+    t = {k: to_dev(v) for k, v in inp.items()}
+    a = ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                      t["ctx_lens"], mode)
+    b = ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                      t["ctx_lens"], mode, flags=ba.ATTN_EARLY_KV)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
