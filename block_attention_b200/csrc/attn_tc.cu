@@ -30,10 +30,11 @@
 // 128-key S tiles: a tcgen05.mma with N = 64 costs the issuing thread as much
 // as one with N = 128, so the wider tile halves the MMA issue time per key.
 //
-// attn_tc_combine, grid (16 row groups, Hkv, B): merges the S partials of 8
-// query rows in split order (deterministic) and writes bf16 output.  Its CTAs
-// are small, so they start while the partial kernel drains, and the next
-// kernel in the stream can take the SMs the partial kernel frees.
+// attn_tc_combine, grid (8-row groups, Hkv, B): merges the S partials of each
+// query row (deterministic order) and writes bf16 output.  Its CTAs are small,
+// so they start while the partial kernel drains, and the next kernel in the
+// stream can take the SMs the partial kernel frees.  Partial O is stored as
+// bf16 (one extra rounding, relative 2^-9), halving the epilogue's stores.
 //
 // With ORTHRUS_ATTN_EARLY_KV the partial kernel reads ctx_lens and starts
 // streaming K/V tiles before waiting on the preceding kernel; Q and the block
@@ -62,7 +63,7 @@ constexpr int kThreads = 192;       // 6 warps
 constexpr int kTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256, 256+D)
 constexpr int kOCol = 256;
 constexpr float kLazyThresh = 8.f;  // log2 units
-constexpr int kMaxSplits = 32;
+constexpr int kMaxSplits = 24;     // the combine keeps every split's loads in registers
 constexpr int kGroupRows = 8;       // rows per combine CTA
 constexpr int kCombineThreads = 256;
 
@@ -76,9 +77,12 @@ constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 
-// One split's partial: O as [16 row groups][D/4][8 rows] float4, then m[128], l[128].
+// One split's partial, in 4-byte words: O as bf16 [16 row groups][D/4][8 rows]
+// x 4 values (8 bytes each), then m[128], l[128] as fp32.
 template <int kD>
-__host__ __device__ constexpr int part_floats() { return kRows * kD + 2 * kRows; }
+__host__ __device__ constexpr int part_floats() { return kRows * kD / 2 + 2 * kRows; }
+template <int kD>
+__host__ __device__ constexpr int part_ml() { return kRows * kD / 2; }
 
 struct __align__(64) TcParams {
   CUtensorMap tm_q;   // 3D (D, Hq, B*blk), box (64, G, blk)
@@ -202,6 +206,13 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
   // block tile, which the preceding kernel may still be writing).
   int early_issued = 0;
   int early_n = 0;
+  if (warp == 0 && lane == 0) {
+    for (int h = 0; h < halves; ++h) {
+      ptx::tma_prefetch_l2_3d(&p.tm_q, 64 * h, g * p.G, b * p.blk);
+      ptx::tma_prefetch_l2_3d(&p.tm_kb, 64 * h, g, b * p.blk);
+      ptx::tma_prefetch_l2_3d(&p.tm_vb, 64 * h, g, b * p.blk);
+    }
+  }
   if (p.early && warp == 0 && lane == 0) {
     early_n = p.ctx_lens[b];
     int Tc, t0, U;
@@ -212,6 +223,13 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     }
   }
   ptx::griddep_wait();
+  if (warp == 0 && lane == 0) {
+    // Q does not depend on the length: start it before reading ctx_lens
+    ptx::mbar_expect_tx(bars.q_full, (uint32_t)(halves * rows * 128));
+    for (int h = 0; h < halves; ++h)
+      ptx::tma_load_3d(q_s + h * (kRows * 128), &p.tm_q, bars.q_full, 64 * h, g * p.G,
+                       b * p.blk);
+  }
 
   const int n = p.ctx_lens[b];
   const bool bad = n < 0 || n > p.max_ctx;
@@ -236,10 +254,6 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     // ================================================== TMA producer
     if (lane == 0 && U > 0) {
       int issued = early_issued;
-      ptx::mbar_expect_tx(bars.q_full, (uint32_t)(halves * rows * 128));
-      for (int h = 0; h < halves; ++h)
-        ptx::tma_load_3d(q_s + h * (kRows * 128), &p.tm_q, bars.q_full, 64 * h, g * p.G,
-                         b * p.blk);
       for (int u = early_issued; u < U && !*abort_flag; ++u) {
         const int st = u % kStages;
         if (!ptx::mbar_wait(bars.empty[st], ((u / kStages) & 1) ^ 1)) {
@@ -253,8 +267,8 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
       for (int u = max(0, issued - kStages); u < issued; ++u)
         if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1))
           record_timeout(p.err, abort_flag);
-      if (!ptx::mbar_wait(bars.q_full, 0)) record_timeout(p.err, abort_flag);
     }
+    if (lane == 0 && !ptx::mbar_wait(bars.q_full, 0)) record_timeout(p.err, abort_flag);
   } else if (warp == 1) {
     // ================================================== MMA issuer
     if (lane == 0 && U > 0) {
@@ -405,21 +419,23 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     }
     if (have) ptx::tc_fence_after();
     const int rg = r / kGroupRows, ri = r % kGroupRows;
-    float4* po = reinterpret_cast<float4*>(part) + (int64_t)rg * (kD / 4) * kGroupRows + ri;
+    uint2* po = reinterpret_cast<uint2*>(part) + (int64_t)rg * (kD / 4) * kGroupRows + ri;
 #pragma unroll
     for (int cb = 0; cb < kD / 32; ++cb) {
       uint32_t o[32];
       if (have) ptx::tmem_ld32_sync(lane_addr + kOCol + cb * 32, o);
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
-        const float4 v = have ? make_float4(__uint_as_float(o[j]), __uint_as_float(o[j + 1]),
-                                            __uint_as_float(o[j + 2]), __uint_as_float(o[j + 3]))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        uint2 v = make_uint2(0u, 0u);
+        if (have) {
+          v.x = ptx::pack_bf16x2(__uint_as_float(o[j]), __uint_as_float(o[j + 1]));
+          v.y = ptx::pack_bf16x2(__uint_as_float(o[j + 2]), __uint_as_float(o[j + 3]));
+        }
         __stcg(po + (cb * 8 + j / 4) * kGroupRows, v);
       }
     }
-    __stcg(part + kRows * kD + r, have ? m_ref : -INFINITY);
-    __stcg(part + kRows * kD + kRows + r, have ? l : 0.f);
+    __stcg(part + part_ml<kD>() + r, have ? m_ref : -INFINITY);
+    __stcg(part + part_ml<kD>() + kRows + r, have ? l : 0.f);
   }
   __syncwarp();
   ptx::tc_fence_before();
@@ -430,64 +446,59 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
   }
 }
 
-// Merge the S split partials of 8 query rows, in split order, and write bf16.
+// Merge the S split partials of one 8-row group and write bf16.  One thread
+// per output item (4 dims of one row); consecutive lanes take consecutive
+// rows, so each split's slice is read as contiguous 256-byte runs, and every
+// split's loads are issued before any is used (one L2 round trip).  Splits
+// are merged in index order, so the result does not depend on timing.
 template <int kD>
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, 2)
 attn_tc_combine(const __grid_constant__ TcParams p) {
+  constexpr int kItemsPerRow = kD / 4;
   const int rg = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int it = threadIdx.x;  // item: (d4, row in group)
+  const int it = threadIdx.x;
+  const int d4 = it / kGroupRows, ri = it % kGroupRows;
+  const int r = rg * kGroupRows + ri;
   ptx::griddep_launch_dependents();
   ptx::griddep_wait();
   const int n = p.ctx_lens[b];
   if (n < 0 || n > p.max_ctx) return;  // reported by the partial kernel
-  if (it >= (kD / 4) * kGroupRows) return;
-  const int d4 = it / kGroupRows, ri = it % kGroupRows;
-  const int r = rg * kGroupRows + ri;
-  if (r >= p.G * p.blk) return;
+  if (d4 >= kItemsPerRow || r >= p.G * p.blk) return;
   const int S = p.S;
   const float* base = p.part + (int64_t)(b * p.Hkv + g) * S * part_floats<kD>();
-  const int64_t o_off = ((int64_t)rg * (kD / 4) + d4) * kGroupRows + ri;  // float4 index
-  float M = -INFINITY;
-  for (int s0 = 0; s0 < S; s0 += 8) {
-    float m8[8];
+  const int64_t o_off = ((int64_t)rg * kItemsPerRow + d4) * kGroupRows + ri;  // uint2 index
+  float ms[kMaxSplits], ls[kMaxSplits];
+  uint2 os[kMaxSplits];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      m8[k] = s0 + k < S ? __ldcg(base + (int64_t)(s0 + k) * part_floats<kD>() + kRows * kD + r)
-                         : -INFINITY;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) M = fmaxf(M, m8[k]);
-  }
-  float L = 0.f;
-  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < S; s0 += 8) {
-    float m8[8], l8[8];
-    float4 o8[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (s0 + k < S) {
-        const float* ps = base + (int64_t)(s0 + k) * part_floats<kD>();
-        m8[k] = __ldcg(ps + kRows * kD + r);
-        l8[k] = __ldcg(ps + kRows * kD + kRows + r);
-        o8[k] = __ldcg(reinterpret_cast<const float4*>(ps) + o_off);
-      }
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < S) {
+      const float* ps = base + (int64_t)s * part_floats<kD>();
+      ms[s] = __ldcg(ps + part_ml<kD>() + r);
+      ls[s] = __ldcg(ps + part_ml<kD>() + kRows + r);
+      os[s] = __ldcg(reinterpret_cast<const uint2*>(ps) + o_off);
     }
+  }
+  float M = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (s0 + k < S) {
-        const float w = M == -INFINITY ? 0.f : ptx::ex2(m8[k] - M);
-        L = fmaf(w, l8[k], L);
-        O.x = fmaf(w, o8[k].x, O.x);
-        O.y = fmaf(w, o8[k].y, O.y);
-        O.z = fmaf(w, o8[k].z, O.z);
-        O.w = fmaf(w, o8[k].w, O.w);
-      }
+  for (int s = 0; s < kMaxSplits; ++s)
+    if (s < S) M = fmaxf(M, ms[s]);
+  float L = 0.f, O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < S) {
+      const float w = M == -INFINITY ? 0.f : ptx::ex2(ms[s] - M);
+      L = fmaf(w, ls[s], L);
+      O0 = fmaf(w, __uint_as_float(os[s].x << 16), O0);
+      O1 = fmaf(w, __uint_as_float(os[s].x & 0xffff0000u), O1);
+      O2 = fmaf(w, __uint_as_float(os[s].y << 16), O2);
+      O3 = fmaf(w, __uint_as_float(os[s].y & 0xffff0000u), O3);
     }
   }
   const float inv = 1.f / L;
   const int i = r / p.G, h = g * p.G + r % p.G;
   uint2 pkd;
-  pkd.x = ptx::pack_bf16x2(O.x * inv, O.y * inv);
-  pkd.y = ptx::pack_bf16x2(O.z * inv, O.w * inv);
+  pkd.x = ptx::pack_bf16x2(O0 * inv, O1 * inv);
+  pkd.y = ptx::pack_bf16x2(O2 * inv, O3 * inv);
   *reinterpret_cast<uint2*>(p.out + ((int64_t)(b * p.blk + i) * p.Hq + h) * kD + 4 * d4) = pkd;
 }
 
@@ -604,7 +615,7 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   cudaError_t e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_partial<64>, p)
                             : cudaLaunchKernelEx(&cfg, attn_tc_partial<128>, p);
   if (e != cudaSuccess) return ORTHRUS_ECUDA;
-  cfg.gridDim = dim3(kRows / kGroupRows, a.Hkv, a.B);
+  cfg.gridDim = dim3(ceil_div(G * a.blk, kGroupRows), a.Hkv, a.B);
   cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   e = a.D == 64 ? cudaLaunchKernelEx(&cfg, attn_tc_combine<64>, p)
