@@ -11,6 +11,8 @@
 // which order CTAs finish.  Each CTA folds its key into the row's slot with
 // atomicMax; the last CTA of the row (ticket counter) decodes the key, writes
 // idx/maxval and returns the slot and the ticket to zero for the next call.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace orthrus {
@@ -131,3 +133,62 @@ cudaError_t launch_argmax(int dtype, const void* logits, int rows, int vocab,
 }
 
 }  // namespace orthrus
+
+// ---------------------------------------------------------------------------
+// Scratch-free variant of the argmax entry point.
+//
+// Some callers cannot allocate device memory for a workspace: code that runs
+// where no allocator is available or allowed (inside another library's
+// fixed memory budget, from a plugin handed only the tensors it works on, or
+// in a process whose device memory is already fully reserved).  For them the
+// argmax keeps its per-row scratch -- one 64-bit key and one ticket counter
+// per row -- in a file-scope device array that every GPU loading this
+// library holds until the process exits.
+namespace orthrus {
+namespace {
+
+constexpr int kNoAllocMaxRows = ORTHRUS_NOALLOC_ARGMAX_MAX_ROWS;
+constexpr size_t kNoAllocBytes = (size_t)kNoAllocMaxRows * 12;
+
+static __device__ __align__(256) unsigned char g_argmax_scratch[kNoAllocBytes];
+
+// Device address of g_argmax_scratch, looked up once per device (in host
+// code the symbol itself is only a host-side stand-in, never a device address).
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {nullptr};
+
+}  // namespace
+}  // namespace orthrus
+
+extern "C" int orthrus_vocab_argmax_noalloc(int32_t dtype, const void* logits, int32_t rows,
+                                            int32_t vocab, int64_t row_stride, int32_t* idx,
+                                            float* maxval, orthrus_stream_t stream) {
+  using namespace orthrus;
+  if (!(dtype == ORTHRUS_F32 || dtype == ORTHRUS_BF16) || rows < 0 || vocab <= 0 ||
+      row_stride < vocab)
+    return ORTHRUS_EINVAL;
+  if (rows > kNoAllocMaxRows) return ORTHRUS_EUNSUPPORTED;  // beyond the static scratch
+  if (rows == 0) return ORTHRUS_OK;
+  if (!logits || !idx) return ORTHRUS_EINVAL;
+  if (reinterpret_cast<uintptr_t>(logits) % (dtype == ORTHRUS_F32 ? 4 : 2)) return ORTHRUS_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ORTHRUS_ECUDA;
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_argmax_scratch) != cudaSuccess || !ptr)
+        return ORTHRUS_ECUDA;
+      g_scratch_ptr[dev] = ptr;
+    }
+    ws = g_scratch_ptr[dev];
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the rows' keys and tickets must start at zero (the kernel also leaves them zero)
+  if (cudaMemsetAsync(ws, 0, (size_t)rows * 12, st) != cudaSuccess) return ORTHRUS_ECUDA;
+  return launch_argmax(dtype, logits, rows, vocab, row_stride, idx, maxval, ws, st) ==
+                 cudaSuccess
+             ? ORTHRUS_OK
+             : ORTHRUS_ECUDA;
+}

@@ -149,6 +149,26 @@ int orthrus_vocab_argmax(int32_t dtype, const void* logits, int32_t rows,
                          float* maxval, void* workspace, size_t workspace_bytes,
                          orthrus_stream_t stream);
 
+/* Scratch-free variant of orthrus_vocab_argmax, for callers that cannot
+ * allocate device memory (no allocator available or allowed where they run,
+ * e.g. code handed only the tensors it works on, or a process whose device
+ * memory is fully reserved).  The pages describe no such entry point; it is
+ * a property of this library only.  Same arguments and results as
+ * orthrus_vocab_argmax minus the workspace: the per-row scratch (12 bytes a
+ * row) lives in a static device array of ORTHRUS_NOALLOC_ARGMAX_MAX_ROWS rows
+ * that every GPU loading the library holds until the process exits.
+ *   - rows > ORTHRUS_NOALLOC_ARGMAX_MAX_ROWS returns ORTHRUS_EUNSUPPORTED.
+ *   - Allocates nothing (no cudaMalloc/cudaFree); each call clears the rows it
+ *     uses with cudaMemsetAsync on `stream`, then launches the argmax kernel.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (other
+ *     streams, other threads) race and give wrong indices; serialise them. */
+#define ORTHRUS_NOALLOC_ARGMAX_MAX_ROWS 4096
+int orthrus_vocab_argmax_noalloc(int32_t dtype, const void* logits, int32_t rows,
+                                 int32_t vocab, int64_t row_stride, int32_t* idx,
+                                 float* maxval, orthrus_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Prefix consensus (explainer §四 step 3), per sequence b:
  *   accept_len[b]  = first j with draft[b,j] != verify[b,j], else blk
