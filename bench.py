@@ -34,6 +34,18 @@ METRIC = "block-attn HBM GB/s (% of peak) and consensus rounds/s, Qwen3-8B shape
 WORKLOAD = dict(name="qwen3_8b_round", layers=36, B=1, Hq=32, Hkv=8, D=128, ctx=8192,
                 blk=32, vocab=151936, dtype="bf16", logits_dtype="f32", accept_mean=5.4)
 FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes (read + write) of one block-attention call at this workload, from
+# the ncu capture summarised in profiles/attn_tc_partial_b8_ctx8192_full.md
+# (8-sequence case scaled to one sequence).  Valid only for the kernel source
+# it was measured on: reported as null once attn_tc.cu changes.
+TRAFFIC = {"attn_tc_sha256_prefix": "67000c0f6b677a6d", "bytes_per_call": 34766250}
+
+
+def measured_traffic():
+    import hashlib
+    src = os.path.join(ROOT, "block_attention_b200", "csrc", "attn_tc.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return TRAFFIC["bytes_per_call"] if h == TRAFFIC["attn_tc_sha256_prefix"] else None
 
 
 def peaks():
@@ -338,7 +350,7 @@ def main():
                        "us_per_launch": attn_launch_us, "bytes_per_launch": bytes_per_launch,
                        "launches_per_round": 2 * w["layers"]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "peak_source": src, "traffic": None,
+                     "frac": achieved / hbm, "peak_source": src, "traffic": measured_traffic(),
                      "kernel": "block_attn (both views, per-layer launches)"},
         "round_bytes": rb,
         "round_hbm_gbs": sum(rb.values()) / (total_ms / args.steps * 1e-3) / 1e9,
