@@ -11,6 +11,9 @@ Entry points (same names as the C ABI, minus the ``orthrus_`` prefix):
     vocab_argmax    per-row argmax, lowest index on ties
     consensus       accepted prefix, tokens to emit, next anchor
     kv_commit       copy accepted block K/V rows into every layer's cache
+and the row-invariant decoder building blocks of ``include/orthrus_decoder.h``
+(embed, rmsnorm, linear, qkv_rope, swiglu, block_tokens) that
+``block_attention_b200.decoder`` composes into the end-to-end consensus loop.
 """
 from __future__ import annotations
 
@@ -63,7 +66,10 @@ class CommitArgs(ctypes.Structure):
 EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_block_attn_launches", "orthrus_vocab_argmax",
            "orthrus_vocab_argmax_workspace", "orthrus_consensus", "orthrus_kv_commit",
-           "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version")
+           "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version",
+           # decoder building blocks (include/orthrus_decoder.h)
+           "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
+           "orthrus_swiglu", "orthrus_block_tokens")
 
 _lib = None
 
@@ -93,6 +99,13 @@ def lib() -> ctypes.CDLL:
         L.orthrus_status_str.argtypes = [c.c_int]
         L.orthrus_status_str.restype = c.c_char_p
         L.orthrus_version.restype = c.c_int
+        L.orthrus_embed.argtypes = [i32, vp, i32, i32, vp, i32, vp, vp, vp]
+        L.orthrus_rmsnorm.argtypes = [i32, vp, vp, i32, i32, c.c_float, vp, vp]
+        L.orthrus_linear.argtypes = [i32, vp, vp, vp, i32, i32, i32, vp, vp]
+        L.orthrus_qkv_rope.argtypes = [i32, vp, i32, i32, i32, i32, i32, vp, c.c_double,
+                                       vp, vp, vp, vp]
+        L.orthrus_swiglu.argtypes = [i32, vp, i32, i32, vp, vp]
+        L.orthrus_block_tokens.argtypes = [vp, vp, i32, i32, i32, vp, vp]
         _lib = L
     return _lib
 
@@ -192,9 +205,8 @@ def block_attn(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, *, out=No
                   max_ctx, err, flags)
     need = block_attn_workspace_bytes(a)
     if need:
-        # fp32 calls use the buffer as scratch; bf16 calls also keep zeroed
-        # ticket counters at its end: separate default buffers per dtype
-        buf = _ws(workspace, q.device, f"attn_{q.dtype}").get(need)
+        # scratch for the split partials; one default buffer per device
+        buf = _ws(workspace, q.device, "attn").get(need)
         a.workspace, a.workspace_bytes = buf.data_ptr(), buf.numel()
     _check("orthrus_block_attn", lib().orthrus_block_attn(ctypes.byref(a), _stream(stream)))
     return out
@@ -252,3 +264,72 @@ def kv_commit(k_cache, v_cache, k_blk, v_blk, ctx_lens, n_emit, *, err=None,
     a.workspace, a.workspace_bytes = buf.data_ptr(), buf.numel()
     _check("orthrus_kv_commit", lib().orthrus_kv_commit(ctypes.byref(a), _stream(stream)))
     return ctx_lens
+
+
+# ------------------------------------------------- decoder building blocks
+
+def embed(table, tokens, *, out=None, err=None, stream=None):
+    """out [rows, d] = table[tokens] (tokens int32 [rows])."""
+    _dev(table, tokens, out, err)
+    V, d = table.shape
+    rows = tokens.numel()
+    if out is None:
+        out = torch.empty(rows, d, dtype=table.dtype, device=table.device)
+    _check("orthrus_embed", lib().orthrus_embed(_dtype(table), _ptr(table), V, d, _ptr(tokens),
+                                                rows, _ptr(out), _ptr(err), _stream(stream)))
+    return out
+
+
+def rmsnorm(x, gain, eps, *, out=None, stream=None):
+    """Row-wise RMSNorm of x [rows, d] with gain [d] (out may be x)."""
+    _dev(x, gain, out)
+    d = x.shape[-1]
+    rows = x.numel() // d
+    if out is None:
+        out = torch.empty_like(x)
+    _check("orthrus_rmsnorm", lib().orthrus_rmsnorm(_dtype(x), _ptr(x), _ptr(gain), rows, d,
+                                                    float(eps), _ptr(out), _stream(stream)))
+    return out
+
+
+def linear(x, w, *, residual=None, out=None, stream=None):
+    """out [rows, N] = residual + x [rows, K] @ w[N, K]^T (out may be residual)."""
+    _dev(x, w, residual, out)
+    N, K = w.shape
+    rows = x.numel() // K
+    if out is None:
+        out = torch.empty(rows, N, dtype=x.dtype, device=x.device)
+    _check("orthrus_linear", lib().orthrus_linear(_dtype(x), _ptr(x), _ptr(w), _ptr(residual),
+                                                  rows, K, N, _ptr(out), _stream(stream)))
+    return out
+
+
+def qkv_rope(qkv, ctx_lens, B, blk, Hq, Hkv, hd, theta, *, q, k, v, stream=None):
+    """Split qkv [B*blk, (Hq+2Hkv)*hd] into q/k/v with RoPE at ctx_lens[b] + j."""
+    _dev(qkv, ctx_lens, q, k, v)
+    _check("orthrus_qkv_rope", lib().orthrus_qkv_rope(
+        _dtype(qkv), _ptr(qkv), B, blk, Hq, Hkv, hd, _ptr(ctx_lens), float(theta), _ptr(q),
+        _ptr(k), _ptr(v), _stream(stream)))
+    return q, k, v
+
+
+def swiglu(gu, *, out=None, stream=None):
+    """out [rows, F] = silu(gu[:, :F]) * gu[:, F:]."""
+    _dev(gu, out)
+    rows, F2 = gu.shape
+    if out is None:
+        out = torch.empty(rows, F2 // 2, dtype=gu.dtype, device=gu.device)
+    _check("orthrus_swiglu", lib().orthrus_swiglu(_dtype(gu), _ptr(gu), rows, F2 // 2,
+                                                  _ptr(out), _stream(stream)))
+    return out
+
+
+def block_tokens(anchor, draft, blk, mask_id, *, out=None, stream=None):
+    """[anchor, MASK...] (draft None) or [anchor, draft[:, :blk-1]] as int32 [B, blk]."""
+    _dev(anchor, draft, out)
+    B = anchor.numel()
+    if out is None:
+        out = torch.empty(B, blk, dtype=torch.int32, device=anchor.device)
+    _check("orthrus_block_tokens", lib().orthrus_block_tokens(
+        _ptr(anchor), _ptr(draft), B, blk, int(mask_id), _ptr(out), _stream(stream)))
+    return out

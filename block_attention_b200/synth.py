@@ -27,6 +27,9 @@ WORKLOADS = {
                      layers=36),
     "ragged": dict(B=16, Hq=32, Hkv=8, D=128, ctx_lo=1024, ctx_hi=32768, blk=32,
                    vocab=151936),
+    # end-to-end consensus loop on a random-init Qwen3-style decoder
+    "e2e_decoder": dict(V=8192, d=512, L=4, Hq=8, Hkv=4, hd=64, ffn=1536, std=0.02,
+                        prompts=256, prompt_lo=64, prompt_hi=512, n_new=256, blk=32),
 }
 
 # Stream ids, one per kind of tensor.

@@ -25,10 +25,12 @@
  *     device can see (a device-resident length out of range) set the optional
  *     device error word `err` (first error code wins) and skip the affected
  *     sequence's writes; kernels never trap.
- *   - Workspaces: query the size, allocate it once, zero it once
- *     (cudaMemset 0).  Kernels leave their ticket counters at zero again, so
- *     the same workspace serves every later call on the same stream.  After a
- *     call that reported an error, zero it again.
+ *   - Workspaces: query the size and allocate it once.  Argmax and commit
+ *     workspaces hold ticket counters: zero them once (cudaMemset 0); the
+ *     kernels leave the counters at zero again, so the buffer serves every
+ *     later call on the same stream (zero it again after a call that reported
+ *     an error).  The block-attention workspace is scratch only.  Calls that
+ *     may run at the same time (different streams) need separate workspaces.
  *   - Tensors are dense, row-major, with the layouts written next to each
  *     field.  dtype applies to every floating-point tensor of a call.
  */
@@ -114,16 +116,15 @@ typedef struct orthrus_attn_args {
   void* out;           /* [B, blk, Hq, D], same dtype as q */
   int32_t* err;        /* optional device int32 error word (NULL = none) */
   void* workspace;     /* >= orthrus_block_attn_workspace() bytes, 256-byte aligned,
-                          zero-initialised once (see below) */
+                          scratch (see below) */
   size_t workspace_bytes; /* size of the caller's buffer */
 } orthrus_attn_args;
 
-/* Workspace of orthrus_block_attn.  BF16 calls keep 16*B*Hkv bytes of ticket
- * counters at the END of the buffer (last workspace_bytes) and use the front
- * as scratch; every call leaves its counters at zero.  One buffer, zeroed
- * once, may serve any sequence of BF16 calls on one stream whose sizes fit it.
- * FP32 calls use the buffer as scratch only: give FP32 and BF16 calls
- * separate buffers. */
+/* Workspace of orthrus_block_attn: scratch for the per-split partial results
+ * of the split-KV reduction (unnormalised O plus row max and row sum), written
+ * and read back within the call; it needs no initialisation and carries
+ * nothing from one call to the next.  One buffer may serve any sequence of
+ * FP32 and BF16 calls on one stream whose sizes fit it. */
 
 /* Bytes of workspace orthrus_block_attn needs for these arguments (0 if none).
  * Pointers in `a` are not read.  Returns 0 for invalid shapes as well. */

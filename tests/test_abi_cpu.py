@@ -1,5 +1,5 @@
 """CPU-only checks of the C ABI: the library loads, exports every function
-include/orthrus.h declares, the ctypes structs match the C layout, and
+the headers under include/ declare, the ctypes structs match the C layout, and
 host-side argument checks return their status codes without launching
 anything (no GPU is touched by these calls)."""
 import ctypes
@@ -13,7 +13,8 @@ import block_attention_b200 as ba
 from block_attention_b200 import build as ba_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "orthrus.h")
+INCLUDE = os.path.join(ROOT, "include")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -23,9 +24,11 @@ def L():
 
 
 def _declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(orthrus_\w+)\s*\(", src)))
+    names = set()
+    for h in HEADERS:
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(orthrus_\w+)\s*\(", src))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
@@ -141,3 +144,30 @@ def test_python_binding_refuses_cpu_tensors():
     x = torch.zeros(2, 8)
     with pytest.raises(ValueError):
         ba.vocab_argmax(x)
+
+
+def test_decoder_entry_points_host_checks(L):
+    c = ctypes
+    vp = c.c_void_p
+    # bad dtype, negative sizes and null pointers are refused before any launch
+    assert L.orthrus_embed(5, vp(256), 10, 8, vp(256), 2, vp(256), None, None) == -1
+    assert L.orthrus_embed(0, None, 10, 8, None, 0, None, None, None) == 0
+    assert L.orthrus_embed(0, None, 10, 8, vp(256), 2, vp(256), None, None) == -1
+    assert L.orthrus_rmsnorm(0, vp(256), vp(256), 2, 0, c.c_float(1e-6), vp(256), None) == -1
+    assert L.orthrus_rmsnorm(0, vp(256), vp(256), 2, 8, c.c_float(float("nan")), vp(256),
+                             None) == -1
+    assert L.orthrus_rmsnorm(1, None, None, 0, 8, c.c_float(1e-6), None, None) == 0
+    assert L.orthrus_linear(0, vp(256), vp(512), None, 4, 0, 8, vp(1024), None) == -1
+    assert L.orthrus_linear(0, vp(256), vp(512), None, 4, 8, 8, vp(256), None) == -1  # out == x
+    assert L.orthrus_linear(0, None, None, None, 0, 8, 8, None, None) == 0
+    assert L.orthrus_linear(0, vp(256), vp(512), None, 128 * 65536, 8, 8, vp(1024),
+                            None) == -2
+    assert L.orthrus_qkv_rope(0, vp(256), 1, 4, 2, 1, 7, vp(256), c.c_double(1e6), vp(256),
+                              vp(256), vp(256), None) == -1  # odd head dim
+    assert L.orthrus_qkv_rope(0, vp(256), 1, 4, 2, 1, 8, vp(256), c.c_double(0.0), vp(256),
+                              vp(256), vp(256), None) == -1  # theta <= 0
+    assert L.orthrus_swiglu(0, vp(256), 2, 0, vp(256), None) == -1
+    assert L.orthrus_swiglu(0, None, 0, 8, None, None) == 0
+    assert L.orthrus_block_tokens(vp(256), None, 1, 33, 0, vp(256), None) == -1
+    assert L.orthrus_block_tokens(None, None, 1, 32, 0, vp(256), None) == -1
+    assert L.orthrus_block_tokens(None, None, 0, 32, 0, None, None) == 0
