@@ -224,6 +224,41 @@ def kernel_alone(args):
 
 # ---------------------------------------------------------------- GPU arm
 
+def decoder_report():
+    """The end-to-end consensus loop on the random-init decoder (4 layers,
+    d_model 512, Hq 8, Hkv 4, head dim 64, SwiGLU 1536, vocab 8192; 256
+    prompts of U{64..512} random tokens, 256 greedy tokens each): FP32 loop
+    against FP32 greedy (must be exact), BF16 trajectory-match rates, tokens
+    per forward.  Runs after the timed regions; it times nothing of the bench."""
+    import torch
+    from block_attention_b200 import synth
+    from block_attention_b200.decoder import TinyDecoder, trajectory_report
+    E = synth.WORKLOADS["e2e_decoder"]
+    seed = 1004
+    W = synth.decoder_weights(E["V"], E["d"], E["L"], E["Hq"], E["Hkv"], E["hd"], E["ffn"],
+                              seed=seed, std=E["std"])
+    prompts = synth.prompts(E["prompts"], E["V"], E["prompt_lo"], E["prompt_hi"], seed=seed,
+                            exclude=E["V"] - 1)
+    t0 = time.perf_counter()
+    rep = {"workload": "random-init decoder L4 d512 Hq8 Hkv4 hd64 ffn1536 V8192; "
+                       "256 prompts U{64..512}, 256 new tokens, block 32"}
+    out = {}
+    for name, dt in (("fp32", torch.float32), ("bf16", torch.bfloat16)):
+        m = TinyDecoder(W, E["Hq"], E["Hkv"], E["hd"], dtype=dt)
+        out[name + "_greedy"] = m.greedy(prompts, E["n_new"])
+        toks, st = m.consensus(prompts, E["n_new"], blk=E["blk"])
+        out[name + "_loop"] = toks
+        rep.setdefault("tokens_per_forward", {})[name] = st["tokens_per_forward"]
+        del m
+    rep["fp32_loop_vs_fp32_greedy"] = trajectory_report(out["fp32_loop"], out["fp32_greedy"])
+    rep["bf16_loop_vs_fp32_greedy"] = trajectory_report(out["bf16_loop"], out["fp32_greedy"])
+    rep["bf16_loop_vs_bf16_greedy"] = trajectory_report(out["bf16_loop"], out["bf16_greedy"])
+    rep["bf16_greedy_vs_fp32_greedy"] = trajectory_report(out["bf16_greedy"],
+                                                          out["fp32_greedy"])
+    rep["seconds"] = time.perf_counter() - t0
+    return rep
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -231,6 +266,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e-decoder", action="store_true",
+                    help="skip the end-to-end decoder report (runs after the timing)")
     ap.add_argument("--kernel", choices=["attn"], default=None,
                     help="time one kernel alone on a case larger than L2 (for profiling)")
     args = ap.parse_args()
@@ -334,6 +371,10 @@ def main():
         cpu = {"value": v, "unit": "rounds/s", "cores": cores, "kind": "oracle",
                "sample": sample}
 
+    dec = None
+    if rank == 0 and world == 1 and not args.no_e2e_decoder:
+        dec = decoder_report()
+
     if world > 1:
         dist.barrier()
         rnd.graphs = None
@@ -360,6 +401,7 @@ def main():
         "gpu_launches": gpu_launches,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "e2e_decoder": dec,
     }
     print(json.dumps(line), flush=True)
 

@@ -18,15 +18,26 @@
 // cache[0, n) of a (sequence, kv-head) are cut into 128-key tiles, followed by
 // one tile holding the blk block rows; the tiles are dealt out contiguously
 // over the S splits.  Per CTA:
-//   warp 0      TMA producer: Q once, then K/V tiles through a 3 x 64 KB ring
+//   warp 0      TMA producers: lane 0 streams K tiles, lane 1 V tiles, through
+//               a 3-stage ring (32 KB of K + 32 KB of V per stage); a K slot
+//               is refilled as soon as its S = Q K^T product has read it, a V
+//               slot once its P V product has
 //   warp 1      MMA issuer (one thread): S = Q K^T (M=128, N=128 per
-//               instruction) into a double-buffered TMEM tile, then O += P V
-//               with P read from TMEM
-//   warps 2..5  softmax, one query row per thread: online softmax with lazy
+//               instruction, Q read from TMEM) into a double-buffered TMEM
+//               tile, and O += P V with P read from TMEM.  Once P(u) is ready
+//               the 8 instructions of P(u) V(u) go out, then the 8 of S(u+2):
+//               each product is a chain of dependent accumulations, and the
+//               second chain overlaps the tail of the first in the tensor pipe
+//   warps 2..5  softmax, one query row per thread: first they copy Q from
+//               shared memory into TMEM; per tile, online softmax with lazy
 //               rescaling (O in TMEM is rescaled only when a row's running
-//               maximum grows by more than 2^8), P written back to TMEM as
-//               bf16; finally the split's unnormalised O, row max and row sum
-//               go to an L2-resident workspace.
+//               maximum grows by more than 2^8), P written to its own TMEM
+//               buffer as bf16; finally the split's unnormalised O, row max
+//               and row sum go to an L2-resident workspace.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+D) Q (bf16 pairs,
+// D/2 columns) and P (64 columns) after it.  Operands read from TMEM leave
+// shared-memory bandwidth to the TMA stream: per tile the tensor pipe reads
+// only the K and V tiles from shared memory.
 // 128-key S tiles: a tcgen05.mma with N = 64 costs the issuing thread as much
 // as one with N = 128, so the wider tile halves the MMA issue time per key.
 //
@@ -60,8 +71,9 @@ constexpr int kRows = 128;          // UMMA M
 constexpr int kTile = 128;          // keys per tile (UMMA N of S = Q K^T)
 constexpr int kStages = 3;          // K/V ring depth
 constexpr int kThreads = 192;       // 6 warps
-constexpr int kTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256, 256+D)
+constexpr int kTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256,256+D) Q, P after it
 constexpr int kOCol = 256;
+static_assert(kOCol + 128 + 64 + kTile / 2 <= kTmemCols, "TMEM columns at D = 128");
 constexpr float kLazyThresh = 8.f;  // log2 units
 constexpr int kMaxSplits = 24;     // the combine keeps every split's loads in registers
 constexpr int kGroupRows = 8;       // rows per combine CTA
@@ -73,7 +85,7 @@ constexpr int kQBytes = 2 * kRows * 128;    // two 64-dim halves, 128 B rows
 constexpr int kStageBytes = 4 * kHalfTile;  // K (2 halves) + V (2 halves)
 constexpr int kRingOff = kQBytes;
 constexpr int kBarOff = kRingOff + kStages * kStageBytes;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+constexpr int kNumBars = 9 + 4 * kStages;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
 constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
 
@@ -98,8 +110,20 @@ struct __align__(64) TcParams {
   float scale_log2;
 };
 
+// mbarrier addresses, laid out consecutively from `base` (8 bytes each)
 struct Bars {
-  uint32_t q_full, full[kStages], empty[kStages], s_full[2], p_full[2], pv_done[2], mma_done;
+  uint32_t base;
+  __device__ uint32_t at(int i) const { return base + 8 * i; }
+  __device__ uint32_t q_full() const { return at(0); }   // Q landed in shared memory
+  __device__ uint32_t q_tmem() const { return at(1); }   // Q copied into TMEM
+  __device__ uint32_t k_full(int s) const { return at(2 + s); }
+  __device__ uint32_t v_full(int s) const { return at(2 + kStages + s); }
+  __device__ uint32_t k_empty(int s) const { return at(2 + 2 * kStages + s); }
+  __device__ uint32_t v_empty(int s) const { return at(2 + 3 * kStages + s); }
+  __device__ uint32_t s_full(int b) const { return at(2 + 4 * kStages + b); }
+  __device__ uint32_t p_full(int b) const { return at(4 + 4 * kStages + b); }
+  __device__ uint32_t pv_done(int b) const { return at(6 + 4 * kStages + b); }
+  __device__ uint32_t mma_done() const { return at(8 + 4 * kStages); }
 };
 
 __device__ __forceinline__ void record_timeout(int32_t* err, volatile int* abort_flag) {
@@ -111,6 +135,8 @@ template <int kD>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_partial(const __grid_constant__ TcParams p) {
   constexpr int halves = kD / 64;
+  constexpr uint32_t kQCol = kOCol + kD;           // Q as bf16 pairs, D/2 columns
+  constexpr uint32_t kPCol = kOCol + kD + kD / 2;  // P as bf16 pairs, 64 columns
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -120,17 +146,7 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
   const int S = p.S;
   const unsigned full_mask = 0xffffffffu;
 
-  Bars bars;
-  {
-    uint32_t a = sbase + kBarOff;
-    bars.q_full = a; a += 8;
-    for (int s = 0; s < kStages; ++s) { bars.full[s] = a; a += 8; }
-    for (int s = 0; s < kStages; ++s) { bars.empty[s] = a; a += 8; }
-    for (int s = 0; s < 2; ++s) { bars.s_full[s] = a; a += 8; }
-    for (int s = 0; s < 2; ++s) { bars.p_full[s] = a; a += 8; }
-    for (int s = 0; s < 2; ++s) { bars.pv_done[s] = a; a += 8; }
-    bars.mma_done = a;
-  }
+  const Bars bars{sbase + kBarOff};
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kMiscOff + 8);
   const int rows = p.G * p.blk;
@@ -138,17 +154,20 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
   // ---- setup that reads nothing a preceding kernel writes
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    ptx::mbar_init(bars.q_full, 1);
+    ptx::mbar_init(bars.q_full(), 1);
+    ptx::mbar_init(bars.q_tmem(), 128);
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(bars.full[s], 1);
-      ptx::mbar_init(bars.empty[s], 1);
+      ptx::mbar_init(bars.k_full(s), 1);
+      ptx::mbar_init(bars.v_full(s), 1);
+      ptx::mbar_init(bars.k_empty(s), 1);
+      ptx::mbar_init(bars.v_empty(s), 1);
     }
     for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(bars.s_full[s], 1);
-      ptx::mbar_init(bars.p_full[s], 128);
-      ptx::mbar_init(bars.pv_done[s], 1);
+      ptx::mbar_init(bars.s_full(s), 1);
+      ptx::mbar_init(bars.p_full(s), 128);
+      ptx::mbar_init(bars.pv_done(s), 1);
     }
-    ptx::mbar_init(bars.mma_done, 1);
+    ptx::mbar_init(bars.mma_done(), 1);
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -186,19 +205,21 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     t0 = (int)(((int64_t)split * T) / S);
     U = (int)(((int64_t)(split + 1) * T) / S) - t0;
   };
-  auto issue_tile = [&](int u, int t, int Tc) {
+  // K (is_v false) or V half of tile t into ring slot u % kStages
+  auto issue = [&](bool is_v, int u, int t, int Tc) {
     const int st = u % kStages;
     const bool blk_tile = t == Tc;
     const int rows_ld = blk_tile ? p.blk : kTile;
-    ptx::mbar_expect_tx(bars.full[st], (uint32_t)(2 * halves * rows_ld * 128));
+    const uint32_t bar = is_v ? bars.v_full(st) : bars.k_full(st);
+    const uint32_t dst = is_v ? v_s(st) : k_s(st);
+    ptx::mbar_expect_tx(bar, (uint32_t)(halves * rows_ld * 128));
     for (int h = 0; h < halves; ++h) {
-      if (blk_tile) {
-        ptx::tma_load_3d(k_s(st) + h * kHalfTile, &p.tm_kb, bars.full[st], 64 * h, g, b * p.blk);
-        ptx::tma_load_3d(v_s(st) + h * kHalfTile, &p.tm_vb, bars.full[st], 64 * h, g, b * p.blk);
-      } else {
-        ptx::tma_load_2d(k_s(st) + h * kHalfTile, &p.tm_kc, bars.full[st], 64 * h, slab + t * kTile);
-        ptx::tma_load_2d(v_s(st) + h * kHalfTile, &p.tm_vc, bars.full[st], 64 * h, slab + t * kTile);
-      }
+      if (blk_tile)
+        ptx::tma_load_3d(dst + h * kHalfTile, is_v ? &p.tm_vb : &p.tm_kb, bar, 64 * h, g,
+                         b * p.blk);
+      else
+        ptx::tma_load_2d(dst + h * kHalfTile, is_v ? &p.tm_vc : &p.tm_kc, bar, 64 * h,
+                         slab + t * kTile);
     }
   };
 
@@ -218,16 +239,17 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     int Tc, t0, U;
     geometry(early_n, Tc, t0, U);
     while (early_issued < min(U, kStages) && t0 + early_issued < Tc) {
-      issue_tile(early_issued, t0 + early_issued, Tc);
+      issue(false, early_issued, t0 + early_issued, Tc);
+      issue(true, early_issued, t0 + early_issued, Tc);
       ++early_issued;
     }
   }
   ptx::griddep_wait();
   if (warp == 0 && lane == 0) {
     // Q does not depend on the length: start it before reading ctx_lens
-    ptx::mbar_expect_tx(bars.q_full, (uint32_t)(halves * rows * 128));
+    ptx::mbar_expect_tx(bars.q_full(), (uint32_t)(halves * rows * 128));
     for (int h = 0; h < halves; ++h)
-      ptx::tma_load_3d(q_s + h * (kRows * 128), &p.tm_q, bars.q_full, 64 * h, g * p.G,
+      ptx::tma_load_3d(q_s + h * (kRows * 128), &p.tm_q, bars.q_full(), 64 * h, g * p.G,
                        b * p.blk);
   }
 
@@ -240,77 +262,100 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     // the EARLY_KV contract was broken (the length changed under us): drain
     // the early loads and produce nothing for this split
     for (int u = 0; u < early_issued; ++u)
-      if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1))
+      if (!ptx::mbar_wait(bars.k_full(u % kStages), (u / kStages) & 1) ||
+          !ptx::mbar_wait(bars.v_full(u % kStages), (u / kStages) & 1))
         record_timeout(p.err, abort_flag);
     set_err(p.err, ORTHRUS_EINVAL);
     *abort_flag = 1;
     early_issued = 0;
   }
+  // lane 0 issued the early tiles: both producer lanes start after them
+  if (warp == 0) early_issued = __shfl_sync(full_mask, early_issued, 0);
   __syncthreads();
   if (*abort_flag) U = 0;
   float* part = p.part + ((int64_t)(b * p.Hkv + g) * S + split) * part_floats<kD>();
 
   if (warp == 0) {
-    // ================================================== TMA producer
-    if (lane == 0 && U > 0) {
+    // ================================================== TMA producers
+    if (lane < 2 && U > 0) {
+      const bool is_v = lane == 1;
       int issued = early_issued;
       for (int u = early_issued; u < U && !*abort_flag; ++u) {
         const int st = u % kStages;
-        if (!ptx::mbar_wait(bars.empty[st], ((u / kStages) & 1) ^ 1)) {
+        const uint32_t empty = is_v ? bars.v_empty(st) : bars.k_empty(st);
+        if (!ptx::mbar_wait(empty, ((u / kStages) & 1) ^ 1)) {
           record_timeout(p.err, abort_flag);
           break;
         }
-        issue_tile(u, t0 + u, Tc);
+        issue(is_v, u, t0 + u, Tc);
         issued = u + 1;
       }
       // drain: every issued load must have landed before the CTA exits
-      for (int u = max(0, issued - kStages); u < issued; ++u)
-        if (!ptx::mbar_wait(bars.full[u % kStages], (u / kStages) & 1))
-          record_timeout(p.err, abort_flag);
+      for (int u = max(0, issued - kStages); u < issued; ++u) {
+        const uint32_t full = is_v ? bars.v_full(u % kStages) : bars.k_full(u % kStages);
+        if (!ptx::mbar_wait(full, (u / kStages) & 1)) record_timeout(p.err, abort_flag);
+      }
     }
-    if (lane == 0 && !ptx::mbar_wait(bars.q_full, 0)) record_timeout(p.err, abort_flag);
+    if (lane == 0 && !ptx::mbar_wait(bars.q_full(), 0)) record_timeout(p.err, abort_flag);
   } else if (warp == 1) {
     // ================================================== MMA issuer
     if (lane == 0 && U > 0) {
       const uint32_t id_s = ptx::idesc_bf16(kRows, kTile, false, false);
       const uint32_t id_pv = ptx::idesc_bf16(kRows, kD, false, true);
-      bool ok = ptx::mbar_wait(bars.q_full, 0);
-      auto pv = [&](int u) -> bool {
-        const int buf = u & 1, st = u % kStages;
-        if (!ptx::mbar_wait(bars.p_full[buf], (u >> 1) & 1)) return false;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kTile / 16; ++k) {
-          // V tile as the MN-major B operand: 8-key groups 1024 B apart,
-          // 64-dim halves kHalfTile apart
-          const uint64_t bd = ptx::sdesc_sw128(v_s(st) + k * 2048, kHalfTile, 1024);
-          ptx::mma_ts(tmem + kOCol, tmem + buf * kTile + k * 8, bd, id_pv,
-                      (u > 0 || k > 0) ? 1u : 0u);
-        }
-        ptx::tc_commit(bars.pv_done[buf]);
-        ptx::tc_commit(bars.empty[st]);
-        return true;
+      // S(u) = Q K(u)^T into S buffer u & 1 (dims in 16-wide steps k), and
+      // O += P(u) V(u) (keys in 16-wide steps k); S(u + 2) reuses the buffer
+      // of S(u), which the softmax has read before it published P(u)
+      auto s_step = [&](int u, int k) {
+        const int st = u % kStages;
+        const uint32_t h = k >> 2, kk = k & 3;  // 64-dim half, 16-dim step in it
+        const uint64_t bd = ptx::sdesc_sw128(k_s(st) + h * kHalfTile + kk * 32, 16, 1024);
+        ptx::mma_ts(tmem + (u & 1) * kTile, tmem + kQCol + k * 8, bd, id_s, k > 0 ? 1u : 0u);
       };
-      for (int u = 0; ok && u < U && !*abort_flag; ++u) {
-        const int buf = u & 1, st = u % kStages;
-        if (!ptx::mbar_wait(bars.full[st], (u / kStages) & 1)) { ok = false; break; }
-        if (u >= 2 && !ptx::mbar_wait(bars.pv_done[buf], ((u - 2) >> 1) & 1)) { ok = false; break; }
+      auto pv_step = [&](int u, int k) {
+        // V tile as the MN-major B operand: 8-key groups 1024 B apart,
+        // 64-dim halves kHalfTile apart
+        const uint64_t bd = ptx::sdesc_sw128(v_s(u % kStages) + k * 2048, kHalfTile, 1024);
+        ptx::mma_ts(tmem + kOCol, tmem + kPCol + k * 8, bd, id_pv, (u > 0 || k > 0) ? 1u : 0u);
+      };
+      auto s_done = [&](int u) {
+        ptx::tc_commit(bars.s_full(u & 1));
+        ptx::tc_commit(bars.k_empty(u % kStages));
+      };
+      bool ok = ptx::mbar_wait(bars.q_tmem(), 0);
+      // S(0) and S(1): two independent chains, back to back
+      for (int u = 0; ok && u < min(U, 2); ++u) {
+        if (!ptx::mbar_wait(bars.k_full(u % kStages), (u / kStages) & 1)) { ok = false; break; }
         ptx::tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k) {
-          const uint32_t h = k >> 2, kk = k & 3;  // 64-dim half, 16-dim step in it
-          const uint64_t ad = ptx::sdesc_sw128(q_s + h * (kRows * 128) + kk * 32, 16, 1024);
-          const uint64_t bd = ptx::sdesc_sw128(k_s(st) + h * kHalfTile + kk * 32, 16, 1024);
-          ptx::mma_ss(tmem + buf * kTile, ad, bd, id_s, k > 0 ? 1u : 0u);
-        }
-        ptx::tc_commit(bars.s_full[buf]);
-        if (u >= 1 && !pv(u - 1)) { ok = false; break; }
+        for (int k = 0; k < kD / 16; ++k) s_step(u, k);
+        s_done(u);
       }
-      if (ok && !*abort_flag) ok = pv(U - 1);
+      for (int u = 0; ok && u < U && !*abort_flag; ++u) {
+        const int st = u % kStages, nx = u + 2;
+        const bool with_s = nx < U;
+        if (!ptx::mbar_wait(bars.v_full(st), (u / kStages) & 1) ||
+            !ptx::mbar_wait(bars.p_full(u & 1), (u >> 1) & 1) ||
+            (with_s && !ptx::mbar_wait(bars.k_full(nx % kStages), (nx / kStages) & 1))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        // P(u) V(u) first and committed on its own: the softmax waits on it
+        // before writing P(u + 1); S(u + 2) is needed only a tile later
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k) pv_step(u, k);
+        ptx::tc_commit(bars.pv_done(u & 1));
+        ptx::tc_commit(bars.v_empty(st));
+        if (with_s) {
+#pragma unroll
+          for (int k = 0; k < kD / 16; ++k) s_step(nx, k);
+          s_done(nx);
+        }
+      }
       if (!ok) record_timeout(p.err, abort_flag);
       // every MMA issued so far has finished before TMEM is released
-      ptx::tc_commit(bars.mma_done);
-      if (!ptx::mbar_wait(bars.mma_done, 0)) record_timeout(p.err, abort_flag);
+      ptx::tc_commit(bars.mma_done());
+      if (!ptx::mbar_wait(bars.mma_done(), 0)) record_timeout(p.err, abort_flag);
     }
   } else {
     // ================================================== softmax
@@ -319,19 +364,42 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     const int i_blk = r < rows ? r / p.G : p.blk;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const int sm_tid = threadIdx.x - 64;  // 0..127
-    const float c = p.scale_log2;
+    const float c = p.scale_log2;         // > 0 (checked on the host)
     float m_ref = -INFINITY, l = 0.f;
-    bool alive = true;
-    for (int u = 0; u < U; ++u) {
+    bool alive = U > 0;
+    // Q row r -> TMEM columns [kQCol, kQCol + D/2) as bf16 pairs; in shared
+    // memory the row's 16-byte chunks sit 128-byte swizzled (chunk j at j ^ (r & 7))
+    if (alive) {
+      if (!__all_sync(full_mask, ptx::mbar_wait(bars.q_full(), 0))) {
+        record_timeout(p.err, abort_flag);
+        alive = false;
+      }
+#pragma unroll
+      for (int h = 0; h < halves; ++h) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(smem + h * (kRows * 128) + r * 128 +
+                                                           ((j ^ (r & 7)) << 4));
+          qv[4 * j] = q4.x; qv[4 * j + 1] = q4.y; qv[4 * j + 2] = q4.z; qv[4 * j + 3] = q4.w;
+        }
+        ptx::tmem_st32(lane_addr + kQCol + h * 32, qv);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bars.q_tmem());
+    }
+    for (int u = 0; alive && u < U; ++u) {
       if (__any_sync(full_mask, *abort_flag != 0)) { alive = false; break; }
       const int t = t0 + u, buf = u & 1, st = u % kStages;
-      if (!__all_sync(full_mask, ptx::mbar_wait(bars.s_full[buf], (u >> 1) & 1))) {
+      if (!__all_sync(full_mask, ptx::mbar_wait(bars.s_full(buf), (u >> 1) & 1))) {
         record_timeout(p.err, abort_flag); alive = false; break;
       }
       ptx::tc_fence_after();
       uint32_t sv[4][32];
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) ptx::tmem_ld32_sync(lane_addr + buf * kTile + cb * 32, sv[cb]);
+      for (int cb = 0; cb < 4; ++cb) ptx::tmem_ld32(lane_addr + buf * kTile + cb * 32, sv[cb]);
+      ptx::tmem_wait_ld();
       const bool blk_tile = t == Tc;
       const int nv_tile = blk_tile ? p.blk : min(kTile, n - t * kTile);
       int nv = nv_tile;
@@ -351,14 +419,37 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
         for (int j = 0; j < 32; ++j) mt[cb] = fmaxf(mt[cb], __uint_as_float(sv[cb][j]));
       const float ms = fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3])) * c;
       const bool need = ms > m_ref + kLazyThresh;
-      if (__any_sync(full_mask, need)) {
+      const bool rescale = __any_sync(full_mask, need);
+      float f = 1.f;
+      if (rescale) {
         const float m_new = need ? ms : m_ref;
-        const float f = ptx::ex2(m_ref - m_new);  // 0 for the first tile, 1 if unchanged
-        if (u > 0) {
-          if (!__all_sync(full_mask, ptx::mbar_wait(bars.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1))) {
-            record_timeout(p.err, abort_flag); alive = false; break;
-          }
-          ptx::tc_fence_after();
+        f = ptx::ex2(m_ref - m_new);  // 0 for the first tile, 1 if unchanged
+        m_ref = m_new;
+      }
+      // P = 2^(s*c - m_ref) as bf16 pairs; ex2(-inf) = 0 for masked keys
+      const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half][2 * j]), c, nm));
+          const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half][2 * j + 1]), c, nm));
+          const float p2 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half + 1][2 * j]), c, nm));
+          const float p3 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half + 1][2 * j + 1]), c, nm));
+          ls[0] += p0; ls[1] += p1; ls[2] += p2; ls[3] += p3;
+          pk[half][j] = ptx::pack_bf16x2(p0, p1);
+          pk[half][16 + j] = ptx::pack_bf16x2(p2, p3);
+        }
+      l = l * f + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+      // P(u - 1) V(u - 1) must be done: it reads the P buffer and adds into O
+      if (u > 0) {
+        if (!__all_sync(full_mask, ptx::mbar_wait(bars.pv_done((u - 1) & 1), ((u - 1) >> 1) & 1))) {
+          record_timeout(p.err, abort_flag); alive = false; break;
+        }
+        ptx::tc_fence_after();
+        if (rescale) {
 #pragma unroll
           for (int cb = 0; cb < kD / 32; ++cb) {
             uint32_t o[32];
@@ -367,36 +458,15 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
             ptx::tmem_st32(lane_addr + kOCol + cb * 32, o);
           }
-          ptx::tmem_wait_st();
         }
-        l *= f;
-        m_ref = m_new;
       }
-      // P = 2^(s*c - m_ref) as bf16 pairs into the first 64 columns of this S
-      // buffer; ex2(-inf) = 0 for masked keys
-      const float nm = -m_ref;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half][2 * j]), c, nm));
-          const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half][2 * j + 1]), c, nm));
-          const float p2 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half + 1][2 * j]), c, nm));
-          const float p3 = ptx::ex2(fmaf(__uint_as_float(sv[2 * half + 1][2 * j + 1]), c, nm));
-          ls[0] += p0; ls[1] += p1; ls[2] += p2; ls[3] += p3;
-          pk[j] = ptx::pack_bf16x2(p0, p1);
-          pk[16 + j] = ptx::pack_bf16x2(p2, p3);
-        }
-        ptx::tmem_st32(lane_addr + buf * kTile + half * 32, pk);
-      }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      ptx::tmem_st32(lane_addr + kPCol, pk[0]);
+      ptx::tmem_st32(lane_addr + kPCol + 32, pk[1]);
       ptx::tmem_wait_st();
       if (nv_tile < kTile) {
         // rows past the valid keys hold stale or foreign data: zero them in V
         // so 0 * garbage cannot reach O
-        if (!__all_sync(full_mask, ptx::mbar_wait(bars.full[st], (u / kStages) & 1))) {
+        if (!__all_sync(full_mask, ptx::mbar_wait(bars.v_full(st), (u / kStages) & 1))) {
           record_timeout(p.err, abort_flag); alive = false; break;
         }
         const int nz = (kTile - nv_tile) * 8 * halves;  // 16-byte chunks
@@ -409,11 +479,11 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
         ptx::fence_proxy_async_smem();
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bars.p_full[buf]);
+      ptx::mbar_arrive(bars.p_full(buf));
     }
     // ---- this split's unnormalised O, row max and row sum -> workspace
     bool have = alive && U > 0 && !__any_sync(full_mask, *abort_flag != 0);
-    if (have && !__all_sync(full_mask, ptx::mbar_wait(bars.pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1))) {
+    if (have && !__all_sync(full_mask, ptx::mbar_wait(bars.pv_done((U - 1) & 1), ((U - 1) >> 1) & 1))) {
       record_timeout(p.err, abort_flag);
       have = false;
     }

@@ -35,7 +35,7 @@ int check_attn_shape(const orthrus_attn_args* a) {
       a->max_ctx < 0)
     return ORTHRUS_EINVAL;
   if (a->Hq % a->Hkv) return ORTHRUS_EINVAL;
-  if (!isfinite(a->scale)) return ORTHRUS_EINVAL;
+  if (!isfinite(a->scale) || !(a->scale > 0.f)) return ORTHRUS_EINVAL;
   if (a->max_ctx > a->cap) return ORTHRUS_ECAPACITY;
   if (a->D != 64 && a->D != 128) return ORTHRUS_EUNSUPPORTED;
   if (a->blk > 32 || (a->Hq / a->Hkv) * a->blk > 128) return ORTHRUS_EUNSUPPORTED;

@@ -105,7 +105,7 @@ typedef struct orthrus_attn_args {
   int32_t cap;       /* cache rows per (sequence, kv-head) */
   int32_t max_ctx;   /* host bound on every ctx_lens[b]; 0 <= max_ctx <= cap.
                         Sizes the grid; a device length above it is an error. */
-  float scale;       /* softmax scale, usually 1/sqrt(D) */
+  float scale;       /* softmax scale, finite and > 0; usually 1/sqrt(D) */
   int32_t flags;     /* bitwise OR of orthrus_attn_flags (0 = none) */
   const void* q;       /* [B, blk, Hq, D] */
   const void* k_blk;   /* [B, blk, Hkv, D] block K (bidir: diffusion K_diff; causal: AR K) */

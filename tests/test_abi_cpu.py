@@ -95,6 +95,7 @@ def _args(**kw):
     (dict(dtype=7), -1), (dict(mask_mode=2), -1), (dict(Hq=5), -1), (dict(blk=0), -1),
     (dict(D=96), -2), (dict(blk=33), -2), (dict(Hq=16, Hkv=2, blk=32), -2),
     (dict(max_ctx=301), -4), (dict(scale=float("inf")), -1),
+    (dict(scale=0.0), -1), (dict(scale=-0.125), -1),
 ])
 def test_block_attn_rejects_bad_shapes_without_launch(L, kw, code):
     a = _args(**kw)
