@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 # the ncu capture summarised in profiles/attn_tc_partial_b8_ctx8192_full.md
 # (8-sequence case scaled to one sequence).  Valid only for the kernel source
 # it was measured on: reported as null once attn_tc.cu changes.
-TRAFFIC = {"attn_tc_sha256_prefix": "67000c0f6b677a6d", "bytes_per_call": 34766250}
+TRAFFIC = {"attn_tc_sha256_prefix": "7b738b971b3b616f", "bytes_per_call": 34630624}
 
 
 def measured_traffic():
@@ -222,7 +222,103 @@ def kernel_alone(args):
                       "peak": hbm, "peak_source": src}), flush=True)
 
 
+def block_size_sweep(args):
+    """Block attention at the Qwen3-8B layer shape (B=1, ctx 8192) for block
+    sizes K in {4, 8, 16, 32}, both views, 72 calls per CUDA graph chained as in
+    a round: the explainer's ablation (section 六) finds per-round latency
+    roughly constant in K; this checks it at the kernel level."""
+    import torch
+    import block_attention_b200 as ba
+    w = WORKLOAD
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(1002)
+    rnd = lambda *shape: torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)
+    ctx, Hq, Hkv, D, layers = w["ctx"], w["Hq"], w["Hkv"], w["D"], w["layers"]
+    cap = ctx + 32
+    kc, vc = rnd(layers, 1, Hkv, cap, D), rnd(layers, 1, Hkv, cap, D)
+    lens = torch.full((1,), ctx, dtype=torch.int32, device=dev)
+    res = {}
+    for K in (4, 8, 16, 32):
+        q, kb, vb = rnd(2, layers, 1, K, Hq, D), rnd(2, layers, 1, K, Hkv, D), rnd(2, layers, 1, K, Hkv, D)
+        out = torch.empty_like(q)
+        ws = ba.Workspace(dev)
+
+        def seq():
+            for view in (0, 1):
+                for l in range(layers):
+                    ba.block_attn(q[view, l], kb[view, l], vb[view, l], kc[l], vc[l], lens, view,
+                                  out=out[view, l], max_ctx=ctx, workspace=ws, flags=ba.ATTN_EARLY_KV)
+        seq()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            seq()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(max(args.steps, 1)):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res[K] = e0.elapsed_time(e1) * 1e3 / (max(args.steps, 1) * 2 * layers)
+        del graph
+    print(json.dumps({"kernel": "block_attn", "sweep": "block size K",
+                      "case": f"B=1 ctx={ctx} Hq={Hq} Hkv={Hkv} D={D} bf16, both views, "
+                              f"{2 * layers} chained calls per graph",
+                      "us_per_call": res}), flush=True)
+
+
 # ---------------------------------------------------------------- GPU arm
+
+def batched_ragged_leg(dev, hbm, launches=10):
+    """Block attention of the batched ragged Qwen3-8B configuration: 16
+    sequences with contexts ~ U{1k..32k}, Hq 32, Hkv 8, head dim 128, block 32,
+    bf16, both views alternating.  Seeded random bf16 tensors are generated on
+    the device (values do not change the work; parity for this shape is in the
+    tests).  The K/V caches hold about 2.2 GB, far beyond the L2.  Runs after the
+    timed round; it reports its own time and roofline fraction."""
+    import torch
+    import block_attention_b200 as ba
+    from block_attention_b200 import synth
+    B, Hq, Hkv, D, blk = 16, 32, 8, 128, 32
+    lens = synth.ragged_lens(B, 1024, 32768, seed=1004)
+    cap = int(lens.max()) + blk
+    g = torch.Generator(device=dev).manual_seed(1004)
+    rnd = lambda *shape: torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)
+    q, kb, vb = rnd(B, blk, Hq, D), rnd(B, blk, Hkv, D), rnd(B, blk, Hkv, D)
+    kc, vc = rnd(B, Hkv, cap, D), rnd(B, Hkv, cap, D)
+    ctx = torch.from_numpy(lens.astype(np.int32)).to(dev)
+    out = torch.empty_like(q)
+    ws = ba.Workspace(dev)
+
+    def call(k):
+        ba.block_attn(q, kb, vb, kc, vc, ctx, k % 2, out=out, max_ctx=cap - blk, workspace=ws,
+                      flags=ba.ATTN_EARLY_KV)
+    for k in range(4):
+        call(k)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for k in range(launches):
+            call(k)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / launches
+    nbytes = 2 * int(lens.sum()) * Hkv * D * 2 + 2 * B * blk * Hq * D * 2 + 2 * B * blk * Hkv * D * 2
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del graph
+    return {"workload": "batched ragged Qwen3-8B layer: 16 sequences, ctx ~ U{1024..32768} "
+                        f"(sum {int(lens.sum())}), Hq 32, Hkv 8, D 128, block 32, bf16, both views",
+            "us_per_launch": us, "bytes_per_launch": nbytes, "gbs": gbs, "peak": hbm,
+            "frac": gbs / hbm, "launches": launches, "l2": "inputs larger than L2"}
+
 
 def decoder_report():
     """The end-to-end consensus loop on the random-init decoder (4 layers,
@@ -268,12 +364,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e-decoder", action="store_true",
                     help="skip the end-to-end decoder report (runs after the timing)")
-    ap.add_argument("--kernel", choices=["attn"], default=None,
-                    help="time one kernel alone on a case larger than L2 (for profiling)")
+    ap.add_argument("--no-batched", action="store_true",
+                    help="skip the batched ragged attention leg (runs after the timing)")
+    ap.add_argument("--kernel", choices=["attn", "blk"], default=None,
+                    help="attn: time block attention alone on a case larger than L2 (for "
+                         "profiling); blk: block-size sweep K in {4, 8, 16, 32}")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.kernel:
+    if args.kernel == "attn":
         return kernel_alone(args)
+    if args.kernel == "blk":
+        return block_size_sweep(args)
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -374,6 +475,9 @@ def main():
     dec = None
     if rank == 0 and world == 1 and not args.no_e2e_decoder:
         dec = decoder_report()
+    batched = None
+    if rank == 0 and world == 1 and not args.no_batched:
+        batched = batched_ragged_leg(dev, hbm)
 
     if world > 1:
         dist.barrier()
@@ -402,6 +506,7 @@ def main():
         "clocks": clk,
         "cpu_baseline": cpu,
         "e2e_decoder": dec,
+        "block_attn_batched_ragged": batched,
     }
     print(json.dumps(line), flush=True)
 

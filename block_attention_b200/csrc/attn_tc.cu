@@ -48,8 +48,8 @@
 // bf16 (one extra rounding, relative 2^-9), halving the epilogue's stores.
 //
 // With ORTHRUS_ATTN_EARLY_KV the partial kernel reads ctx_lens and starts
-// streaming K/V tiles before waiting on the preceding kernel; Q and the block
-// K/V are read only after that wait.
+// streaming its first K/V tiles before waiting on the preceding kernel; Q and
+// the block K/V are read only after that wait.
 //
 // Every mbarrier wait is bounded: on a timeout the kernel records
 // ORTHRUS_ETIMEOUT in the error word, stops issuing work and drains what it
@@ -70,6 +70,11 @@ namespace {
 constexpr int kRows = 128;          // UMMA M
 constexpr int kTile = 128;          // keys per tile (UMMA N of S = Q K^T)
 constexpr int kStages = 3;          // K/V ring depth
+// Cache tiles requested before the dependency wait under EARLY_KV.  They
+// stream while the preceding kernel drains; requesting the whole ring makes
+// the burst collide with that kernel's own memory traffic (measured on B200:
+// 2 tiles ahead beat both 1 and 3 by 3% per call at the Qwen3-8B shape).
+constexpr int kEarlyTiles = 2;
 constexpr int kThreads = 192;       // 6 warps
 constexpr int kTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256,256+D) Q, P after it
 constexpr int kOCol = 256;
@@ -223,7 +228,7 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     }
   };
 
-  // Early cache streaming: the first ring's worth of cache tiles (never the
+  // Early cache streaming: the first kEarlyTiles cache tiles (never the
   // block tile, which the preceding kernel may still be writing).
   int early_issued = 0;
   int early_n = 0;
@@ -238,7 +243,7 @@ attn_tc_partial(const __grid_constant__ TcParams p) {
     early_n = p.ctx_lens[b];
     int Tc, t0, U;
     geometry(early_n, Tc, t0, U);
-    while (early_issued < min(U, kStages) && t0 + early_issued < Tc) {
+    while (early_issued < min(U, kEarlyTiles) && t0 + early_issued < Tc) {
       issue(false, early_issued, t0 + early_issued, Tc);
       issue(true, early_issued, t0 + early_issued, Tc);
       ++early_issued;
@@ -610,13 +615,17 @@ bool prepare(int device) {
   return true;
 }
 
-// Splits per (sequence, kv-head): one wave of CTAs (one per SM) when the
-// batch is small, else 4 per head so ragged lengths still balance; never more
-// splits than the longest sequence has tiles.
+// Splits per (sequence, kv-head): enough to fill one wave of CTAs (one per
+// SM) when the batch is small, and at least enough that no split of the
+// longest possible sequence exceeds 64 tiles, so long or ragged batches spread
+// over several waves instead of leaving their longest sequences to a few CTAs;
+// never more splits than the longest sequence has tiles.
 int choose_splits(const orthrus_attn_args& a) {
   const int heads = a.B * a.Hkv;
-  int S = heads >= 148 ? 4 : 148 / heads;
-  S = min(S, ceil_div(a.max_ctx, kTile) + 1);
+  const int tiles = ceil_div(a.max_ctx, kTile) + 1;
+  int S = heads >= 148 ? 1 : 148 / heads;
+  S = max(S, ceil_div(tiles, 64));
+  S = min(S, tiles);
   return max(1, min(S, kMaxSplits));
 }
 

@@ -171,3 +171,13 @@ def test_early_kv_flag_same_result(oracle_mod, mode):
                       t["ctx_lens"], mode, flags=ba.ATTN_EARLY_KV)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("blk", [4, 8, 16])
+def test_block_size_variants(oracle_mod, dtype, mode, blk):
+    """Block sizes K in {4, 8, 16} (the explainer's ablation, section 六) at the
+    Qwen3-8B head layout, with a ragged pair of contexts."""
+    inp = synth.attn_inputs(2, 32, 8, 128, blk, [2000, 333], 2000 + blk, dtype, seed=150 + blk)
+    check(inp, mode, dtype, oracle_mod=oracle_mod)
