@@ -328,7 +328,7 @@ def decoder_report():
     per forward.  Runs after the timed regions; it times nothing of the bench."""
     import torch
     from block_attention_b200 import synth
-    from block_attention_b200.decoder import TinyDecoder, trajectory_report
+    from block_attention_b200.decoder import TinyDecoder, perplexity_report, trajectory_report
     E = synth.WORKLOADS["e2e_decoder"]
     seed = 1004
     W = synth.decoder_weights(E["V"], E["d"], E["L"], E["Hq"], E["Hkv"], E["hd"], E["ffn"],
@@ -341,7 +341,8 @@ def decoder_report():
     out = {}
     for name, dt in (("fp32", torch.float32), ("bf16", torch.bfloat16)):
         m = TinyDecoder(W, E["Hq"], E["Hkv"], E["hd"], dtype=dt)
-        out[name + "_greedy"] = m.greedy(prompts, E["n_new"])
+        out[name + "_greedy"], out[name + "_logprob"] = m.greedy(prompts, E["n_new"],
+                                                                 logprob=True)
         toks, st = m.consensus(prompts, E["n_new"], blk=E["blk"])
         out[name + "_loop"] = toks
         rep.setdefault("tokens_per_forward", {})[name] = st["tokens_per_forward"]
@@ -351,6 +352,8 @@ def decoder_report():
     rep["bf16_loop_vs_bf16_greedy"] = trajectory_report(out["bf16_loop"], out["bf16_greedy"])
     rep["bf16_greedy_vs_fp32_greedy"] = trajectory_report(out["bf16_greedy"],
                                                           out["fp32_greedy"])
+    rep["bf16_loop_vs_fp32_greedy_by_reference_perplexity"] = perplexity_report(
+        out["bf16_loop"], out["fp32_greedy"], out["fp32_logprob"])
     rep["seconds"] = time.perf_counter() - t0
     return rep
 

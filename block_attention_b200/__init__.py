@@ -69,7 +69,7 @@ EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
-           "orthrus_swiglu", "orthrus_block_tokens")
+           "orthrus_swiglu", "orthrus_block_tokens", "orthrus_token_logprob")
 
 _lib = None
 
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
                                        vp, vp, vp, vp]
         L.orthrus_swiglu.argtypes = [i32, vp, i32, i32, vp, vp]
         L.orthrus_block_tokens.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+        L.orthrus_token_logprob.argtypes = [i32, vp, i32, i32, i64, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -332,4 +333,18 @@ def block_tokens(anchor, draft, blk, mask_id, *, out=None, stream=None):
         out = torch.empty(B, blk, dtype=torch.int32, device=anchor.device)
     _check("orthrus_block_tokens", lib().orthrus_block_tokens(
         _ptr(anchor), _ptr(draft), B, blk, int(mask_id), _ptr(out), _stream(stream)))
+    return out
+
+
+def token_logprob(logits, idx, *, out=None, stream=None):
+    """float [rows]: log-softmax of logits [rows, vocab] at idx (int32 [rows])."""
+    _dev(idx, out)
+    if not logits.is_cuda or logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits must be a 2-D CUDA tensor with unit column stride")
+    rows, vocab = logits.shape
+    if out is None:
+        out = torch.empty(rows, dtype=torch.float32, device=logits.device)
+    _check("orthrus_token_logprob", lib().orthrus_token_logprob(
+        _dtype(logits), _ptr(logits), rows, vocab, logits.stride(0), _ptr(idx), _ptr(out),
+        _stream(stream)))
     return out

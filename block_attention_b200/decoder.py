@@ -119,10 +119,11 @@ class TinyDecoder:
     def prefill(self, prompts, cap: int, chunk: int = 32):
         """Causal AR pass over every prompt in blocks of ``chunk`` rows.
 
-        Returns the state (cache holding each prompt) and the first generated
-        token per sequence (host int32 [B]).  Rows past a prompt's end are
-        computed but never committed; causal masking keeps them from
-        influencing the prompt's own rows."""
+        Returns the state (cache holding each prompt), the first generated
+        token per sequence (host int32 [B]) and its log-probability (host
+        float32 [B]).  Rows past a prompt's end are computed but never
+        committed; causal masking keeps them from influencing the prompt's own
+        rows."""
         B = len(prompts)
         lens = np.array([len(p) for p in prompts], np.int64)
         if lens.min() < 1 or lens.max() + chunk > cap:
@@ -133,35 +134,45 @@ class TinyDecoder:
             toks[b, :len(p)] = p
         st = DecodeState(self, B, cap)
         first = np.zeros(B, np.int32)
+        first_lp = np.zeros(B, np.float32)
         last_chunk, last_row = (lens - 1) // chunk, (lens - 1) % chunk
         for c in range(nchunks):
             t = torch.from_numpy(np.ascontiguousarray(toks[:, c * chunk:(c + 1) * chunk]))
             logits, kb, vb = self.forward(st, t.to(self.device), AR_VIEW)
             here = np.nonzero(last_chunk == c)[0]  # prompts that end in this chunk
             if here.size:
-                idx_h = ba.vocab_argmax(logits).view(B, chunk).cpu().numpy()
+                idx = ba.vocab_argmax(logits)
+                idx_h = idx.view(B, chunk).cpu().numpy()
+                lp_h = ba.token_logprob(logits, idx).view(B, chunk).cpu().numpy()
                 first[here] = idx_h[here, last_row[here]]
+                first_lp[here] = lp_h[here, last_row[here]]
             valid = np.clip(lens - c * chunk, 0, chunk).astype(np.int32)
             self.commit(st, kb, vb, torch.from_numpy(valid).to(self.device))
         self.check(st)
-        return st, first
+        return st, first, first_lp
 
     # ---------------------------------------------------------- greedy AR
-    def greedy(self, prompts, n_new: int, cap: int | None = None) -> np.ndarray:
+    def greedy(self, prompts, n_new: int, cap: int | None = None, logprob: bool = False):
         """Plain greedy autoregressive decoding, one token per forward:
-        int32 [B, n_new] (the first token comes from the prefill)."""
+        int32 [B, n_new] (the first token comes from the prefill); with
+        ``logprob`` also each chosen token's log-probability, float32 [B, n_new]."""
         cap = cap or max(len(p) for p in prompts) + n_new + 64
-        st, first = self.prefill(prompts, cap)
+        st, first, first_lp = self.prefill(prompts, cap)
         B = st.B
         out = torch.empty(n_new, B, dtype=torch.int32, device=self.device)
         out[0].copy_(torch.from_numpy(first))
+        lp = torch.empty(n_new, B, dtype=torch.float32, device=self.device)
+        lp[0].copy_(torch.from_numpy(first_lp))
         ones = torch.ones(B, dtype=torch.int32, device=self.device)
         for t in range(1, n_new):
             logits, kb, vb = self.forward(st, out[t - 1].view(B, 1), AR_VIEW)
             ba.vocab_argmax(logits, idx=out[t])
+            if logprob:
+                ba.token_logprob(logits, out[t], out=lp[t])
             self.commit(st, kb, vb, ones)
         self.check(st)
-        return out.t().contiguous().cpu().numpy()
+        toks = out.t().contiguous().cpu().numpy()
+        return (toks, lp.t().contiguous().cpu().numpy()) if logprob else toks
 
     # ----------------------------------------------------- consensus loop
     def consensus(self, prompts, n_new: int, blk: int = 32, draft_fn=None,
@@ -173,7 +184,7 @@ class TinyDecoder:
         that any draft gives the greedy trajectory.  Sequences that reach
         n_new tokens stop committing; the loop ends when all have."""
         cap = cap or max(len(p) for p in prompts) + n_new + 2 * blk
-        st, first = self.prefill(prompts, cap)
+        st, first, _ = self.prefill(prompts, cap)
         B = st.B
         out = [[int(f)] for f in first]
         counts = np.ones(B, np.int64)
@@ -236,3 +247,27 @@ def trajectory_report(test: np.ndarray, ref: np.ndarray) -> dict:
             "exact_match_rate": float(exact.mean()),
             "token_match_rate": float(eq.mean()),
             "mean_first_divergence": float(first_div.mean())}
+
+
+def perplexity_report(test: np.ndarray, ref: np.ndarray, ref_logprob: np.ndarray,
+                      groups: int = 4) -> dict:
+    """Exact-trajectory match of ``test`` against ``ref`` within groups of
+    sequences ordered by the reference's response-conditional perplexity
+    exp(-mean log p(token)) (the reproduction study finds exact matching
+    strongly associated with it), plus the rank correlation between that
+    perplexity and where the trajectories first diverge."""
+    ppl = np.exp(-ref_logprob.astype(np.float64).mean(axis=1))
+    eq = test == ref
+    exact = eq.all(axis=1)
+    first_div = np.where(exact, ref.shape[1], np.argmin(eq, axis=1))
+    order = np.argsort(ppl, kind="stable")
+    rows = []
+    for gi, part in enumerate(np.array_split(order, groups)):
+        rows.append({"group": gi, "sequences": int(part.size),
+                     "perplexity_min": float(ppl[part].min()),
+                     "perplexity_max": float(ppl[part].max()),
+                     "exact_match_rate": float(exact[part].mean()),
+                     "mean_first_divergence": float(first_div[part].mean())})
+    rank = lambda a: np.argsort(np.argsort(a, kind="stable"), kind="stable").astype(np.float64)
+    rho = float(np.corrcoef(rank(ppl), rank(first_div))[0, 1]) if ref.shape[0] > 1 else 0.0
+    return {"groups": rows, "spearman_perplexity_vs_first_divergence": rho}

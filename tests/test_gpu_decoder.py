@@ -172,3 +172,12 @@ def test_bf16_trajectory_match_rate(model16, prompts, greedy32):
         assert rep["token_match_rate"] > 0.0
     assert ((toks >= 0) & (toks < E["V"])).all()
     assert st["tokens_per_forward"] >= 0.5
+
+
+def test_greedy_logprobs_bounded(model32, prompts):
+    """The greedy token is the row's argmax, so its probability is at least 1/V:
+    every reported log-probability lies in [-log V, 0]."""
+    toks, lp = model32.greedy(prompts[:8], 24, logprob=True)
+    assert toks.shape == lp.shape == (8, 24)
+    assert np.isfinite(lp).all()
+    assert (lp <= 1e-6).all() and (lp >= -np.log(E["V"]) - 1e-4).all()

@@ -162,3 +162,34 @@ def test_commit_full_block_bytes_match_explainer_figure(oracle_mod):
     per_layer_bytes = int(changed_rows) * shp["D"] * 2
     assert per_layer_bytes * shp["layers"] == fig["block_state_bytes"]["value"]
     assert fig["block_state_bytes"]["value"] == 4.5 * 2 ** 20
+
+
+# ---------------------------------------------------------- token log-prob
+
+def test_token_logprob_matches_scipy_logsumexp(oracle_mod):
+    from scipy.special import logsumexp
+    g = np.random.default_rng(7)
+    x = g.normal(0, 3, (6, 1000))
+    idx = g.integers(0, 1000, 6)
+    got = oracle_mod.token_logprob(x, idx)
+    ref = x[np.arange(6), idx] - logsumexp(x, axis=1)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_token_logprob_closed_forms(oracle_mod):
+    V = 512
+    # uniform row: every token has probability 1/V
+    np.testing.assert_allclose(oracle_mod.token_logprob(np.zeros((1, V)), [17]), [-np.log(V)],
+                               atol=1e-12)
+    # shifting a row leaves log-probabilities unchanged; a dominant logit -> ~0
+    x = np.random.default_rng(8).normal(0, 1, (2, V))
+    x[1] = x[0] + 123.0
+    lp = oracle_mod.token_logprob(x, [5, 5])
+    assert abs(lp[0] - lp[1]) < 1e-9
+    y = np.zeros((1, V)); y[0, 9] = 60.0
+    assert abs(oracle_mod.token_logprob(y, [9])[0]) < 1e-20 + (V - 1) * np.exp(-60)
+    # probabilities of a row sum to one
+    tot = np.exp(oracle_mod.token_logprob(np.repeat(x[:1], V, 0), np.arange(V))).sum()
+    assert abs(tot - 1.0) < 1e-12
+    # an index outside the row gives NaN
+    assert np.isnan(oracle_mod.token_logprob(x[:1], [V])[0])
