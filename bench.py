@@ -34,6 +34,7 @@ METRIC = "block-attn HBM GB/s (% of peak) and consensus rounds/s, Qwen3-8B shape
 WORKLOAD = dict(name="qwen3_8b_round", layers=36, B=1, Hq=32, Hkv=8, D=128, ctx=8192,
                 blk=32, vocab=151936, dtype="bf16", logits_dtype="f32", accept_mean=5.4)
 FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20  # written between cold timings: twice the 126 MB L2
 # DRAM bytes (read + write) of one block-attention call at this workload, from
 # the ncu capture summarised in profiles/attn_tc_partial_b8_ctx8192_full.md
 # (8-sequence case scaled to one sequence).  Valid only for the kernel source
@@ -222,6 +223,57 @@ def kernel_alone(args):
                       "peak": hbm, "peak_source": src}), flush=True)
 
 
+def sampling_kernels(args):
+    """The stochastic round's kernels one at a time at the Qwen3-8B shape (32
+    rows x vocab 151936, fp32 logits, T = 1): draft sampling with and without
+    the fused log-sum-exp, the stand-alone log-probability pass, and the
+    consensus (log p + acceptance, then the correction).  Each is captured
+    `steps` times in its own CUDA graph; the logits stay L2-resident."""
+    import torch
+    import block_attention_b200 as ba
+    dev = torch.device("cuda", 0)
+    w = WORKLOAD
+    rows, V, B, blk = w["B"] * w["blk"], w["vocab"], w["B"], w["blk"]
+    g = torch.Generator(device=dev).manual_seed(1005)
+    zq = torch.randn(rows, V, generator=g, device=dev) * 3
+    zp = zq + torch.randn(rows, V, generator=g, device=dev) * 0.5
+    f32 = dict(dtype=torch.float32, device=dev)
+    lq, lp, sq, sp = (torch.empty(rows, **f32) for _ in range(4))
+    d = torch.empty(rows, dtype=torch.int32, device=dev)
+    outs = [torch.empty(B, dtype=torch.int32, device=dev) for _ in range(3)]
+    em = torch.empty(B, blk, dtype=torch.int32, device=dev)
+    ops = {
+        "vocab_sample": lambda k: ba.vocab_sample(zq, 1.0, 7, k, idx=d),
+        "vocab_sample_with_lse": lambda k: ba.vocab_sample(zq, 1.0, 7, k, idx=d, logprob=lq,
+                                                           lse=sq),
+        "token_logprob": lambda k: ba.token_logprob(zq, d, temperature=1.0, out=lq, lse=sq),
+        "consensus_sample": lambda k: ba.consensus_sample(
+            d.view(B, blk), zp, zq, lq, sq, 1.0, 7, k, logp=lp, lse_ar=sp, accept_len=outs[0],
+            n_emit=outs[1], emitted=em, next_anchor=outs[2]),
+    }
+    res = {}
+    for name, f in ops.items():
+        for k in range(args.warmup):
+            f(k)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for k in range(args.steps):
+                f(k)
+        gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = e0.elapsed_time(e1) * 1e3 / args.steps
+        del gr
+    print(json.dumps({"kernel": "stochastic round kernels",
+                      "case": f"{rows} rows x vocab {V}, fp32 logits, T = 1, L2-resident",
+                      "us_per_launch": res}), flush=True)
+
+
 def block_size_sweep(args):
     """Block attention at the Qwen3-8B layer shape (B=1, ctx 8192) for block
     sizes K in {4, 8, 16, 32}, both views, 72 calls per CUDA graph chained as in
@@ -320,6 +372,73 @@ def batched_ragged_leg(dev, hbm, launches=10):
             "frac": gbs / hbm, "launches": launches, "l2": "inputs larger than L2"}
 
 
+def stochastic_round_leg(dev, hbm, iters=20):
+    """The stochastic consensus step of one round at the Qwen3-8B shape (B = 1,
+    block 32, vocab 151936, fp32 logits of both views): draft sampling with the
+    drafts' log q and log-sum-exp from the same pass, then the consensus (log p
+    over the AR logits with the acceptance test, and the correction), three
+    launches in one CUDA graph.  Algorithmic bytes: one read of each logit
+    matrix plus the two rows of the correction.  Timed twice: 20 rounds back
+    to back (the logits stay L2-resident, as right after the LM head writes
+    them), and single rounds after an L2 flush (HBM reads; the fraction of
+    peak refers to these)."""
+    import torch
+    import block_attention_b200 as ba
+    w = WORKLOAD
+    rows, V, B, blk = w["B"] * w["blk"], w["vocab"], w["B"], w["blk"]
+    g = torch.Generator(device=dev).manual_seed(1005)
+    zq = torch.randn(rows, V, generator=g, device=dev) * 3
+    zp = zq + torch.randn(rows, V, generator=g, device=dev) * 0.5
+    f32 = dict(dtype=torch.float32, device=dev)
+    lq, lp, sq, sp = (torch.empty(rows, **f32) for _ in range(4))
+    d = torch.empty(rows, dtype=torch.int32, device=dev)
+    outs = [torch.empty(B, dtype=torch.int32, device=dev) for _ in range(3)]
+    em = torch.empty(B, blk, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(k):
+        ba.vocab_sample(zq, 1.0, 7, k, idx=d, logprob=lq, lse=sq)
+        ba.consensus_sample(d.view(B, blk), zp, zq, lq, sq, 1.0, 7, k, logp=lp, lse_ar=sp,
+                            accept_len=outs[0], n_emit=outs[1], emitted=em,
+                            next_anchor=outs[2])
+    for k in range(3):
+        step(k)
+    torch.cuda.synchronize()
+    graph, one = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for k in range(iters):
+            step(k)
+    with torch.cuda.graph(one):
+        step(0)
+    graph.replay()
+    one.replay()
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    e0, e1 = ev(), ev()
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    hot = e0.elapsed_time(e1) * 1e3 / iters
+    cold = []
+    for k in range(10):
+        flush.fill_(k & 0xFF)
+        e0, e1 = ev(), ev()
+        e0.record()
+        one.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        cold.append(e0.elapsed_time(e1) * 1e3)
+    cold = sorted(cold)[len(cold) // 2]
+    nbytes = 2 * rows * V * 4 + 2 * V * 4
+    del graph, one
+    return {"workload": f"stochastic consensus, B=1 block 32, vocab {V}, fp32 logits, T = 1",
+            "kernels_per_round": 3, "bytes_per_round": nbytes,
+            "us_per_round_l2_resident": hot, "us_per_round_cold": cold,
+            "gbs_cold": nbytes / (cold * 1e-6) / 1e9, "peak": hbm,
+            "frac_cold": nbytes / (cold * 1e-6) / 1e9 / hbm}
+
+
 def decoder_report():
     """The end-to-end consensus loop on the random-init decoder (4 layers,
     d_model 512, Hq 8, Hkv 4, head dim 64, SwiGLU 1536, vocab 8192; 256
@@ -368,16 +487,20 @@ def main():
     ap.add_argument("--no-e2e-decoder", action="store_true",
                     help="skip the end-to-end decoder report (runs after the timing)")
     ap.add_argument("--no-batched", action="store_true",
-                    help="skip the batched ragged attention leg (runs after the timing)")
-    ap.add_argument("--kernel", choices=["attn", "blk"], default=None,
+                    help="skip the batched ragged attention and stochastic consensus legs "
+                         "(they run after the timing)")
+    ap.add_argument("--kernel", choices=["attn", "blk", "sample"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
-                         "profiling); blk: block-size sweep K in {4, 8, 16, 32}")
+                         "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
+                         "the stochastic round's kernels one at a time")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel == "attn":
         return kernel_alone(args)
     if args.kernel == "blk":
         return block_size_sweep(args)
+    if args.kernel == "sample":
+        return sampling_kernels(args)
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -478,9 +601,10 @@ def main():
     dec = None
     if rank == 0 and world == 1 and not args.no_e2e_decoder:
         dec = decoder_report()
-    batched = None
+    batched = stochastic = None
     if rank == 0 and world == 1 and not args.no_batched:
         batched = batched_ragged_leg(dev, hbm)
+        stochastic = stochastic_round_leg(dev, hbm)
 
     if world > 1:
         dist.barrier()
@@ -510,6 +634,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e_decoder": dec,
         "block_attn_batched_ragged": batched,
+        "stochastic_consensus": stochastic,
     }
     print(json.dumps(line), flush=True)
 

@@ -63,13 +63,29 @@ class CommitArgs(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class SampleArgs(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("B", ctypes.c_int32), ("blk", ctypes.c_int32),
+                ("vocab", ctypes.c_int32), ("row_stride", ctypes.c_int64),
+                ("temperature", ctypes.c_float), ("step", ctypes.c_uint32),
+                ("seed", ctypes.c_uint64),
+                ("draft", ctypes.c_void_p), ("logq", ctypes.c_void_p),
+                ("lse_diff", ctypes.c_void_p),
+                ("logits_ar", ctypes.c_void_p), ("logits_diff", ctypes.c_void_p),
+                ("logp", ctypes.c_void_p), ("lse_ar", ctypes.c_void_p),
+                ("accept_len", ctypes.c_void_p), ("n_emit", ctypes.c_void_p),
+                ("emitted", ctypes.c_void_p), ("next_anchor", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
 EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_block_attn_launches", "orthrus_vocab_argmax",
            "orthrus_vocab_argmax_workspace", "orthrus_consensus", "orthrus_kv_commit",
            "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version",
+           "orthrus_vocab_sample", "orthrus_vocab_sample_workspace", "orthrus_token_logprob", "orthrus_token_logprob_workspace",
+           "orthrus_consensus_sample", "orthrus_consensus_sample_workspace",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
-           "orthrus_swiglu", "orthrus_block_tokens", "orthrus_token_logprob")
+           "orthrus_swiglu", "orthrus_block_tokens")
 
 _lib = None
 
@@ -106,7 +122,17 @@ def lib() -> ctypes.CDLL:
                                        vp, vp, vp, vp]
         L.orthrus_swiglu.argtypes = [i32, vp, i32, i32, vp, vp]
         L.orthrus_block_tokens.argtypes = [vp, vp, i32, i32, i32, vp, vp]
-        L.orthrus_token_logprob.argtypes = [i32, vp, i32, i32, i64, vp, vp, vp]
+        L.orthrus_token_logprob.argtypes = [i32, vp, i32, i32, i64, vp, c.c_float, vp, vp, vp,
+                                            sz, vp]
+        L.orthrus_token_logprob_workspace.argtypes = [i32, i32]
+        L.orthrus_token_logprob_workspace.restype = sz
+        L.orthrus_consensus_sample_workspace.argtypes = [i32, i32, i32]
+        L.orthrus_consensus_sample_workspace.restype = sz
+        L.orthrus_vocab_sample_workspace.argtypes = [i32, i32]
+        L.orthrus_vocab_sample_workspace.restype = sz
+        L.orthrus_vocab_sample.argtypes = [i32, vp, i32, i32, i64, c.c_float, c.c_uint64,
+                                           c.c_uint32, vp, vp, vp, vp, sz, vp]
+        L.orthrus_consensus_sample.argtypes = [c.POINTER(SampleArgs), vp]
         _lib = L
     return _lib
 
@@ -336,15 +362,74 @@ def block_tokens(anchor, draft, blk, mask_id, *, out=None, stream=None):
     return out
 
 
-def token_logprob(logits, idx, *, out=None, stream=None):
-    """float [rows]: log-softmax of logits [rows, vocab] at idx (int32 [rows])."""
-    _dev(idx, out)
+def token_logprob(logits, idx, *, temperature=1.0, out=None, lse=None, workspace=None,
+                  stream=None):
+    """float [rows]: log-softmax of logits [rows, vocab] / temperature at idx
+    (int32 [rows]); fills lse [rows] with each row's log-sum-exp if given."""
+    _dev(idx, out, lse)
     if not logits.is_cuda or logits.dim() != 2 or logits.stride(1) != 1:
         raise ValueError("logits must be a 2-D CUDA tensor with unit column stride")
     rows, vocab = logits.shape
     if out is None:
         out = torch.empty(rows, dtype=torch.float32, device=logits.device)
+    need = lib().orthrus_token_logprob_workspace(rows, vocab)
+    buf = _ws(workspace, logits.device, "logprob").get(need)
     _check("orthrus_token_logprob", lib().orthrus_token_logprob(
-        _dtype(logits), _ptr(logits), rows, vocab, logits.stride(0), _ptr(idx), _ptr(out),
-        _stream(stream)))
+        _dtype(logits), _ptr(logits), rows, vocab, logits.stride(0), _ptr(idx),
+        float(temperature), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream(stream)))
     return out
+
+
+def vocab_sample(logits, temperature, seed, step, *, idx=None, logprob=None, lse=None,
+                 workspace=None, stream=None):
+    """int32 [rows]: one sample per row of softmax(logits / temperature)
+    (Gumbel-max, Philox stream of orthrus.h; purpose 1, x1 = row).  Given
+    float32 [rows] tensors ``logprob`` / ``lse``, the same pass also writes the
+    sample's log-probability and the row's log-sum-exp at that temperature."""
+    _dev(idx, logprob, lse)
+    if not logits.is_cuda or logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits must be a 2-D CUDA tensor with unit column stride")
+    rows, vocab = logits.shape
+    if idx is None:
+        idx = torch.empty(rows, dtype=torch.int32, device=logits.device)
+    need = lib().orthrus_vocab_sample_workspace(rows, vocab)
+    buf = _ws(workspace, logits.device, "sample").get(need)
+    _check("orthrus_vocab_sample", lib().orthrus_vocab_sample(
+        _dtype(logits), _ptr(logits), rows, vocab, logits.stride(0), float(temperature),
+        int(seed) & (2 ** 64 - 1), int(step) & 0xFFFFFFFF, _ptr(idx), _ptr(logprob), _ptr(lse),
+        _ptr(buf), buf.numel(), _stream(stream)))
+    return idx
+
+
+def consensus_sample(draft, logits_ar, logits_diff, logq, lse_diff, temperature, seed, step, *,
+                     logp=None, lse_ar=None, accept_len=None, n_emit=None, emitted=None,
+                     next_anchor=None, workspace=None, stream=None):
+    """Stochastic consensus (see orthrus.h).  draft int32 [B, blk]; logits_*
+    [B*blk, vocab]; logq / lse_diff float32 [B*blk], the logprob / lse outputs
+    of vocab_sample on logits_diff at the same temperature.  Writes log p and
+    the AR rows' log-sum-exp into ``logp`` / ``lse_ar`` (allocated if None).
+    Returns (accept_len, n_emit, emitted, next_anchor)."""
+    _dev(draft, logq, lse_diff, logp, lse_ar)
+    B, blk = draft.shape
+    rows, vocab = logits_ar.shape
+    if logits_diff.shape != logits_ar.shape or logits_ar.stride(1) != 1 or \
+            logits_diff.stride(0) != logits_ar.stride(0):
+        raise ValueError("logit matrices must share shape and row stride")
+    dev = draft.device
+    mk = lambda t, shp, dt=torch.int32: t if t is not None else torch.empty(shp, dtype=dt,
+                                                                            device=dev)
+    accept_len, n_emit, next_anchor = mk(accept_len, B), mk(n_emit, B), mk(next_anchor, B)
+    emitted = mk(emitted, (B, blk))
+    logp, lse_ar = mk(logp, rows, torch.float32), mk(lse_ar, rows, torch.float32)
+    a = SampleArgs(_dtype(logits_ar), B, blk, vocab, logits_ar.stride(0), float(temperature),
+                   int(step) & 0xFFFFFFFF, int(seed) & (2 ** 64 - 1), draft.data_ptr(),
+                   logq.data_ptr(), lse_diff.data_ptr(), logits_ar.data_ptr(),
+                   logits_diff.data_ptr(), logp.data_ptr(), lse_ar.data_ptr(),
+                   accept_len.data_ptr(), n_emit.data_ptr(), emitted.data_ptr(),
+                   next_anchor.data_ptr())
+    need = lib().orthrus_consensus_sample_workspace(B, blk, vocab)
+    buf = _ws(workspace, dev, "consensus_sample").get(need)
+    a.workspace, a.workspace_bytes = buf.data_ptr(), buf.numel()
+    _check("orthrus_consensus_sample", lib().orthrus_consensus_sample(ctypes.byref(a),
+                                                                      _stream(stream)))
+    return accept_len, n_emit, emitted, next_anchor

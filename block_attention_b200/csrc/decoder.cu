@@ -227,55 +227,6 @@ block_tokens_kernel(const int32_t* __restrict__ anchor, const int32_t* __restric
       j == 0 ? anchor[b] : (draft ? draft[(int64_t)b * blk + j - 1] : mask_id);
 }
 
-// ------------------------------------------------------- token log-prob
-// One CTA per row: max, then sum of exp(x - max), each as per-thread strided
-// partials (thread t takes j = t, t + 256, ...) merged in a fixed tree.
-constexpr int kLpThreads = 256;
-
-template <typename T>
-__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, off);
-    v = is_max ? fmaxf(v, o) : v + o;
-  }
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) red[w] = v;
-  __syncthreads();
-  if (w == 0) {
-    v = lane < kLpThreads / 32 ? red[lane] : (is_max ? -INFINITY : 0.f);
-#pragma unroll
-    for (int off = 4; off > 0; off >>= 1) {
-      const float o = __shfl_xor_sync(0xffffffffu, v, off);
-      v = is_max ? fmaxf(v, o) : v + o;
-    }
-    if (lane == 0) red[kLpThreads / 32] = v;
-  }
-  __syncthreads();
-  const float r = red[kLpThreads / 32];
-  __syncthreads();
-  return r;
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kLpThreads)
-token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
-                     const int32_t* __restrict__ idx, float* __restrict__ out) {
-  __shared__ float red[kLpThreads / 32 + 1];
-  const int r = blockIdx.x;
-  const T* row = logits + (int64_t)r * stride;
-  float m = -INFINITY;
-  for (int j = threadIdx.x; j < vocab; j += kLpThreads) m = fmaxf(m, to_f32(row[j]));
-  m = block_reduce<T>(m, true, red);
-  float s = 0.f;
-  for (int j = threadIdx.x; j < vocab; j += kLpThreads) s += expf(to_f32(row[j]) - m);
-  s = block_reduce<T>(s, false, red);
-  if (threadIdx.x == 0) {
-    const int k = idx[r];
-    out[r] = (k >= 0 && k < vocab) ? (to_f32(row[k]) - m) - logf(s) : __int_as_float(0x7fc00000);
-  }
-}
-
 }  // namespace
 }  // namespace orthrus
 
@@ -397,22 +348,6 @@ int orthrus_block_tokens(const int32_t* anchor, const int32_t* draft, int32_t B,
   if (!anchor || !out) return ORTHRUS_EINVAL;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   block_tokens_kernel<<<B, 32, 0, st>>>(anchor, draft, blk, mask_id, out);
-  return status(cudaGetLastError());
-}
-
-int orthrus_token_logprob(int32_t dtype, const void* logits, int32_t rows, int32_t vocab,
-                          int64_t row_stride, const int32_t* idx, float* out,
-                          orthrus_stream_t stream) {
-  if (!dtype_ok(dtype) || rows < 0 || vocab <= 0 || row_stride < vocab) return ORTHRUS_EINVAL;
-  if (rows == 0) return ORTHRUS_OK;
-  if (!logits || !idx || !out) return ORTHRUS_EINVAL;
-  auto st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == ORTHRUS_F32)
-    token_logprob_kernel<float><<<rows, kLpThreads, 0, st>>>(static_cast<const float*>(logits),
-                                                             vocab, row_stride, idx, out);
-  else
-    token_logprob_kernel<__nv_bfloat16><<<rows, kLpThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(logits), vocab, row_stride, idx, out);
   return status(cudaGetLastError());
 }
 

@@ -1,0 +1,483 @@
+// sampling.cu -- the stochastic variant of the Orthrus consensus (cjcn.com.cn
+// explainer of "Orthrus", §四: for sampling with a temperature the framework
+// aligns the two views' distributions by strict rejection sampling).
+// Declared in orthrus.h:
+//   orthrus_vocab_sample      draft tokens d_j ~ softmax(z_diff[j] / T) by Gumbel-max
+//   orthrus_token_logprob     log p(d_j), log q(d_j) and the rows' log-sum-exp at T
+//   orthrus_consensus_sample  accept while u_j < p/q, correction ~ normalize(max(0, p - q))
+// Random numbers: Philox4x32-10 (philox.cuh), counter layout in orthrus.h.
+#include "common.cuh"
+#include "philox.cuh"
+
+namespace orthrus {
+namespace {
+
+bool dtype_ok(int32_t t) { return t == ORTHRUS_F32 || t == ORTHRUS_BF16; }
+int status(cudaError_t e) { return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA; }
+
+// Keys ordering (value, lowest index first) as one unsigned 64-bit number.
+__device__ __forceinline__ unsigned long long order_key(float v, int j) {
+  if (v != v) return 0ull;  // NaN never wins
+  if (v == 0.f) v = 0.f;    // -0 == +0
+  unsigned u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (unsigned)j);
+}
+__device__ __forceinline__ int key_index(unsigned long long k) {
+  return (int)(0xFFFFFFFFu - (unsigned)(k & 0xFFFFFFFFull));
+}
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a,
+                                                     unsigned long long b) {
+  return a > b ? a : b;
+}
+__device__ __forceinline__ uint32_t word(const uint4& v, int e) {
+  return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+}
+
+// ------------------------------------------------------------ shared pieces
+// Every kernel here cuts rows into chunks of kChunk elements, one CTA per
+// (chunk, row), kPer elements per thread held in registers.
+constexpr int kThreads = 256;
+constexpr int kPer = 16;
+constexpr int kChunk = kThreads * kPer;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ float qnan() { return __int_as_float(0x7fc00000); }
+
+// Gumbel noise -log(-log u).  The inner log keeps full relative accuracy
+// (near u = 1, -log u ~ 1 - u is tiny and its relative error becomes the
+// noise's absolute error); the outer one needs only absolute accuracy.
+__device__ __forceinline__ float gumbel(uint32_t w) {
+  return -__logf(-logf(philox_uniform(w)));
+}
+
+// Block-wide max or sum in a fixed tree; every thread gets the result.
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    v = lane < kWarps ? red[lane] : (is_max ? -INFINITY : 0.f);
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, v, off);
+      v = is_max ? fmaxf(v, o) : v + o;
+    }
+    if (lane == 0) red[kWarps] = v;
+  }
+  __syncthreads();
+  const float res = red[kWarps];
+  __syncthreads();
+  return res;
+}
+
+// (max, sum of exp(x - max)) over the CTA's chunk.
+__device__ __forceinline__ float2 chunk_pair(const float (&x)[kPer], float m, float* red) {
+  m = block_reduce(m, true, red);
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) s += expf(x[e] - m);  // exp(-inf) = 0 past the row
+  return make_float2(m, block_reduce(s, false, red));
+}
+
+// One warp merges a row's chunk pairs -- lane i takes chunks i, i + 32, ...,
+// then a fixed shuffle tree -- and zeroes them (where pairs sit depends on
+// the call's shapes: a later call may read these bytes as counters).
+// Returns log sum_k exp(x_k) in every lane.
+__device__ __forceinline__ float merge_pairs(float2* pr, int nchunks, int lane) {
+  float M = -INFINITY;
+  for (int i = lane; i < nchunks; i += 32) M = fmaxf(M, __ldcg(&pr[i].x));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float S = 0.f;
+  for (int i = lane; i < nchunks; i += 32) {
+    const float2 q = __ldcg(&pr[i]);
+    S += q.y * expf(q.x - M);
+    pr[i] = make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
+  return M + logf(S);
+}
+
+__device__ __forceinline__ unsigned long long warp_max64(unsigned long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = umax64(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// ------------------------------------------------------------ draft sample
+// Thread t of chunk c takes the groups g = c * kChunk/4 + i * kThreads + t
+// (i < kPer/4), each the 4 consecutive elements one Philox call covers.  The
+// best (key, index) of the CTA goes to the row's slot by atomicMax; with kLse
+// the CTA also stores its chunk pair.  The row's last CTA (ticket) writes
+// idx, lse and logprob and returns slot and ticket to zero.
+template <typename T, bool kLse>
+__global__ void __launch_bounds__(kThreads)
+vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, float inv_t,
+                    uint32_t k0, uint32_t k1, uint32_t step, int nchunks,
+                    unsigned long long* keys, unsigned* tickets, float2* pairs,
+                    int32_t* __restrict__ idx, float* __restrict__ logprob,
+                    float* __restrict__ lse) {
+  __shared__ float red[kWarps + 1];
+  __shared__ unsigned long long wbest[kWarps];
+  __shared__ bool last;
+  const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, lane = t & 31;
+  const T* row = logits + (int64_t)r * stride;
+  float x[kPer];
+  float m = -INFINITY;
+  unsigned long long best = 0ull;
+#pragma unroll
+  for (int i = 0; i < kPer / 4; ++i) {
+    const int g = c * (kChunk / 4) + i * kThreads + t;
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step),
+                                  k0, k1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * g + e;
+      const bool in = j < vocab;
+      x[4 * i + e] = in ? to_f32(row[j]) * inv_t : -INFINITY;
+      m = fmaxf(m, x[4 * i + e]);
+      if (in) best = umax64(best, order_key(x[4 * i + e] + gumbel(word(w, e)), j));
+    }
+  }
+  best = warp_max64(best);
+  if (lane == 0) wbest[t >> 5] = best;
+  float2 pr = make_float2(0.f, 0.f);
+  if constexpr (kLse) pr = chunk_pair(x, m, red);  // its barriers publish wbest
+  else __syncthreads();
+  if (t == 0) {
+    for (int w = 1; w < kWarps; ++w) best = umax64(best, wbest[w]);
+    atomicMax(&keys[r], best);
+    if constexpr (kLse) pairs[(int64_t)r * nchunks + c] = pr;
+    __threadfence();
+    last = atomicAdd(&tickets[r], 1u) == (unsigned)nchunks - 1u;
+  }
+  __syncthreads();
+  if (!last || t >= 32) return;
+  __threadfence();
+  int j = 0;
+  if (lane == 0) {
+    const unsigned long long k = atomicExch(&keys[r], 0ull);
+    tickets[r] = 0u;
+    j = k ? key_index(k) : 0;
+    idx[r] = j;
+  }
+  if constexpr (kLse) {
+    const float l = merge_pairs(pairs + (int64_t)r * nchunks, nchunks, lane);
+    if (lane == 0) {
+      if (lse) lse[r] = l;
+      if (logprob) logprob[r] = to_f32(row[j]) * inv_t - l;
+    }
+  }
+}
+
+// ------------------------------------------------------------ log-prob at T
+// Grid (chunks, rows); element e of thread t is c * kChunk + e * kThreads + t
+// (coalesced).  The row's last CTA merges the chunk pairs.  Workspace:
+// tickets [rows] then the pairs [rows][chunks].
+template <typename T>
+__device__ __forceinline__ float load_chunk(const T* row, int c, int vocab, float inv_t,
+                                            float (&x)[kPer]) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int k = c * kChunk + e * kThreads + threadIdx.x;
+    x[e] = k < vocab ? to_f32(row[k]) * inv_t : -INFINITY;
+    m = fmaxf(m, x[e]);
+  }
+  return m;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
+                     const int32_t* __restrict__ idx, float inv_t, int nchunks,
+                     unsigned* tickets, float2* pairs, float* __restrict__ logprob,
+                     float* __restrict__ lse) {
+  __shared__ float red[kWarps + 1];
+  __shared__ bool last;
+  const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x;
+  const T* row = logits + (int64_t)r * stride;
+  float x[kPer];
+  const float2 pr = chunk_pair(x, load_chunk(row, c, vocab, inv_t, x), red);
+  if (t == 0) {
+    pairs[(int64_t)r * nchunks + c] = pr;
+    __threadfence();
+    last = atomicAdd(&tickets[r], 1u) == (unsigned)nchunks - 1u;
+  }
+  __syncthreads();
+  if (!last || t >= 32) return;
+  __threadfence();
+  const float l = merge_pairs(pairs + (int64_t)r * nchunks, nchunks, t);
+  if (t == 0) {
+    tickets[r] = 0u;
+    if (lse) lse[r] = l;
+    const int k = idx[r];
+    logprob[r] = (k >= 0 && k < vocab) ? to_f32(row[k]) * inv_t - l : qnan();
+  }
+}
+
+// ------------------------------------------------------ stochastic consensus
+// Launch 1, grid (chunks, B*blk) over the AR logits: log p_j(d_j) and the
+// row's log-sum-exp as in token_logprob_kernel; the CTA that merges a
+// sequence's last row (per-sequence ticket) then tests the acceptances of
+// the sequence in one warp: log u_j < log p_j(d_j) - log q_j(d_j), left to
+// right, and writes every output except the correction.
+// Launch 2, grid (chunks, B): Gumbel-max over the rejected row's residual
+// max(0, p - q) (the AR row's argmax as the fallback), folded per sequence
+// with atomicMax; the last CTA writes the correction.
+// Workspace: SeqSlot [B], row tickets [B*blk], chunk pairs [B*blk][chunks].
+struct SeqSlot {
+  uint32_t rows_done, ticket;
+  unsigned long long key_res, key_max;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+consensus_verify_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, float inv_t,
+                        int nchunks, SeqSlot* seq, unsigned* row_tickets, float2* pairs) {
+  __shared__ float red[kWarps + 1];
+  __shared__ bool last;
+  const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, blk = p.blk, b = r / blk;
+  const T* row = static_cast<const T*>(p.logits_ar) + (int64_t)r * p.row_stride;
+  float x[kPer];
+  const float2 pr = chunk_pair(x, load_chunk(row, c, p.vocab, inv_t, x), red);
+  if (t == 0) {
+    pairs[(int64_t)r * nchunks + c] = pr;
+    __threadfence();
+    last = atomicAdd(&row_tickets[r], 1u) == (unsigned)nchunks - 1u;
+  }
+  __syncthreads();
+  if (!last || t >= 32) return;
+  __threadfence();
+  const int lane = t;
+  const float l = merge_pairs(pairs + (int64_t)r * nchunks, nchunks, lane);
+  int seq_last = 0;
+  if (lane == 0) {
+    row_tickets[r] = 0u;
+    const int d = p.draft[r];
+    p.lse_ar[r] = l;
+    p.logp[r] = (d >= 0 && d < p.vocab) ? to_f32(row[d]) * inv_t - l : qnan();
+    __threadfence();
+    seq_last = atomicAdd(&seq[b].rows_done, 1u) == (unsigned)blk - 1u;
+  }
+  if (!__shfl_sync(0xffffffffu, seq_last, 0)) return;
+  __threadfence();
+  bool acc = true;
+  if (lane < blk) {
+    const int rj = b * blk + lane;
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)lane, (uint32_t)b, kPurposeAccept, p.step),
+                                  k0, k1);
+    acc = logf(philox_uniform(w.x)) < __ldcg(&p.logp[rj]) - p.logq[rj];  // NaN: reject
+  }
+  const unsigned miss = __ballot_sync(0xffffffffu, !acc);
+  const int L = miss ? __ffs(miss) - 1 : blk;
+  if (lane < blk) {
+    const int d = p.draft[(int64_t)b * blk + lane];
+    if (p.emitted && lane != L) p.emitted[(int64_t)b * blk + lane] = lane < L ? d : -1;
+    if (L == blk && lane == blk - 1 && p.next_anchor) p.next_anchor[b] = d;
+  }
+  if (lane == 0) {
+    seq[b].rows_done = 0u;
+    p.accept_len[b] = L;
+    p.n_emit[b] = min(L + 1, blk);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, float inv_t,
+                          int nchunks, SeqSlot* seq) {
+  __shared__ unsigned long long wres[kWarps], wmax[kWarps];
+  const int c = blockIdx.x, b = blockIdx.y, t = threadIdx.x, blk = p.blk;
+  const int L = p.accept_len[b];
+  if (L >= blk) return;  // every draft accepted: no correction
+  const int r = b * blk + L;
+  const T* za = static_cast<const T*>(p.logits_ar) + (int64_t)r * p.row_stride;
+  const T* zd = static_cast<const T*>(p.logits_diff) + (int64_t)r * p.row_stride;
+  const float la = p.lse_ar[r], ld = p.lse_diff[r];
+  unsigned long long best = 0ull, bmax = 0ull;
+#pragma unroll
+  for (int i = 0; i < kPer / 4; ++i) {
+    const int g = c * (kChunk / 4) + i * kThreads + t;
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)b, kPurposeResidual, p.step),
+                                  k0, k1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = 4 * g + e;
+      if (k < p.vocab) {
+        const float xa = to_f32(za[k]);
+        const float d = expf(xa * inv_t - la) - expf(to_f32(zd[k]) * inv_t - ld);
+        if (d > 0.f) best = umax64(best, order_key(logf(d) + gumbel(word(w, e)), k));
+        bmax = umax64(bmax, order_key(xa, k));
+      }
+    }
+  }
+  best = warp_max64(best);
+  bmax = warp_max64(bmax);
+  if ((t & 31) == 0) { wres[t >> 5] = best; wmax[t >> 5] = bmax; }
+  __syncthreads();
+  if (t != 0) return;
+  for (int i = 1; i < kWarps; ++i) {
+    best = umax64(best, wres[i]);
+    bmax = umax64(bmax, wmax[i]);
+  }
+  SeqSlot* sc = &seq[b];
+  atomicMax(&sc->key_res, best);
+  atomicMax(&sc->key_max, bmax);
+  __threadfence();
+  if (atomicAdd(&sc->ticket, 1u) == (unsigned)nchunks - 1u) {
+    const unsigned long long kr = atomicExch(&sc->key_res, 0ull);
+    const unsigned long long km = atomicExch(&sc->key_max, 0ull);
+    sc->ticket = 0u;
+    const int corr = kr ? key_index(kr) : key_index(km);
+    if (p.emitted) p.emitted[(int64_t)b * blk + L] = corr;
+    if (p.next_anchor) p.next_anchor[b] = corr;
+  }
+}
+
+size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
+constexpr int32_t kMaxVocab = 1 << 30;
+
+}  // namespace
+}  // namespace orthrus
+
+using namespace orthrus;
+
+extern "C" {
+
+size_t orthrus_vocab_sample_workspace(int32_t rows, int32_t vocab) {
+  if (rows < 0 || vocab <= 0 || vocab > kMaxVocab) return 0;
+  const int64_t nchunks = ceil_div(vocab, kChunk);
+  return round256((int64_t)rows * 8) + round256((int64_t)rows * 4) +
+         (size_t)((int64_t)rows * nchunks * 8);
+}
+
+int orthrus_vocab_sample(int32_t dtype, const void* logits, int32_t rows, int32_t vocab,
+                         int64_t row_stride, float temperature, uint64_t seed, uint32_t step,
+                         int32_t* idx, float* logprob, float* lse, void* workspace,
+                         size_t workspace_bytes, orthrus_stream_t stream) {
+  if (!dtype_ok(dtype) || rows < 0 || vocab <= 0 || row_stride < vocab ||
+      !(temperature > 0.f) || !isfinite(temperature))
+    return ORTHRUS_EINVAL;
+  if (vocab > kMaxVocab) return ORTHRUS_EUNSUPPORTED;
+  if (rows == 0) return ORTHRUS_OK;
+  if (!logits || !idx) return ORTHRUS_EINVAL;
+  if (!workspace || workspace_bytes < orthrus_vocab_sample_workspace(rows, vocab) ||
+      reinterpret_cast<uintptr_t>(workspace) % 16)
+    return ORTHRUS_EWORKSPACE;
+  if (rows > 65535) return ORTHRUS_EUNSUPPORTED;
+  char* ws = static_cast<char*>(workspace);
+  auto keys = reinterpret_cast<unsigned long long*>(ws);
+  auto tickets = reinterpret_cast<unsigned*>(ws + round256((int64_t)rows * 8));
+  auto pairs = reinterpret_cast<float2*>(ws + round256((int64_t)rows * 8) +
+                                         round256((int64_t)rows * 4));
+  const int nchunks = ceil_div(vocab, kChunk);
+  const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  const float inv_t = 1.f / temperature;
+  const bool want = logprob || lse;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(nchunks, rows);
+#define ORTHRUS_SAMPLE(T, L)                                                              \
+  vocab_sample_kernel<T, L><<<grid, kThreads, 0, st>>>(                                   \
+      static_cast<const T*>(logits), vocab, row_stride, inv_t, k0, k1, step, nchunks, keys, \
+      tickets, pairs, idx, logprob, lse)
+  if (dtype == ORTHRUS_F32) {
+    if (want) ORTHRUS_SAMPLE(float, true); else ORTHRUS_SAMPLE(float, false);
+  } else {
+    if (want) ORTHRUS_SAMPLE(__nv_bfloat16, true); else ORTHRUS_SAMPLE(__nv_bfloat16, false);
+  }
+#undef ORTHRUS_SAMPLE
+  return status(cudaGetLastError());
+}
+
+size_t orthrus_token_logprob_workspace(int32_t rows, int32_t vocab) {
+  if (rows < 0 || vocab <= 0 || vocab > kMaxVocab) return 0;
+  const int64_t nchunks = ceil_div(vocab, kChunk);
+  return round256((int64_t)rows * 4) + (size_t)((int64_t)rows * nchunks * 8);
+}
+
+int orthrus_token_logprob(int32_t dtype, const void* logits, int32_t rows, int32_t vocab,
+                          int64_t row_stride, const int32_t* idx, float temperature,
+                          float* logprob, float* lse, void* workspace, size_t workspace_bytes,
+                          orthrus_stream_t stream) {
+  if (!dtype_ok(dtype) || rows < 0 || vocab <= 0 || row_stride < vocab ||
+      !(temperature > 0.f) || !isfinite(temperature))
+    return ORTHRUS_EINVAL;
+  if (vocab > kMaxVocab) return ORTHRUS_EUNSUPPORTED;
+  if (rows == 0) return ORTHRUS_OK;
+  if (!logits || !idx || !logprob) return ORTHRUS_EINVAL;
+  if (!workspace || workspace_bytes < orthrus_token_logprob_workspace(rows, vocab) ||
+      reinterpret_cast<uintptr_t>(workspace) % 16)
+    return ORTHRUS_EWORKSPACE;
+  if (rows > 65535) return ORTHRUS_EUNSUPPORTED;
+  const int nchunks = ceil_div(vocab, kChunk);
+  auto tickets = static_cast<unsigned*>(workspace);
+  auto pairs = reinterpret_cast<float2*>(static_cast<char*>(workspace) +
+                                         round256((int64_t)rows * 4));
+  const float inv_t = 1.f / temperature;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(nchunks, rows);
+  if (dtype == ORTHRUS_F32)
+    token_logprob_kernel<float><<<grid, kThreads, 0, st>>>(
+        static_cast<const float*>(logits), vocab, row_stride, idx, inv_t, nchunks, tickets,
+        pairs, logprob, lse);
+  else
+    token_logprob_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(logits), vocab, row_stride, idx, inv_t, nchunks,
+        tickets, pairs, logprob, lse);
+  return status(cudaGetLastError());
+}
+
+size_t orthrus_consensus_sample_workspace(int32_t B, int32_t blk, int32_t vocab) {
+  if (B < 0 || blk < 1 || vocab <= 0 || vocab > kMaxVocab) return 0;
+  const int64_t rows = (int64_t)B * blk, nchunks = ceil_div(vocab, kChunk);
+  return round256((int64_t)B * sizeof(SeqSlot)) + round256(rows * 4) +
+         (size_t)(rows * nchunks * 8);
+}
+
+int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stream) {
+  if (!a || !dtype_ok(a->dtype) || a->B < 0 || a->blk < 1 || a->vocab <= 0 ||
+      a->row_stride < a->vocab || !(a->temperature > 0.f) || !isfinite(a->temperature))
+    return ORTHRUS_EINVAL;
+  if (a->blk > 32 || a->vocab > kMaxVocab) return ORTHRUS_EUNSUPPORTED;
+  if (a->B == 0) return ORTHRUS_OK;
+  if (!a->draft || !a->logq || !a->lse_diff || !a->logits_ar || !a->logits_diff ||
+      !a->logp || !a->lse_ar || !a->accept_len || !a->n_emit)
+    return ORTHRUS_EINVAL;
+  if (!a->workspace ||
+      a->workspace_bytes < orthrus_consensus_sample_workspace(a->B, a->blk, a->vocab) ||
+      reinterpret_cast<uintptr_t>(a->workspace) % 16)
+    return ORTHRUS_EWORKSPACE;
+  const int64_t rows = (int64_t)a->B * a->blk;
+  if (rows > 65535) return ORTHRUS_EUNSUPPORTED;
+  const uint32_t k0 = (uint32_t)a->seed, k1 = (uint32_t)(a->seed >> 32);
+  char* ws = static_cast<char*>(a->workspace);
+  auto seq = reinterpret_cast<SeqSlot*>(ws);
+  auto row_tickets = reinterpret_cast<unsigned*>(ws + round256((int64_t)a->B * sizeof(SeqSlot)));
+  auto pairs = reinterpret_cast<float2*>(ws + round256((int64_t)a->B * sizeof(SeqSlot)) +
+                                         round256(rows * 4));
+  const int nchunks = ceil_div(a->vocab, kChunk);
+  const float inv_t = 1.f / a->temperature;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 g1(nchunks, (unsigned)rows), g2(nchunks, a->B);
+  if (a->dtype == ORTHRUS_F32) {
+    consensus_verify_kernel<float><<<g1, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks, seq,
+                                                             row_tickets, pairs);
+    consensus_residual_kernel<float><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks, seq);
+  } else {
+    consensus_verify_kernel<__nv_bfloat16><<<g1, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks,
+                                                                     seq, row_tickets, pairs);
+    consensus_residual_kernel<__nv_bfloat16><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t,
+                                                                      nchunks, seq);
+  }
+  return status(cudaGetLastError());
+}
+
+}  // extern "C"

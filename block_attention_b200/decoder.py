@@ -174,15 +174,38 @@ class TinyDecoder:
         toks = out.t().contiguous().cpu().numpy()
         return (toks, lp.t().contiguous().cpu().numpy()) if logprob else toks
 
+    def sample_ar(self, prompts, n_new: int, temperature: float, seed: int,
+                  cap: int | None = None) -> np.ndarray:
+        """Plain autoregressive sampling at ``temperature``, one token per
+        forward (the first token is the prefill's greedy one, as in the
+        loop): int32 [B, n_new].  Step t uses Philox step t of ``seed``."""
+        cap = cap or max(len(p) for p in prompts) + n_new + 64
+        st, first, _ = self.prefill(prompts, cap)
+        B = st.B
+        out = torch.empty(n_new, B, dtype=torch.int32, device=self.device)
+        out[0].copy_(torch.from_numpy(first))
+        ones = torch.ones(B, dtype=torch.int32, device=self.device)
+        for t in range(1, n_new):
+            logits, kb, vb = self.forward(st, out[t - 1].view(B, 1), AR_VIEW)
+            ba.vocab_sample(logits, temperature, seed, t, idx=out[t])
+            self.commit(st, kb, vb, ones)
+        self.check(st)
+        return out.t().contiguous().cpu().numpy()
+
     # ----------------------------------------------------- consensus loop
     def consensus(self, prompts, n_new: int, blk: int = 32, draft_fn=None,
-                  cap: int | None = None):
+                  cap: int | None = None, temperature: float = 0.0, seed: int = 0):
         """The Orthrus loop: int32 [B, n_new] tokens and per-round stats.
 
         ``draft_fn(counts, d)`` may replace the diffusion drafts d (device
         int32 [B, blk]) given each sequence's emitted-token count, to show
-        that any draft gives the greedy trajectory.  Sequences that reach
-        n_new tokens stop committing; the loop ends when all have."""
+        that any draft gives the greedy trajectory.  With ``temperature`` > 0
+        the round samples instead (explainer §四): drafts d_j ~ softmax of the
+        diffusion logits / T, and the stochastic consensus accepts d_j with
+        probability min(1, p_j(d_j) / q_j(d_j)) and draws the correction from
+        normalize(max(0, p - q)); round r uses Philox step r of ``seed``.
+        Sequences that reach n_new tokens stop committing; the loop ends when
+        all have."""
         cap = cap or max(len(p) for p in prompts) + n_new + 2 * blk
         st, first, _ = self.prefill(prompts, cap)
         B = st.B
@@ -194,13 +217,28 @@ class TinyDecoder:
             active = counts < n_new
             dtok = ba.block_tokens(anchor, None, blk, self.mask_id)
             dlog, _, _ = self.forward(st, dtok, DIFFUSION_VIEW)
-            d = ba.vocab_argmax(dlog).view(B, blk)
+            step = stats["rounds"]
+            if temperature > 0:
+                rows = B * blk
+                logq = torch.empty(rows, dtype=torch.float32, device=self.device)
+                lse_d = torch.empty_like(logq)
+                d = ba.vocab_sample(dlog, temperature, seed, step, logprob=logq,
+                                    lse=lse_d).view(B, blk)
+            else:
+                d = ba.vocab_argmax(dlog).view(B, blk)
             if draft_fn is not None:
                 d = draft_fn(counts, d)
             vtok = ba.block_tokens(anchor, d, blk, self.mask_id)
             vlog, kb, vb = self.forward(st, vtok, AR_VIEW)
-            a = ba.vocab_argmax(vlog).view(B, blk)
-            acc, ne, em, na = ba.consensus(d, a)
+            if temperature > 0:
+                if draft_fn is not None:  # replaced drafts: their log q under the diffusion view
+                    ba.token_logprob(dlog, d.reshape(-1).contiguous(), temperature=temperature,
+                                     out=logq, lse=lse_d)
+                acc, ne, em, na = ba.consensus_sample(d.contiguous(), vlog, dlog, logq, lse_d,
+                                                      temperature, seed, step)
+            else:
+                a = ba.vocab_argmax(vlog).view(B, blk)
+                acc, ne, em, na = ba.consensus(d, a)
             ne_h, em_h, acc_h = ne.cpu().numpy(), em.cpu().numpy(), acc.cpu().numpy()
             commit = np.where(active, ne_h, 0).astype(np.int32)
             self.commit(st, kb, vb, torch.from_numpy(commit).to(self.device))

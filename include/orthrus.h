@@ -214,6 +214,96 @@ size_t orthrus_kv_commit_workspace(const orthrus_commit_args* a);
 
 int orthrus_kv_commit(const orthrus_commit_args* a, orthrus_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Stochastic consensus (explainer §四: for sampling with a temperature the
+ * framework aligns the two views' distributions by strict rejection
+ * sampling, which keeps decoding lossless).  Per sequence, with
+ * q_j = softmax(z_diff[j] / T) and p_j = softmax(z_ar[j] / T):
+ *   drafts      d_j ~ q_j                               (orthrus_vocab_sample)
+ *   accept      d_j while u_j < p_j(d_j) / q_j(d_j), left to right
+ *   correction  at the first rejected position L: c ~ normalize(max(0, p_L - q_L))
+ *   emit        d_0 .. d_{L-1}, c (n_emit = L + 1), or all blk drafts when every
+ *               one is accepted (n_emit = min(L + 1, blk), as in the greedy rule)
+ * Sampling from a softmax uses Gumbel-max: argmax_k x_k + g_k with
+ * g_k = -log(-log u_k).  Uniforms: Philox4x32-10 (Salmon et al., SC'11) with
+ * key = seed (low, high 32 bits) and counter (x0, x1, purpose, step):
+ * purpose 1 draft noise (x0 = vocab index / 4, x1 = row, word = index % 4),
+ * purpose 2 acceptance (x0 = block position, x1 = sequence, word 0), purpose 3
+ * correction noise (x0 = vocab index / 4, x1 = sequence); a word w becomes
+ * u = ((w >> 9) + 1/2) 2^-23 (exact in FP32).  `step` must differ between rounds.  z / T is an
+ * FP32 division; reductions are FP32.
+ * ---------------------------------------------------------------------- */
+
+/* Draft sampling, with the draft's log-probability from the same read:
+ *   idx[r]     = argmax_k logits[r, k] / T + g_k (purpose 1, x1 = r), lowest
+ *                index on equal keys
+ *   lse[r]     = log sum_k exp(logits[r, k] / T)          (nullable)
+ *   logprob[r] = logits[r, idx[r]] / T - lse[r]           (nullable)
+ * temperature > 0 and finite; vocab <= 2^30.  Grid: 4096-element chunks x
+ * rows; each CTA folds its best key into the row's slot with an atomic max
+ * and, when lse or logprob is wanted, stores its chunk's maximum and sum of
+ * exponentials; the row's last CTA writes idx and merges the chunk pairs in
+ * a fixed order.  workspace: orthrus_vocab_sample_workspace(rows, vocab)
+ * bytes, 16-byte aligned, zeroed once; every call leaves it all zero. */
+size_t orthrus_vocab_sample_workspace(int32_t rows, int32_t vocab);
+int orthrus_vocab_sample(int32_t dtype, const void* logits, int32_t rows, int32_t vocab,
+                         int64_t row_stride, float temperature, uint64_t seed, uint32_t step,
+                         int32_t* idx, float* logprob, float* lse, void* workspace,
+                         size_t workspace_bytes, orthrus_stream_t stream);
+
+/* Log-probability of a chosen token per row at temperature T:
+ *   lse[r]     = log sum_k exp(logits[r, k] / T)
+ *   logprob[r] = logits[r, idx[r]] / T - lse[r]
+ * idx int32 [rows] device, each in [0, vocab) (else logprob[r] = NaN); lse
+ * nullable.  Rows are cut into 4096-element chunks; each chunk's maximum and
+ * sum of exp(z/T - max) are reduced in FP32 in a fixed order and the chunks
+ * are merged in index order, so the result depends only on the row.  T = 1
+ * gives the plain log-softmax the precision study uses (the reproduction "How
+ * Lossless Is Lossless Speculative Decoding? The Role of Numerical Precision
+ * in Orthrus", abstract, relates exact trajectory matching to the reference's
+ * perplexity).  workspace: orthrus_token_logprob_workspace(rows, vocab) bytes,
+ * 16-byte aligned, zeroed once: every call leaves it all zero, so one buffer
+ * serves later calls of any shape on the same stream. */
+size_t orthrus_token_logprob_workspace(int32_t rows, int32_t vocab);
+int orthrus_token_logprob(int32_t dtype, const void* logits, int32_t rows, int32_t vocab,
+                          int64_t row_stride, const int32_t* idx, float temperature,
+                          float* logprob, float* lse, void* workspace, size_t workspace_bytes,
+                          orthrus_stream_t stream);
+
+typedef struct orthrus_sample_args {
+  int32_t dtype;          /* of both logit matrices */
+  int32_t B, blk, vocab;  /* 1 <= blk <= 32, B * blk <= 65535, vocab <= 2^30 */
+  int64_t row_stride;     /* elements between logit rows, >= vocab */
+  float temperature;      /* > 0 */
+  uint32_t step;
+  uint64_t seed;
+  const int32_t* draft;   /* [B, blk] d_j: orthrus_vocab_sample of logits_diff ... */
+  const float* logq;      /* [B*blk] log q_j(d_j): ... its logprob output */
+  const float* lse_diff;  /* [B*blk] log-sum-exp of logits_diff / T: ... its lse output */
+  const void* logits_ar;  /* [B*blk, vocab] row b*blk + j: AR view */
+  const void* logits_diff;/* [B*blk, vocab] diffusion view */
+  float* logp;            /* out [B*blk] log p_j(d_j) */
+  float* lse_ar;          /* out [B*blk] log-sum-exp of logits_ar / T */
+  int32_t* accept_len;    /* out [B] L */
+  int32_t* n_emit;        /* out [B] */
+  int32_t* emitted;       /* out [B, blk] (nullable), -1 past n_emit */
+  int32_t* next_anchor;   /* out [B] (nullable) */
+  void* workspace;        /* orthrus_consensus_sample_workspace(B, blk, vocab) bytes,
+                             16-byte aligned, zeroed once; left all zero */
+  size_t workspace_bytes;
+} orthrus_sample_args;
+
+/* Outputs as orthrus_consensus.  Two launches.  (1) Grid 4096-element chunks
+ * x rows over logits_ar: log p_j(d_j) and the row's log-sum-exp (chunk pairs
+ * merged in a fixed order by the row's last CTA); the CTA that completes a
+ * sequence's last row then runs its acceptance test in one warp.  (2) Grid
+ * chunks x sequences: Gumbel-max over the rejected row's max(0, p - q),
+ * folded per sequence with an atomic max; the last CTA writes the
+ * correction.  When no token has p > q at the rejected position (impossible
+ * in exact arithmetic) the correction is argmax p. */
+size_t orthrus_consensus_sample_workspace(int32_t B, int32_t blk, int32_t vocab);
+int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 const char* orthrus_status_str(int status);
 int orthrus_version(void);

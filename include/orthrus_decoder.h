@@ -88,19 +88,6 @@ int orthrus_block_tokens(const int32_t* anchor, const int32_t* draft, int32_t B,
                          int32_t blk, int32_t mask_id, int32_t* out,
                          orthrus_stream_t stream);
 
-/* Log-probability of a chosen token per row, for the precision study (the
- * reproduction "How Lossless Is Lossless Speculative Decoding? The Role of
- * Numerical Precision in Orthrus", abstract, ties exact trajectory matching
- * to the reference model's response-conditional perplexity):
- *   out[r] = logits[r, idx[r]] - log(sum_j exp(logits[r, j]))
- * logits [rows, vocab] with row stride row_stride (>= vocab); idx int32 [rows]
- * device, each in [0, vocab) (else out[r] = NaN); out float [rows].  The row
- * maximum and the sum of exponentials are reduced in FP32 in an order fixed by
- * vocab (one CTA per row). */
-int orthrus_token_logprob(int32_t dtype, const void* logits, int32_t rows, int32_t vocab,
-                          int64_t row_stride, const int32_t* idx, float* out,
-                          orthrus_stream_t stream);
-
 #ifdef __cplusplus
 }
 #endif

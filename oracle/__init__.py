@@ -109,23 +109,26 @@ def block_attn(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode,
     return out
 
 
-def token_logprob(logits, idx):
-    """Log-softmax of each row at idx, in float64: x[idx] - (m + log(sum exp(x - m)))
-    with m the row maximum (the definition; no blocking).  bf16 bit patterns
-    (uint16) are widened exactly.  idx outside [0, vocab) gives NaN."""
+def token_logprob(logits, idx, temperature=1.0, return_lse=False):
+    """Log-softmax of each row of logits / temperature at idx, in float64:
+    s[idx] - lse with s = x / T and lse = m + log(sum exp(s - m)), m the row
+    maximum (the definition; no blocking).  bf16 bit patterns (uint16) are
+    widened exactly.  idx outside [0, vocab) gives NaN."""
     x = np.asarray(logits)
     if x.dtype == np.uint16:
         x = (x.astype(np.uint32) << 16).view(np.float32)
-    x = x.astype(np.float64)
+    x = x.astype(np.float64) / temperature
     idx = np.asarray(idx, np.int64)
     rows, vocab = x.shape
     out = np.full(rows, np.nan)
+    lse = np.zeros(rows)
     for r in range(rows):
+        m = x[r].max()
+        lse[r] = m + np.log(np.exp(x[r] - m).sum())
         k = int(idx[r])
         if 0 <= k < vocab:
-            m = x[r].max()
-            out[r] = x[r, k] - (m + np.log(np.exp(x[r] - m).sum()))
-    return out
+            out[r] = x[r, k] - lse[r]
+    return (out, lse) if return_lse else out
 
 
 def vocab_argmax(logits, return_max=False):

@@ -66,6 +66,11 @@ int main(void) {
   F(orthrus_commit_args, k_cache); F(orthrus_commit_args, cache_layer_stride);
   F(orthrus_commit_args, blk_layer_stride); F(orthrus_commit_args, n_emit);
   F(orthrus_commit_args, workspace_bytes);
+  printf("orthrus_sample_args size %zu\n", sizeof(orthrus_sample_args));
+  F(orthrus_sample_args, row_stride); F(orthrus_sample_args, temperature);
+  F(orthrus_sample_args, step); F(orthrus_sample_args, seed); F(orthrus_sample_args, draft);
+  F(orthrus_sample_args, logits_diff); F(orthrus_sample_args, next_anchor);
+  F(orthrus_sample_args, workspace_bytes);
   return 0;
 }''')
     exe = tmp_path / "layout"
@@ -75,7 +80,8 @@ int main(void) {
     for line in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines():
         t, m, v = line.split()
         got[(t, m)] = int(v)
-    cls = {"orthrus_attn_args": ba.AttnArgs, "orthrus_commit_args": ba.CommitArgs}
+    cls = {"orthrus_attn_args": ba.AttnArgs, "orthrus_commit_args": ba.CommitArgs,
+           "orthrus_sample_args": ba.SampleArgs}
     for (t, m), v in got.items():
         c = cls[t]
         assert (ctypes.sizeof(c) if m == "size" else getattr(c, m).offset) == v, (t, m)
@@ -172,3 +178,45 @@ def test_decoder_entry_points_host_checks(L):
     assert L.orthrus_block_tokens(vp(256), None, 1, 33, 0, vp(256), None) == -1
     assert L.orthrus_block_tokens(None, None, 1, 32, 0, vp(256), None) == -1
     assert L.orthrus_block_tokens(None, None, 0, 32, 0, None, None) == 0
+
+
+def test_sampling_entry_points_host_checks(L):
+    c = ctypes
+    vp = c.c_void_p
+    ws = L.orthrus_vocab_sample_workspace(4, 10)
+    assert ws >= 4 * 8 + 4 * 4 + 4 * 8  # keys, tickets, one chunk pair per row
+    # temperature must be positive and finite
+    for T in (0.0, -1.0, float("inf"), float("nan")):
+        assert L.orthrus_vocab_sample(0, vp(256), 4, 10, 10, c.c_float(T), 1, 0, vp(256),
+                                      None, None, vp(256), ws, None) == -1
+        assert L.orthrus_token_logprob(0, vp(256), 4, 10, 10, vp(256), c.c_float(T), vp(256),
+                                       None, vp(256), 1 << 20, None) == -1
+    assert L.orthrus_vocab_sample(0, vp(256), 4, 10, 10, c.c_float(1.0), 1, 0, vp(256),
+                                  None, None, vp(256), ws - 1, None) == -3  # workspace
+    assert L.orthrus_vocab_sample(0, vp(256), 4, 10, 10, c.c_float(1.0), 1, 0, vp(256),
+                                  None, None, vp(264), ws, None) == -3  # 16-byte alignment
+    assert L.orthrus_vocab_sample(0, None, 0, 10, 10, c.c_float(1.0), 1, 0, None, None, None,
+                                  None, 0, None) == 0
+    assert L.orthrus_vocab_sample(0, vp(256), 4, (1 << 30) + 1, (1 << 30) + 1, c.c_float(1.0),
+                                  1, 0, vp(256), None, None, vp(256), 1 << 40, None) == -2
+    a = ba.SampleArgs(dtype=0, B=1, blk=33, vocab=10, row_stride=10, temperature=1.0)
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == -2  # blk > 32
+    a.blk = 4
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == -1  # null tensors
+    for f in ("draft", "logq", "lse_diff", "logits_ar", "logits_diff", "logp", "lse_ar",
+              "n_emit"):
+        setattr(a, f, 4096)
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == -1  # accept_len is required
+    a.accept_len = 4096
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == -3  # no workspace
+    a.workspace, a.workspace_bytes = 4096, L.orthrus_consensus_sample_workspace(1, 4, 10)
+    a.B, a.blk = 2048, 32
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == -3  # too small for B = 2048
+    a.workspace_bytes = L.orthrus_consensus_sample_workspace(2048, 32, 10)
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == -2  # B * blk > 65535
+    a.B, a.blk = 1, 4
+    assert L.orthrus_token_logprob(0, vp(256), 4, 10, 10, vp(256), c.c_float(1.0), vp(256),
+                                   None, None, 0, None) == -3
+    assert L.orthrus_consensus_sample_workspace(4, 8, 10) >= 4 * 24 + 32 * 4 + 32 * 8
+    a.B = 0
+    assert L.orthrus_consensus_sample(ctypes.byref(a), None) == 0

@@ -181,3 +181,19 @@ def test_greedy_logprobs_bounded(model32, prompts):
     assert toks.shape == lp.shape == (8, 24)
     assert np.isfinite(lp).all()
     assert (lp <= 1e-6).all() and (lp >= -np.log(E["V"]) - 1e-4).all()
+
+
+def test_fp32_stochastic_loop_at_tiny_temperature_is_greedy(model32, prompts, greedy32):
+    """At a temperature far below every logit gap, sampling is argmax and the
+    stochastic consensus is the greedy one: the loop reproduces greedy AR."""
+    toks, st = model32.consensus(prompts[:8], 48, blk=E["blk"], temperature=1e-6, seed=3)
+    np.testing.assert_array_equal(toks, greedy32[:8, :48])
+
+
+def test_stochastic_loop_runs_and_emits_valid_tokens(model32, prompts):
+    toks, st = model32.consensus(prompts[:16], 64, blk=E["blk"], temperature=1.0, seed=11)
+    assert toks.shape == (16, 64)
+    assert ((toks >= 0) & (toks < E["V"])).all()
+    assert min(st["accept_len"]) >= 0 and st["tokens_per_forward"] >= 0.5
+    ar = model32.sample_ar(prompts[:16], 64, temperature=1.0, seed=11)
+    assert ((ar >= 0) & (ar < E["V"])).all()
