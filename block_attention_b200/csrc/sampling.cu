@@ -113,12 +113,16 @@ __device__ __forceinline__ unsigned long long warp_max64(unsigned long long v) {
 
 // ------------------------------------------------------------ draft sample
 // Thread t of chunk c takes the groups g = c * kChunk/4 + i * kThreads + t
-// (i < kPer/4), each the 4 consecutive elements one Philox call covers.  The
-// best (key, index) of the CTA goes to the row's slot by atomicMax; with kLse
+// (i < kPer/4), each the 4 consecutive elements one Philox call covers.  A
+// thread visits its elements in increasing index, so it keeps its best as a
+// (value, index) pair replaced only by a strictly larger value (NaN never
+// wins; equal values keep the lower index) and forms the 64-bit order key
+// once.  The best (key, index) of the CTA goes to the row's slot by
+// atomicMax; with kLse
 // the CTA also stores its chunk pair.  The row's last CTA (ticket) writes
 // idx, lse and logprob and returns slot and ticket to zero.
 template <typename T, bool kLse>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 8)  // 8 CTAs (2048 threads) per SM
 vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, float inv_t,
                     uint32_t k0, uint32_t k1, uint32_t step, int nchunks,
                     unsigned long long* keys, unsigned* tickets, float2* pairs,
@@ -130,8 +134,8 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, lane = t & 31;
   const T* row = logits + (int64_t)r * stride;
   float x[kPer];
-  float m = -INFINITY;
-  unsigned long long best = 0ull;
+  float m = -INFINITY, bv = -INFINITY;
+  int bi = -1;
 #pragma unroll
   for (int i = 0; i < kPer / 4; ++i) {
     const int g = c * (kChunk / 4) + i * kThreads + t;
@@ -143,9 +147,13 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
       const bool in = j < vocab;
       x[4 * i + e] = in ? to_f32(row[j]) * inv_t : -INFINITY;
       m = fmaxf(m, x[4 * i + e]);
-      if (in) best = umax64(best, order_key(x[4 * i + e] + gumbel(word(w, e)), j));
+      const float key = x[4 * i + e] + gumbel(word(w, e));
+      if (in && (key > bv || bi < 0)) {
+        if (key == key) { bv = key; bi = j; }
+      }
     }
   }
+  unsigned long long best = bi < 0 ? 0ull : order_key(bv, bi);
   best = warp_max64(best);
   if (lane == 0) wbest[t >> 5] = best;
   float2 pr = make_float2(0.f, 0.f);
@@ -229,10 +237,14 @@ token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
 // sequence's last row (per-sequence ticket) then tests the acceptances of
 // the sequence in one warp: log u_j < log p_j(d_j) - log q_j(d_j), left to
 // right, and writes every output except the correction.
-// Launch 2, grid (chunks, B): Gumbel-max over the rejected row's residual
+// Launch 2, grid (kResChunk-element chunks, B): one group of four per thread,
+// so the two rows' work spreads over about one wave; Gumbel-max over the
+// rejected row's residual
 // max(0, p - q) (the AR row's argmax as the fallback), folded per sequence
 // with atomicMax; the last CTA writes the correction.
 // Workspace: SeqSlot [B], row tickets [B*blk], chunk pairs [B*blk][chunks].
+constexpr int kResChunk = kThreads * 4;
+
 struct SeqSlot {
   uint32_t rows_done, ticket;
   unsigned long long key_res, key_max;
@@ -303,20 +315,17 @@ consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1,
   const T* zd = static_cast<const T*>(p.logits_diff) + (int64_t)r * p.row_stride;
   const float la = p.lse_ar[r], ld = p.lse_diff[r];
   unsigned long long best = 0ull, bmax = 0ull;
+  const int g = c * (kResChunk / 4) + t;
+  const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)b, kPurposeResidual, p.step),
+                                k0, k1);
 #pragma unroll
-  for (int i = 0; i < kPer / 4; ++i) {
-    const int g = c * (kChunk / 4) + i * kThreads + t;
-    const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)b, kPurposeResidual, p.step),
-                                  k0, k1);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = 4 * g + e;
-      if (k < p.vocab) {
-        const float xa = to_f32(za[k]);
-        const float d = expf(xa * inv_t - la) - expf(to_f32(zd[k]) * inv_t - ld);
-        if (d > 0.f) best = umax64(best, order_key(logf(d) + gumbel(word(w, e)), k));
-        bmax = umax64(bmax, order_key(xa, k));
-      }
+  for (int e = 0; e < 4; ++e) {
+    const int k = 4 * g + e;
+    if (k < p.vocab) {
+      const float xa = to_f32(za[k]);
+      const float d = expf(xa * inv_t - la) - expf(to_f32(zd[k]) * inv_t - ld);
+      if (d > 0.f) best = umax64(best, order_key(logf(d) + gumbel(word(w, e)), k));
+      bmax = umax64(bmax, order_key(xa, k));
     }
   }
   best = warp_max64(best);
@@ -466,16 +475,17 @@ int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stre
   const int nchunks = ceil_div(a->vocab, kChunk);
   const float inv_t = 1.f / a->temperature;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  const dim3 g1(nchunks, (unsigned)rows), g2(nchunks, a->B);
+  const int nres = ceil_div(a->vocab, kResChunk);
+  const dim3 g1(nchunks, (unsigned)rows), g2(nres, a->B);
   if (a->dtype == ORTHRUS_F32) {
     consensus_verify_kernel<float><<<g1, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks, seq,
                                                              row_tickets, pairs);
-    consensus_residual_kernel<float><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks, seq);
+    consensus_residual_kernel<float><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t, nres, seq);
   } else {
     consensus_verify_kernel<__nv_bfloat16><<<g1, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks,
                                                                      seq, row_tickets, pairs);
     consensus_residual_kernel<__nv_bfloat16><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t,
-                                                                      nchunks, seq);
+                                                                      nres, seq);
   }
   return status(cudaGetLastError());
 }

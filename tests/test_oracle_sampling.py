@@ -102,3 +102,17 @@ def test_identical_views_accept_every_draft():
     assert (L == blk).all() and (ne == blk).all()
     np.testing.assert_array_equal(em, draft.reshape(B, blk))
     np.testing.assert_array_equal(na, draft.reshape(B, blk)[:, -1])
+
+
+def test_token_logprob_temperature_and_lse_match_scipy(oracle_mod):
+    """The temperature path of the log-probability (used by the stochastic
+    consensus) against scipy's logsumexp of the scaled row."""
+    from scipy.special import logsumexp
+    g = np.random.default_rng(13)
+    x = g.normal(0, 3, (5, 777))
+    idx = g.integers(0, 777, 5)
+    for T in (0.3, 1.0, 2.5):
+        lp, lse = oracle_mod.token_logprob(x, idx, temperature=T, return_lse=True)
+        ref_lse = logsumexp(x / T, axis=1)
+        np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lp, x[np.arange(5), idx] / T - ref_lse, rtol=0, atol=1e-12)
