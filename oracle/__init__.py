@@ -146,6 +146,42 @@ def vocab_argmax(logits, return_max=False):
     return (idx, mx) if return_max else idx
 
 
+def _widen64(x):
+    x = np.asarray(x)
+    if x.dtype == np.uint16:  # bf16 bit patterns
+        x = (x.astype(np.uint32) << 16).view(np.float32)
+    return x.astype(np.float64)
+
+
+def lm_head_argmax(h, w, chunk=8192):
+    """The LM head feeding the round's argmax, without the logits leaving it:
+    logits[r, v] = sum_k h[r, k] w[v, k] in float64 (the product of the
+    final hidden states with the output embedding; bf16 bit patterns widened
+    exactly), then each row's argmax with the lowest index among equal maxima
+    (vocab_argmax).  Returns (idx int32 [rows], max float64 [rows], gap
+    float64 [rows], mag float64 [rows]): gap = distance between the row's two
+    largest logits, mag = max_v sum_k |h[r, k]| |w[v, k]|, the scale of the
+    rounding error of any lower-precision evaluation of the row.  The product
+    is taken over vocabulary slices of `chunk` rows (a memory bound only: each
+    logit is one complete dot product)."""
+    H, W = _widen64(h), _widen64(w)
+    rows, V = H.shape[0], W.shape[0]
+    logits = np.empty((rows, V))
+    mag = np.zeros(rows)
+    aH = np.abs(H)
+    for c0 in range(0, V, chunk):
+        Wc = W[c0:c0 + chunk]
+        logits[:, c0:c0 + chunk] = H @ Wc.T
+        mag = np.maximum(mag, (aH @ np.abs(Wc).T).max(axis=1))
+    idx, mx = vocab_argmax(logits, return_max=True)
+    if V > 1:
+        top2 = np.partition(logits, V - 2, axis=1)[:, -2:]
+        gap = top2[:, 1] - top2[:, 0]
+    else:
+        gap = np.full(rows, np.inf)
+    return idx, mx, gap, mag
+
+
 def consensus(draft, verify):
     """(accept_len [B], n_emit [B], emitted [B, blk] (-1 padded), next_anchor [B])."""
     d = np.ascontiguousarray(draft, dtype=np.int32)
