@@ -274,6 +274,54 @@ def sampling_kernels(args):
                       "us_per_launch": res}), flush=True)
 
 
+def lm_head_kernel(args):
+    """The Qwen3-8B LM head with the argmax fused in its epilogue (d 4096,
+    vocabulary 151936, bf16) for 32 and 128 hidden rows (one and four
+    32-row blocks), against the unfused pair a round would otherwise run: a
+    cuBLAS bf16 GEMM writing the logits, then this library's vocab_argmax.
+    The 1.24 GB output embedding is larger than L2, so every launch streams
+    it from HBM.  Algorithmic bytes: the embedding once plus h."""
+    import torch
+    import block_attention_b200 as ba
+    dev = torch.device("cuda", 0)
+    d, V = 4096, WORKLOAD["vocab"]
+    g = torch.Generator(device=dev).manual_seed(1006)
+    w = (torch.randn(V, d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    hbm, src = peaks()
+    out = {}
+    for rows in (32, 128):
+        h = torch.randn(rows, d, generator=g, device=dev).to(torch.bfloat16)
+        idx = torch.empty(rows, dtype=torch.int32, device=dev)
+        fused = lambda: ba.lm_head_argmax(h, w, idx=idx)
+        logits = torch.empty(rows, V, dtype=torch.bfloat16, device=dev)
+        unfused = lambda: (torch.matmul(h, w.t(), out=logits), ba.vocab_argmax(logits, idx=idx))
+        res = {}
+        for name, f in (("fused", fused), ("cublas_gemm_then_argmax", unfused)):
+            for _ in range(args.warmup):
+                f()
+            torch.cuda.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                for _ in range(args.steps):
+                    f()
+            gr.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) * 1e3 / args.steps
+            del gr
+        nbytes = V * d * 2 + rows * d * 2
+        out[f"rows_{rows}"] = {"us_fused": res["fused"],
+                               "us_unfused": res["cublas_gemm_then_argmax"],
+                               "bytes": nbytes, "gbs_fused": nbytes / res["fused"] / 1e3,
+                               "frac_fused": nbytes / res["fused"] / 1e3 / hbm}
+    print(json.dumps({"kernel": "lm_head_argmax", "case": f"d {d}, vocab {V}, bf16",
+                      "peak": hbm, "peak_source": src, **out}), flush=True)
+
+
 def block_size_sweep(args):
     """Block attention at the Qwen3-8B layer shape (B=1, ctx 8192) for block
     sizes K in {4, 8, 16, 32}, both views, 72 calls per CUDA graph chained as in
@@ -489,10 +537,11 @@ def main():
     ap.add_argument("--no-batched", action="store_true",
                     help="skip the batched ragged attention and stochastic consensus legs "
                          "(they run after the timing)")
-    ap.add_argument("--kernel", choices=["attn", "blk", "sample"], default=None,
+    ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
                          "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
-                         "the stochastic round's kernels one at a time")
+                         "the stochastic round's kernels one at a time; lmhead: the LM head "
+                         "with the argmax in its epilogue against GEMM + argmax")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel == "attn":
@@ -501,6 +550,8 @@ def main():
         return block_size_sweep(args)
     if args.kernel == "sample":
         return sampling_kernels(args)
+    if args.kernel == "lmhead":
+        return lm_head_kernel(args)
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -83,6 +83,7 @@ EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version",
            "orthrus_vocab_sample", "orthrus_vocab_sample_workspace", "orthrus_token_logprob", "orthrus_token_logprob_workspace",
            "orthrus_consensus_sample", "orthrus_consensus_sample_workspace",
+           "orthrus_lm_head_argmax", "orthrus_lm_head_argmax_workspace",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
            "orthrus_swiglu", "orthrus_block_tokens")
@@ -133,6 +134,10 @@ def lib() -> ctypes.CDLL:
         L.orthrus_vocab_sample.argtypes = [i32, vp, i32, i32, i64, c.c_float, c.c_uint64,
                                            c.c_uint32, vp, vp, vp, vp, sz, vp]
         L.orthrus_consensus_sample.argtypes = [c.POINTER(SampleArgs), vp]
+        L.orthrus_lm_head_argmax_workspace.argtypes = [i32]
+        L.orthrus_lm_head_argmax_workspace.restype = sz
+        L.orthrus_lm_head_argmax.argtypes = [i32, vp, i32, i32, i64, vp, i32, vp, vp, vp, vp,
+                                             sz, vp]
         _lib = L
     return _lib
 
@@ -433,3 +438,25 @@ def consensus_sample(draft, logits_ar, logits_diff, logq, lse_diff, temperature,
     _check("orthrus_consensus_sample", lib().orthrus_consensus_sample(ctypes.byref(a),
                                                                       _stream(stream)))
     return accept_len, n_emit, emitted, next_anchor
+
+
+def lm_head_argmax(h, w, *, idx=None, maxval=None, err=None, workspace=None, stream=None):
+    """int32 [rows]: argmax_v of h @ w.T per row (lowest index on ties), the
+    logits never materialised (see orthrus.h).  h bf16 [rows, d] (unit column
+    stride), w bf16 [vocab, d] contiguous; ``maxval`` float32 [rows] receives
+    the maximum logit when given."""
+    _dev(w, idx, maxval, err)  # h may be a row-strided view
+    if not h.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (no CPU path)")
+    if h.dim() != 2 or w.dim() != 2 or h.stride(1) != 1 or not w.is_contiguous():
+        raise ValueError("h must be 2-D with unit column stride, w 2-D contiguous")
+    rows, d = h.shape
+    if w.shape[1] != d:
+        raise ValueError("h and w disagree on the hidden size")
+    if idx is None:
+        idx = torch.empty(rows, dtype=torch.int32, device=h.device)
+    buf = _ws(workspace, h.device, "lm_head").get(lib().orthrus_lm_head_argmax_workspace(rows))
+    _check("orthrus_lm_head_argmax", lib().orthrus_lm_head_argmax(
+        _dtype(h), _ptr(h), rows, d, h.stride(0), _ptr(w), w.shape[0], _ptr(idx),
+        _ptr(maxval), _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
+    return idx

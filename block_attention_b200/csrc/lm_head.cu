@@ -1,0 +1,485 @@
+// lm_head.cu -- the LM head with the row argmax in its epilogue: for each
+// row r of the final hidden states h [R, d] (bf16),
+//   idx[r] = argmax_v sum_k h[r, k] w[v, k]      (lowest index on ties)
+// over the output embedding w [V, d] (bf16), without the R x V logits ever
+// leaving the SM.  Every Orthrus view ends in this product (cjcn.com.cn
+// explainer of "Orthrus", §二: the LM head is shared by both views) and the
+// round takes the argmax of its rows twice (§四: drafts from the diffusion
+// rows, the AR tokens from the verify rows).
+//
+// tcgen05 GEMM, D[hidden row, vocab row] = h w^T, one CTA per SM over a
+// contiguous range of vocabulary tiles of nv rows (nv chosen on the host so
+// the tiles spread evenly over the SMs; 208 at vocabulary 151936):
+//   warp 0     TMA producer: per stage the w slice (nv rows x 64, K-major,
+//              128-byte swizzle) -- the HBM stream -- and the matching 64
+//              columns of h (L2-resident) into a ring of stages
+//   warp 1     MMA issuer (one thread): per stage 4 MMAs of K = 16 with A =
+//              the stage's 64 columns of h from TMEM (128 lanes = hidden rows,
+//              zero past R) and B = the w slice from shared memory, N = nv,
+//              into one TMEM accumulator (kernel support for kk-interleaved
+//              chains is kept; the host uses one, leaving TMEM to the h ring)
+//   warps 2-5  per warp quadrant holding hidden rows: copy each stage's h
+//              slice from shared memory into a small TMEM ring ahead of the
+//              MMAs, then for each finished tile scan the thread's row of D
+//              (the chains added) for its best (value, index), kept across
+//              the CTA's tiles; a stage's slot is free once the MMAs and the
+//              copying warps are done with it
+// Operand A from TMEM leaves shared memory to the w stream: with A in shared
+// memory as well, the MMA issue rate, not HBM, bounded the kernel.
+// At the end each hidden row's CTA best goes to a 64-bit slot (value order,
+// lowest index) by atomicMax, and the last CTA (ticket) writes idx / maxval
+// and returns the workspace to zero.
+//
+// Every mbarrier wait is bounded: on a timeout the kernel records
+// ORTHRUS_ETIMEOUT in the error word, stops issuing work, drains what it
+// issued and still reaches the final ticket, so it always terminates.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <climits>
+#include <mutex>
+
+#include "common.cuh"
+#include "orthrus.h"
+#include "tc_ptx.cuh"
+
+namespace orthrus {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kRowsMax = 128;           // hidden rows per call (UMMA M, TMEM lanes)
+constexpr int kStepK = 64;              // d elements per stage (one 128-byte swizzle row)
+constexpr int kMaxStages = 12;
+constexpr int kRingBudget = 200 * 1024; // shared memory for the w ring
+constexpr int kTmemCols = 512;
+constexpr int kMaxASlots = 8;
+constexpr int kNumBars = 2 * kMaxStages + 2 * kMaxASlots + 3;
+
+struct __align__(64) LmParams {
+  CUtensorMap tm_w;                 // 2D (d, V), box (64, nv)
+  CUtensorMap tm_h;                 // 2D (d, R), row pitch ldh, box (64, 32 * writers)
+  unsigned long long* slots;        // [R] 64-bit (value, index) keys, zero between calls
+  unsigned* ticket;
+  int32_t* idx;
+  float* maxval;
+  int32_t* err;
+  int R, V, nv, nvp, ksteps, tiles, stages, stage_bytes, w_bytes, chains, aslots, a_col,
+      writers;
+};
+
+struct Layout {
+  int bars, misc, total;
+};
+__host__ __device__ inline Layout layout(int stages, int stage_bytes) {
+  Layout l;
+  l.bars = stages * stage_bytes;
+  l.misc = l.bars + kNumBars * 8;
+  l.total = l.misc + 16;
+  return l;
+}
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t at(int i) const { return base + 8 * i; }
+  __device__ uint32_t full(int s) const { return at(s); }
+  __device__ uint32_t empty(int s) const { return at(kMaxStages + s); }
+  __device__ uint32_t a_full(int j) const { return at(2 * kMaxStages + j); }
+  __device__ uint32_t a_empty(int j) const { return at(2 * kMaxStages + kMaxASlots + j); }
+  __device__ uint32_t acc_full() const { return at(2 * kMaxStages + 2 * kMaxASlots); }
+  __device__ uint32_t acc_empty() const { return at(2 * kMaxStages + 2 * kMaxASlots + 1); }
+  __device__ uint32_t mma_done() const { return at(2 * kMaxStages + 2 * kMaxASlots + 2); }
+};
+
+__device__ __forceinline__ void record_timeout(int32_t* err, volatile int* abort_flag) {
+  *abort_flag = 1;
+  set_err(err, ORTHRUS_ETIMEOUT);
+}
+
+// 64-bit key ordering (value, lowest index first); -0 == +0.
+__device__ __forceinline__ unsigned long long pack_key(float v, int i) {
+  if (v == 0.f) v = 0.f;
+  unsigned u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (unsigned)i);
+}
+__device__ __forceinline__ int key_index(unsigned long long k) {
+  return (int)(0xFFFFFFFFu - (unsigned)(k & 0xFFFFFFFFull));
+}
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  unsigned u = (unsigned)(k >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+  return __uint_as_float(u);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned full_mask = 0xffffffffu;
+  const int ST = p.stages, SB = p.stage_bytes, AS = p.aslots, C = p.chains;
+  const Layout L = layout(ST, SB);
+  const Bars bars{sbase + (uint32_t)L.bars};
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L.misc + 8);
+
+  const int t_beg = (int)((int64_t)blockIdx.x * p.tiles / gridDim.x);
+  const int t_end = (int)((int64_t)(blockIdx.x + 1) * p.tiles / gridDim.x);
+  const int ntiles = t_end - t_beg;
+  const int total = ntiles * p.ksteps;  // stages of this CTA
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    *last_flag = 0;
+    for (int s = 0; s < kMaxStages; ++s) {
+      ptx::mbar_init(bars.full(s), 1);
+      ptx::mbar_init(bars.empty(s), 1 + (uint32_t)p.writers);  // MMA commit + copying warps
+    }
+    for (int j = 0; j < kMaxASlots; ++j) {
+      ptx::mbar_init(bars.a_full(j), (uint32_t)p.writers);
+      ptx::mbar_init(bars.a_empty(j), 1);
+    }
+    ptx::mbar_init(bars.acc_full(), 1);
+    ptx::mbar_init(bars.acc_empty(), (uint32_t)p.writers);
+    ptx::mbar_init(bars.mma_done(), 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::tma_prefetch_desc(&p.tm_w);
+    ptx::tma_prefetch_desc(&p.tm_h);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int quad = warp & 3;  // TMEM lane quadrant of warps 2-5
+  const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+  if (warp >= 2) {  // the A ring starts zero on every lane (rows past R stay zero)
+    uint32_t z[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) z[j] = 0u;
+    for (int j = 0; j < AS; ++j) ptx::tmem_st32(lane_addr + (uint32_t)(p.a_col + 32 * j), z);
+    ptx::tmem_wait_st();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+
+  if (warp == 0) {
+    // ================================================== TMA producer
+    if (lane == 0) {
+      int it = 0;
+      for (; it < total; ++it) {
+        if (*abort_flag) break;
+        const int s = it % ST, t = t_beg + it / p.ksteps, k = it % p.ksteps;
+        if (!ptx::mbar_wait(bars.empty(s), ((it / ST) & 1) ^ 1)) {
+          record_timeout(p.err, abort_flag);
+          break;
+        }
+        const uint32_t dst = sbase + (uint32_t)(s * SB);
+        ptx::mbar_expect_tx(bars.full(s), (uint32_t)SB);
+        ptx::tma_load_2d(dst, &p.tm_w, bars.full(s), k * kStepK, t * p.nv);
+        ptx::tma_load_2d(dst + (uint32_t)p.w_bytes, &p.tm_h, bars.full(s), k * kStepK, 0);
+      }
+      // every issued load lands before the CTA can exit
+      for (int u = max(0, it - ST); u < it; ++u)
+        if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(p.err, abort_flag);
+    }
+  } else if (warp == 1) {
+    // ================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t id = ptx::idesc_bf16(kRowsMax, p.nv, false, false);
+      bool ok = true;
+      int it = 0;
+      for (int i = 0; ok && i < ntiles; ++i) {
+        if (i >= 1 && !ptx::mbar_wait(bars.acc_empty(), (i - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int k = 0; k < p.ksteps; ++k, ++it) {
+          const int s = it % ST, a = it % AS;
+          if (*abort_flag || !ptx::mbar_wait(bars.full(s), (it / ST) & 1) ||
+              !ptx::mbar_wait(bars.a_full(a), (it / AS) & 1)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t b0 = sbase + (uint32_t)(s * SB);
+          const uint32_t a0 = tmem + (uint32_t)(p.a_col + 32 * a);
+#pragma unroll
+          for (int kk = 0; kk < kStepK / 16; ++kk)
+            ptx::mma_ts(tmem + (uint32_t)((kk % C) * p.nvp), a0 + 8 * kk,
+                        ptx::sdesc_sw128(b0 + kk * 32, 16, 1024), id,
+                        (k > 0 || kk >= C) ? 1u : 0u);
+          ptx::tc_commit(bars.empty(s));
+          ptx::tc_commit(bars.a_empty(a));
+        }
+        if (!ok) break;
+        ptx::tc_commit(bars.acc_full());
+      }
+      if (!ok) record_timeout(p.err, abort_flag);
+      // every MMA issued has finished before TMEM is released
+      ptx::tc_commit(bars.mma_done());
+      if (!ptx::mbar_wait(bars.mma_done(), 0)) record_timeout(p.err, abort_flag);
+    }
+  } else if (quad < p.writers) {
+    // ================================================== h writer + epilogue
+    const int r = quad * 32 + lane;  // hidden row of this thread
+    const bool valid = r < p.R;
+    float best_v = -INFINITY;
+    int best_i = INT_MAX;
+    bool ok = true;
+    int it_w = 0;  // next h slice to copy (global stage index)
+    for (int i = 0; ok && i < ntiles; ++i) {
+      // this tile's slices, then the next tile's first ones: at most as many
+      // as both the slice ring and the stage ring hold, so that the TMEM slot
+      // and the stage of each are freed by MMAs of this tile, which do not
+      // wait on this tile's scan (one more would wait on an MMA of the next
+      // tile, which waits on that scan)
+      const int ahead = AS < ST ? AS : ST;
+      const int limit = min(min((i + 1) * p.ksteps + ahead, (i + 2) * p.ksteps), total);
+      for (; it_w < limit; ++it_w) {
+        const int a = it_w % AS, s = it_w % ST;
+        if (__any_sync(full_mask, *abort_flag != 0) ||
+            !__all_sync(full_mask, ptx::mbar_wait(bars.full(s), (it_w / ST) & 1)) ||
+            !__all_sync(full_mask, ptx::mbar_wait(bars.a_empty(a), ((it_w / AS) & 1) ^ 1))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        // row r of the slice: 128 bytes, 16-byte chunk j at (j ^ (r & 7)) (128-byte swizzle)
+        const uint8_t* hs = smem + s * SB + p.w_bytes + r * 128;
+        uint32_t x[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 q = *reinterpret_cast<const uint4*>(hs + ((j ^ (r & 7)) << 4));
+          x[4 * j] = q.x; x[4 * j + 1] = q.y; x[4 * j + 2] = q.z; x[4 * j + 3] = q.w;
+        }
+        ptx::tmem_st32(lane_addr + (uint32_t)(p.a_col + 32 * a), x);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(bars.a_full(a));
+          ptx::mbar_arrive(bars.empty(s));  // this warp is done with the stage's h rows
+        }
+      }
+      if (!ok) break;
+      // scan this thread's row of tile i
+      if (__any_sync(full_mask, *abort_flag != 0) ||
+          !__all_sync(full_mask, ptx::mbar_wait(bars.acc_full(), i & 1))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      const int v0 = (t_beg + i) * p.nv;
+      for (int cb = 0; cb < p.nv; cb += 32) {
+        float val[32];
+        if (p.nv - cb >= 32) {
+          for (int c = 0; c < C; ++c) {
+            uint32_t raw[32];
+            ptx::tmem_ld32_sync(lane_addr + (uint32_t)(c * p.nvp + cb), raw);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              val[j] = c ? val[j] + __uint_as_float(raw[j]) : __uint_as_float(raw[j]);
+          }
+        } else {  // the last 16 columns (nv is a multiple of 16)
+          for (int c = 0; c < C; ++c) {
+            uint32_t raw[16];
+            ptx::tmem_ld16_sync(lane_addr + (uint32_t)(c * p.nvp + cb), raw);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              val[j] = c ? val[j] + __uint_as_float(raw[j]) : __uint_as_float(raw[j]);
+          }
+#pragma unroll
+          for (int j = 16; j < 32; ++j) val[j] = -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {  // ascending index: strict > keeps the lowest
+          const int v = v0 + cb + j;
+          if (val[j] > best_v && v < p.V) {
+            best_v = val[j];
+            best_i = v;
+          } else if (best_i == INT_MAX && v < p.V && j < p.nv - cb) {
+            best_i = v;  // all values so far -inf or NaN: the lowest index stands in
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bars.acc_empty());
+    }
+    if (!ok) record_timeout(p.err, abort_flag);
+    if (valid && best_i != INT_MAX) atomicMax(&p.slots[r], pack_key(best_v, best_i));
+    __threadfence();
+  }
+
+  // ---- teardown and the last CTA's write-out
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *last_flag = atomicAdd(p.ticket, 1u) == gridDim.x - 1u;
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  for (int col = threadIdx.x; col < p.R; col += kThreads) {
+    const unsigned long long k = atomicExch(&p.slots[col], 0ull);
+    p.idx[col] = k ? key_index(k) : 0;
+    if (p.maxval) p.maxval[col] = k ? key_value(k) : __int_as_float(0x7fc00000);
+  }
+  if (threadIdx.x == 0) *p.ticket = 0u;
+}
+
+// ------------------------------------------------------------------ host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2D bf16 map (inner extent d, outer extent rows, row pitch in bytes), box
+// (64, box_rows), 128-byte swizzle; out-of-range rows read as zero.
+bool encode_2d(CUtensorMap* m, const void* base, int64_t d, int64_t rows, int64_t pitch_bytes,
+               int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)pitch_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)kStepK, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+bool prepare() {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64 && done[dev]) return true;
+  if (cudaFuncSetAttribute(lm_head_argmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           227 * 1024) != cudaSuccess)
+    return false;
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return true;
+}
+
+size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
+
+// Vocabulary rows per tile (a multiple of 16 in [128, 256], the UMMA N
+// range used): the one that minimises the rows of the busiest CTA, ties
+// going to the larger tile (fewer MMAs).
+int choose_nv(int vocab, int sms) {
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int nv = 256; nv >= 128; nv -= 16) {
+    const int tiles = ceil_div(vocab, nv);
+    const int grid = tiles < sms ? tiles : sms;
+    const int64_t cost = (int64_t)ceil_div(tiles, grid) * nv;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = nv;
+    }
+  }
+  return best;
+}
+
+}  // namespace
+}  // namespace orthrus
+
+using namespace orthrus;
+
+extern "C" {
+
+size_t orthrus_lm_head_argmax_workspace(int32_t rows) {
+  if (rows < 0) return 0;
+  return round256((int64_t)rows * 8) + 256;
+}
+
+int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d,
+                           int64_t h_row_stride, const void* w, int32_t vocab, int32_t* idx,
+                           float* maxval, int32_t* err, void* workspace, size_t workspace_bytes,
+                           orthrus_stream_t stream) {
+  if (dtype != ORTHRUS_F32 && dtype != ORTHRUS_BF16) return ORTHRUS_EINVAL;
+  if (rows < 0 || d <= 0 || vocab <= 0 || h_row_stride < d) return ORTHRUS_EINVAL;
+  if (dtype != ORTHRUS_BF16) return ORTHRUS_EUNSUPPORTED;
+  if (rows == 0) return ORTHRUS_OK;
+  if (rows > kRowsMax || d % kStepK != 0 || h_row_stride % 8 != 0 || vocab > (1 << 30))
+    return ORTHRUS_EUNSUPPORTED;
+  if (!h || !w || !idx) return ORTHRUS_EINVAL;
+  if (reinterpret_cast<uintptr_t>(h) % 16 || reinterpret_cast<uintptr_t>(w) % 16)
+    return ORTHRUS_EINVAL;
+  if (!workspace || workspace_bytes < orthrus_lm_head_argmax_workspace(rows) ||
+      reinterpret_cast<uintptr_t>(workspace) % 16)
+    return ORTHRUS_EWORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return ORTHRUS_ECUDA;
+
+  LmParams p;
+  p.R = rows;
+  p.V = vocab;
+  p.nv = choose_nv(vocab, sms);
+  p.nvp = (p.nv + 31) / 32 * 32;
+  p.ksteps = d / kStepK;
+  p.tiles = ceil_div(vocab, p.nv);
+  p.writers = ceil_div(rows, 32);
+  p.w_bytes = p.nv * 128;
+  p.stage_bytes = p.w_bytes + p.writers * 32 * 128;
+  p.stages = kRingBudget / p.stage_bytes < kMaxStages ? kRingBudget / p.stage_bytes : kMaxStages;
+  // TMEM: the accumulator, then the ring of h slices (32 columns each).  One
+  // chain: a deep slice ring (8 at nv = 208) lets the copying warps run ahead
+  // of the MMAs, which a second chain's columns would take away.
+  p.chains = 1;
+  p.a_col = p.chains * p.nvp;
+  p.aslots = (kTmemCols - p.a_col) / 32 < kMaxASlots ? (kTmemCols - p.a_col) / 32 : kMaxASlots;
+  char* ws = static_cast<char*>(workspace);
+  p.slots = reinterpret_cast<unsigned long long*>(ws);
+  p.ticket = reinterpret_cast<unsigned*>(ws + round256((int64_t)rows * 8));
+  p.idx = idx;
+  p.maxval = maxval;
+  p.err = err;
+  if (!encode_2d(&p.tm_w, w, d, vocab, (int64_t)d * 2, p.nv) ||
+      !encode_2d(&p.tm_h, h, d, rows, h_row_stride * 2, 32 * p.writers))
+    return ORTHRUS_ECUDA;
+  const int smem = layout(p.stages, p.stage_bytes).total + 1024;
+  if (!prepare()) return ORTHRUS_ECUDA;
+  const int grid = p.tiles < sms ? p.tiles : sms;
+  lm_head_argmax_kernel<<<grid, kThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
+}
+
+}  // extern "C"

@@ -68,6 +68,20 @@ def cast(x: np.ndarray, dtype: str) -> np.ndarray:
     raise ValueError(dtype)
 
 
+def lm_head_inputs(rows, d, V, seed=0, std_h=1.0, std_w=0.02, slice_rows=8192):
+    """Final hidden states h [rows, d] ~ N(0, std_h) and an output embedding
+    w [V, d] ~ N(0, std_w) (the usual init scale: logits of std
+    sqrt(d) std_h std_w), both as bf16 bit patterns; w is drawn in row slices
+    so a vocabulary-sized matrix needs no full-size float32 temporary."""
+    h = to_bf16(normal(rng(seed, S_W, 0), (rows, d), std_h))
+    w = np.empty((V, d), np.uint16)
+    g = rng(seed, S_W, 1)
+    for r0 in range(0, V, slice_rows):
+        r1 = min(V, r0 + slice_rows)
+        w[r0:r1] = to_bf16(normal(g, (r1 - r0, d), std_w))
+    return h, w
+
+
 def attn_inputs(B, Hq, Hkv, D, blk, ctx_lens, cap, dtype="f32", seed=0, layer=0,
                 std=1.0, with_cache=True):
     """Q/K/V for one layer of one round: all entries ~ N(0, std).

@@ -304,6 +304,33 @@ typedef struct orthrus_sample_args {
 size_t orthrus_consensus_sample_workspace(int32_t B, int32_t blk, int32_t vocab);
 int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * LM head with the argmax in its epilogue (the output projection every view
+ * ends in -- explainer §二: the LM head is shared -- followed by the row
+ * argmax that gives the drafts and the AR tokens, §四 steps 1-3):
+ *   idx[r]    = argmax_v sum_k h[r, k] w[v, k]   lowest index among equal maxima
+ *   maxval[r] = that maximum                     (nullable)
+ * h [rows, d] bf16, row r at h + r * h_row_stride (elements); w [vocab, d]
+ * bf16, dense (the PyTorch Linear layout of the LM head).  The logits never
+ * reach memory: a tcgen05 GEMM (all hidden rows x one vocabulary tile of
+ * 128-256 rows, fp32 accumulation in TMEM) reduces each tile to per-row bests
+ * in its epilogue.  The dot products are fp32 sums of exact bf16 products in the
+ * tensor core's order, so an argmax whose top two logits lie within fp32
+ * rounding may differ from an exact evaluation; the index returned is then
+ * one of the near-maxima.
+ * Limits: dtype ORTHRUS_BF16 (ORTHRUS_F32: ORTHRUS_EUNSUPPORTED); 1 <= rows
+ * <= 128 (0: no-op); d a multiple of 64; h_row_stride >= d and a multiple of
+ * 8; vocab <= 2^30; h and w 16-byte aligned.  err (nullable) receives
+ * ORTHRUS_ETIMEOUT if a bounded wait inside the kernel gave up.
+ * workspace: orthrus_lm_head_argmax_workspace(rows) bytes, 16-byte aligned,
+ * zeroed once; every call leaves it zero.  One launch, one CTA per SM.
+ * ---------------------------------------------------------------------- */
+size_t orthrus_lm_head_argmax_workspace(int32_t rows);
+int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d,
+                           int64_t h_row_stride, const void* w, int32_t vocab, int32_t* idx,
+                           float* maxval, int32_t* err, void* workspace,
+                           size_t workspace_bytes, orthrus_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 const char* orthrus_status_str(int status);
 int orthrus_version(void);

@@ -164,13 +164,13 @@ def lm_head_argmax(h, w, chunk=8192):
     rounding error of any lower-precision evaluation of the row.  The product
     is taken over vocabulary slices of `chunk` rows (a memory bound only: each
     logit is one complete dot product)."""
-    H, W = _widen64(h), _widen64(w)
-    rows, V = H.shape[0], W.shape[0]
+    H = _widen64(h)
+    rows, V = H.shape[0], np.shape(w)[0]
     logits = np.empty((rows, V))
     mag = np.zeros(rows)
     aH = np.abs(H)
     for c0 in range(0, V, chunk):
-        Wc = W[c0:c0 + chunk]
+        Wc = _widen64(w[c0:c0 + chunk])
         logits[:, c0:c0 + chunk] = H @ Wc.T
         mag = np.maximum(mag, (aH @ np.abs(Wc).T).max(axis=1))
     idx, mx = vocab_argmax(logits, return_max=True)

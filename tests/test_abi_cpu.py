@@ -220,3 +220,27 @@ def test_sampling_entry_points_host_checks(L):
     assert L.orthrus_consensus_sample_workspace(4, 8, 10) >= 4 * 24 + 32 * 4 + 32 * 8
     a.B = 0
     assert L.orthrus_consensus_sample(ctypes.byref(a), None) == 0
+
+
+def test_lm_head_argmax_host_checks(L):
+    c = ctypes
+    vp = c.c_void_p
+    ws = L.orthrus_lm_head_argmax_workspace(32)
+    assert ws >= 32 * 8 + 4
+    args = lambda dtype=1, h=256, rows=32, d=4096, ld=4096, w=512, V=151936, idx=1024, \
+        wsp=2048, wsb=ws: (dtype, vp(h) if h else None, rows, d, ld, vp(w) if w else None, V,
+                          vp(idx) if idx else None, None, None, vp(wsp) if wsp else None, wsb,
+                          None)
+    assert L.orthrus_lm_head_argmax(*args(dtype=7)) == -1          # unknown dtype
+    assert L.orthrus_lm_head_argmax(*args(dtype=0)) == -2          # fp32: not implemented
+    assert L.orthrus_lm_head_argmax(*args(rows=-1)) == -1
+    assert L.orthrus_lm_head_argmax(*args(ld=100, d=128)) == -1    # row stride < d
+    assert L.orthrus_lm_head_argmax(*args(rows=0, h=0, w=0, idx=0, wsp=0)) == 0
+    assert L.orthrus_lm_head_argmax(*args(rows=129)) == -2         # more rows than TMEM lanes
+    assert L.orthrus_lm_head_argmax(*args(d=4000, ld=4000)) == -2  # d not a multiple of 64
+    assert L.orthrus_lm_head_argmax(*args(ld=4100)) == -2          # pitch not 16-byte
+    assert L.orthrus_lm_head_argmax(*args(V=(1 << 30) + 1)) == -2
+    assert L.orthrus_lm_head_argmax(*args(h=0)) == -1
+    assert L.orthrus_lm_head_argmax(*args(w=520)) == -1            # w not 16-byte aligned
+    assert L.orthrus_lm_head_argmax(*args(wsb=ws - 1)) == -3
+    assert L.orthrus_lm_head_argmax(*args(wsp=2056)) == -3         # workspace alignment
