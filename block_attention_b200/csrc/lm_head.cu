@@ -10,9 +10,11 @@
 // tcgen05 GEMM, D[hidden row, vocab row] = h w^T, one CTA per SM over a
 // contiguous range of vocabulary tiles of nv rows (nv chosen on the host so
 // the tiles spread evenly over the SMs; 208 at vocabulary 151936):
-//   warp 0     TMA producer: per stage the w slice (nv rows x 64, K-major,
-//              128-byte swizzle) -- the HBM stream -- and the matching 64
-//              columns of h (L2-resident) into a ring of stages
+//   warp 0     TMA producer: per stage kb consecutive 64-column boxes of the
+//              w slice (nv rows each, K-major, 128-byte swizzle) -- the HBM
+//              stream -- and the matching columns of h (L2-resident) into a
+//              ring of stages; two boxes per stage halve the handshakes per
+//              byte
 //   warp 1     MMA issuer (one thread): per stage 4 MMAs of K = 16 with A =
 //              the stage's 64 columns of h from TMEM (128 lanes = hidden rows,
 //              zero past R) and B = the w slice from shared memory, N = nv,
@@ -65,7 +67,7 @@ struct __align__(64) LmParams {
   float* maxval;
   int32_t* err;
   int R, V, nv, nvp, ksteps, tiles, stages, stage_bytes, w_bytes, chains, aslots, a_col,
-      writers;
+      writers, kb, kst, hb;  // kb boxes per stage, kst stages per tile, hb bytes of one h box
 };
 
 struct Layout {
@@ -130,7 +132,8 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
   const int t_beg = (int)((int64_t)blockIdx.x * p.tiles / gridDim.x);
   const int t_end = (int)((int64_t)(blockIdx.x + 1) * p.tiles / gridDim.x);
   const int ntiles = t_end - t_beg;
-  const int total = ntiles * p.ksteps;  // stages of this CTA
+  const int total = ntiles * p.kst;  // stages of this CTA
+  const int KB = p.kb;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -179,15 +182,19 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
       int it = 0;
       for (; it < total; ++it) {
         if (*abort_flag) break;
-        const int s = it % ST, t = t_beg + it / p.ksteps, k = it % p.ksteps;
+        const int s = it % ST, t = t_beg + it / p.kst, k0 = (it % p.kst) * KB;
         if (!ptx::mbar_wait(bars.empty(s), ((it / ST) & 1) ^ 1)) {
           record_timeout(p.err, abort_flag);
           break;
         }
         const uint32_t dst = sbase + (uint32_t)(s * SB);
         ptx::mbar_expect_tx(bars.full(s), (uint32_t)SB);
-        ptx::tma_load_2d(dst, &p.tm_w, bars.full(s), k * kStepK, t * p.nv);
-        ptx::tma_load_2d(dst + (uint32_t)p.w_bytes, &p.tm_h, bars.full(s), k * kStepK, 0);
+        for (int j = 0; j < KB; ++j)
+          ptx::tma_load_2d(dst + (uint32_t)(j * p.nv * 128), &p.tm_w, bars.full(s),
+                           (k0 + j) * kStepK, t * p.nv);
+        for (int j = 0; j < KB; ++j)
+          ptx::tma_load_2d(dst + (uint32_t)(p.w_bytes + j * p.hb), &p.tm_h, bars.full(s),
+                           (k0 + j) * kStepK, 0);
       }
       // every issued load lands before the CTA can exit
       for (int u = max(0, it - ST); u < it; ++u)
@@ -205,7 +212,7 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
           break;
         }
         ptx::tc_fence_after();
-        for (int k = 0; k < p.ksteps; ++k, ++it) {
+        for (int k = 0; k < p.kst; ++k, ++it) {
           const int s = it % ST, a = it % AS;
           if (*abort_flag || !ptx::mbar_wait(bars.full(s), (it / ST) & 1) ||
               !ptx::mbar_wait(bars.a_full(a), (it / AS) & 1)) {
@@ -214,12 +221,16 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
           }
           ptx::tc_fence_after();
           const uint32_t b0 = sbase + (uint32_t)(s * SB);
-          const uint32_t a0 = tmem + (uint32_t)(p.a_col + 32 * a);
+          const uint32_t a0 = tmem + (uint32_t)(p.a_col + 32 * KB * a);
+          for (int j = 0; j < KB; ++j) {
 #pragma unroll
-          for (int kk = 0; kk < kStepK / 16; ++kk)
-            ptx::mma_ts(tmem + (uint32_t)((kk % C) * p.nvp), a0 + 8 * kk,
-                        ptx::sdesc_sw128(b0 + kk * 32, 16, 1024), id,
-                        (k > 0 || kk >= C) ? 1u : 0u);
+            for (int kk = 0; kk < kStepK / 16; ++kk) {
+              const int q = j * (kStepK / 16) + kk;
+              ptx::mma_ts(tmem + (uint32_t)((q % C) * p.nvp), a0 + 32 * j + 8 * kk,
+                          ptx::sdesc_sw128(b0 + j * p.nv * 128 + kk * 32, 16, 1024), id,
+                          (k > 0 || q >= C) ? 1u : 0u);
+            }
+          }
           ptx::tc_commit(bars.empty(s));
           ptx::tc_commit(bars.a_empty(a));
         }
@@ -246,7 +257,7 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
       // wait on this tile's scan (one more would wait on an MMA of the next
       // tile, which waits on that scan)
       const int ahead = AS < ST ? AS : ST;
-      const int limit = min(min((i + 1) * p.ksteps + ahead, (i + 2) * p.ksteps), total);
+      const int limit = min(min((i + 1) * p.kst + ahead, (i + 2) * p.kst), total);
       for (; it_w < limit; ++it_w) {
         const int a = it_w % AS, s = it_w % ST;
         if (__any_sync(full_mask, *abort_flag != 0) ||
@@ -256,15 +267,17 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
           break;
         }
         ptx::tc_fence_after();
-        // row r of the slice: 128 bytes, 16-byte chunk j at (j ^ (r & 7)) (128-byte swizzle)
-        const uint8_t* hs = smem + s * SB + p.w_bytes + r * 128;
-        uint32_t x[32];
+        for (int b = 0; b < KB; ++b) {
+          // row r of box b: 128 bytes, 16-byte chunk j at (j ^ (r & 7)) (128-byte swizzle)
+          const uint8_t* hs = smem + s * SB + p.w_bytes + b * p.hb + r * 128;
+          uint32_t x[32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 q = *reinterpret_cast<const uint4*>(hs + ((j ^ (r & 7)) << 4));
-          x[4 * j] = q.x; x[4 * j + 1] = q.y; x[4 * j + 2] = q.z; x[4 * j + 3] = q.w;
+          for (int j = 0; j < 8; ++j) {
+            const uint4 q = *reinterpret_cast<const uint4*>(hs + ((j ^ (r & 7)) << 4));
+            x[4 * j] = q.x; x[4 * j + 1] = q.y; x[4 * j + 2] = q.z; x[4 * j + 3] = q.w;
+          }
+          ptx::tmem_st32(lane_addr + (uint32_t)(p.a_col + 32 * (KB * a + b)), x);
         }
-        ptx::tmem_st32(lane_addr + (uint32_t)(p.a_col + 32 * a), x);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
@@ -457,15 +470,19 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
   p.ksteps = d / kStepK;
   p.tiles = ceil_div(vocab, p.nv);
   p.writers = ceil_div(rows, 32);
-  p.w_bytes = p.nv * 128;
-  p.stage_bytes = p.w_bytes + p.writers * 32 * 128;
+  p.kb = p.ksteps % 2 == 0 ? 2 : 1;
+  p.kst = p.ksteps / p.kb;
+  p.hb = p.writers * 32 * 128;
+  p.w_bytes = p.kb * p.nv * 128;
+  p.stage_bytes = p.w_bytes + p.kb * p.hb;
   p.stages = kRingBudget / p.stage_bytes < kMaxStages ? kRingBudget / p.stage_bytes : kMaxStages;
   // TMEM: the accumulator, then the ring of h slices (32 columns each).  One
   // chain: a deep slice ring (8 at nv = 208) lets the copying warps run ahead
   // of the MMAs, which a second chain's columns would take away.
   p.chains = 1;
   p.a_col = p.chains * p.nvp;
-  p.aslots = (kTmemCols - p.a_col) / 32 < kMaxASlots ? (kTmemCols - p.a_col) / 32 : kMaxASlots;
+  p.aslots = (kTmemCols - p.a_col) / (32 * p.kb) < kMaxASlots
+                 ? (kTmemCols - p.a_col) / (32 * p.kb) : kMaxASlots;
   char* ws = static_cast<char*>(workspace);
   p.slots = reinterpret_cast<unsigned long long*>(ws);
   p.ticket = reinterpret_cast<unsigned*>(ws + round256((int64_t)rows * 8));
