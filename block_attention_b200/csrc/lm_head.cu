@@ -13,8 +13,8 @@
 //   warp 0     TMA producer: per stage kb consecutive 64-column boxes of the
 //              w slice (nv rows each, K-major, 128-byte swizzle) -- the HBM
 //              stream -- and the matching columns of h (L2-resident) into a
-//              ring of stages; two boxes per stage halve the handshakes per
-//              byte
+//              ring of stages; more boxes per stage mean fewer handshakes per
+//              byte (4 where two such stages fit, else 2)
 //   warp 1     MMA issuer (one thread): per stage 4 MMAs of K = 16 with A =
 //              the stage's 64 columns of h from TMEM (128 lanes = hidden rows,
 //              zero past R) and B = the w slice from shared memory, N = nv,
@@ -53,7 +53,7 @@ constexpr int kThreads = 192;
 constexpr int kRowsMax = 128;           // hidden rows per call (UMMA M, TMEM lanes)
 constexpr int kStepK = 64;              // d elements per stage (one 128-byte swizzle row)
 constexpr int kMaxStages = 12;
-constexpr int kRingBudget = 200 * 1024; // shared memory for the w ring
+constexpr int kRingBudget = 212 * 1024; // shared memory for the stage ring
 constexpr int kTmemCols = 512;
 constexpr int kMaxASlots = 8;
 constexpr int kNumBars = 2 * kMaxStages + 2 * kMaxASlots + 3;
@@ -416,10 +416,10 @@ size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
 // Vocabulary rows per tile (a multiple of 16 in [128, 256], the UMMA N
 // range used): the one that minimises the rows of the busiest CTA, ties
 // going to the larger tile (fewer MMAs).
-int choose_nv(int vocab, int sms) {
-  int best = 256;
+int choose_nv(int vocab, int sms, int max_nv) {
+  int best = max_nv;
   int64_t best_cost = INT64_MAX;
-  for (int nv = 256; nv >= 128; nv -= 16) {
+  for (int nv = max_nv; nv >= 128; nv -= 16) {
     const int tiles = ceil_div(vocab, nv);
     const int grid = tiles < sms ? tiles : sms;
     const int64_t cost = (int64_t)ceil_div(tiles, grid) * nv;
@@ -465,14 +465,25 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
   LmParams p;
   p.R = rows;
   p.V = vocab;
-  p.nv = choose_nv(vocab, sms);
-  p.nvp = (p.nv + 31) / 32 * 32;
   p.ksteps = d / kStepK;
-  p.tiles = ceil_div(vocab, p.nv);
   p.writers = ceil_div(rows, 32);
-  p.kb = p.ksteps % 2 == 0 ? 2 : 1;
-  p.kst = p.ksteps / p.kb;
   p.hb = p.writers * 32 * 128;
+  // boxes per stage: 4 if two such stages fit (tiles of at most 176 rows),
+  // else 2, else 1
+  p.kb = 1;
+  p.nv = choose_nv(vocab, sms, 256);
+  for (int cand = 4; cand >= 2; cand /= 2) {
+    if (p.ksteps % cand) continue;
+    const int nv = choose_nv(vocab, sms, cand == 4 ? 176 : 256);
+    if (kRingBudget / (cand * (nv * 128 + p.hb)) >= 2) {
+      p.kb = cand;
+      p.nv = nv;
+      break;
+    }
+  }
+  p.nvp = (p.nv + 31) / 32 * 32;
+  p.tiles = ceil_div(vocab, p.nv);
+  p.kst = p.ksteps / p.kb;
   p.w_bytes = p.kb * p.nv * 128;
   p.stage_bytes = p.w_bytes + p.kb * p.hb;
   p.stages = kRingBudget / p.stage_bytes < kMaxStages ? kRingBudget / p.stage_bytes : kMaxStages;
