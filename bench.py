@@ -274,7 +274,7 @@ def sampling_kernels(args):
                       "us_per_launch": res}), flush=True)
 
 
-def lm_head_kernel(args):
+def lm_head_leg(dev, steps=10, warmup=3):
     """The Qwen3-8B LM head with the argmax fused in its epilogue (d 4096,
     vocabulary 151936, bf16) for 32 and 128 hidden rows (one and four
     32-row blocks), against the unfused pair a round would otherwise run: a
@@ -283,7 +283,6 @@ def lm_head_kernel(args):
     it from HBM.  Algorithmic bytes: the embedding once plus h."""
     import torch
     import block_attention_b200 as ba
-    dev = torch.device("cuda", 0)
     d, V = 4096, WORKLOAD["vocab"]
     g = torch.Generator(device=dev).manual_seed(1006)
     w = (torch.randn(V, d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
@@ -297,12 +296,12 @@ def lm_head_kernel(args):
         unfused = lambda: (torch.matmul(h, w.t(), out=logits), ba.vocab_argmax(logits, idx=idx))
         res = {}
         for name, f in (("fused", fused), ("cublas_gemm_then_argmax", unfused)):
-            for _ in range(args.warmup):
+            for _ in range(warmup):
                 f()
             torch.cuda.synchronize()
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr):
-                for _ in range(args.steps):
+                for _ in range(steps):
                     f()
             gr.replay()
             torch.cuda.synchronize()
@@ -311,15 +310,21 @@ def lm_head_kernel(args):
             gr.replay()
             e1.record()
             torch.cuda.synchronize()
-            res[name] = e0.elapsed_time(e1) * 1e3 / args.steps
+            res[name] = e0.elapsed_time(e1) * 1e3 / steps
             del gr
         nbytes = V * d * 2 + rows * d * 2
         out[f"rows_{rows}"] = {"us_fused": res["fused"],
                                "us_unfused": res["cublas_gemm_then_argmax"],
                                "bytes": nbytes, "gbs_fused": nbytes / res["fused"] / 1e3,
                                "frac_fused": nbytes / res["fused"] / 1e3 / hbm}
-    print(json.dumps({"kernel": "lm_head_argmax", "case": f"d {d}, vocab {V}, bf16",
-                      "peak": hbm, "peak_source": src, **out}), flush=True)
+    del w
+    return {"kernel": "lm_head_argmax", "case": f"d {d}, vocab {V}, bf16",
+            "peak": hbm, "peak_source": src, **out}
+
+
+def lm_head_kernel(args):
+    import torch
+    print(json.dumps(lm_head_leg(torch.device("cuda", 0), args.steps, args.warmup)), flush=True)
 
 
 def block_size_sweep(args):
@@ -535,8 +540,8 @@ def main():
     ap.add_argument("--no-e2e-decoder", action="store_true",
                     help="skip the end-to-end decoder report (runs after the timing)")
     ap.add_argument("--no-batched", action="store_true",
-                    help="skip the batched ragged attention and stochastic consensus legs "
-                         "(they run after the timing)")
+                    help="skip the batched ragged attention, stochastic consensus and LM-head "
+                         "legs (they run after the timing)")
     ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
                          "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
@@ -652,10 +657,11 @@ def main():
     dec = None
     if rank == 0 and world == 1 and not args.no_e2e_decoder:
         dec = decoder_report()
-    batched = stochastic = None
+    batched = stochastic = lm_head = None
     if rank == 0 and world == 1 and not args.no_batched:
         batched = batched_ragged_leg(dev, hbm)
         stochastic = stochastic_round_leg(dev, hbm)
+        lm_head = lm_head_leg(dev)
 
     if world > 1:
         dist.barrier()
@@ -686,6 +692,7 @@ def main():
         "e2e_decoder": dec,
         "block_attn_batched_ragged": batched,
         "stochastic_consensus": stochastic,
+        "lm_head_argmax": lm_head,
     }
     print(json.dumps(line), flush=True)
 
