@@ -18,12 +18,11 @@
 //   warp 1     MMA issuer (one thread): per stage 4 MMAs of K = 16 with A =
 //              the stage's 64 columns of h from TMEM (128 lanes = hidden rows,
 //              zero past R) and B = the w slice from shared memory, N = nv,
-//              into one TMEM accumulator (kernel support for kk-interleaved
-//              chains is kept; the host uses one, leaving TMEM to the h ring)
+//              into one TMEM accumulator (the rest of TMEM holds the h ring)
 //   warps 2-5  per warp quadrant holding hidden rows: copy each stage's h
 //              slice from shared memory into a small TMEM ring ahead of the
 //              MMAs, then for each finished tile scan the thread's row of D
-//              (the chains added) for its best (value, index), kept across
+//              for its best (value, index), kept across
 //              the CTA's tiles; a stage's slot is free once the MMAs and the
 //              copying warps are done with it
 // Operand A from TMEM leaves shared memory to the w stream: with A in shared
@@ -66,8 +65,8 @@ struct __align__(64) LmParams {
   int32_t* idx;
   float* maxval;
   int32_t* err;
-  int R, V, nv, nvp, ksteps, tiles, stages, stage_bytes, w_bytes, chains, aslots, a_col,
-      writers, kb, kst, hb;  // kb boxes per stage, kst stages per tile, hb bytes of one h box
+  int R, V, nv, nvp, ksteps, tiles, stages, stage_bytes, w_bytes, aslots, a_col, writers, kb,
+      kst, hb;  // kb boxes per stage, kst stages per tile, hb bytes of one h box
 };
 
 struct Layout {
@@ -122,7 +121,7 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
   const uint32_t sbase = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned full_mask = 0xffffffffu;
-  const int ST = p.stages, SB = p.stage_bytes, AS = p.aslots, C = p.chains;
+  const int ST = p.stages, SB = p.stage_bytes, AS = p.aslots;
   const Layout L = layout(ST, SB);
   const Bars bars{sbase + (uint32_t)L.bars};
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
@@ -225,10 +224,9 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
           for (int j = 0; j < KB; ++j) {
 #pragma unroll
             for (int kk = 0; kk < kStepK / 16; ++kk) {
-              const int q = j * (kStepK / 16) + kk;
-              ptx::mma_ts(tmem + (uint32_t)((q % C) * p.nvp), a0 + 32 * j + 8 * kk,
+              ptx::mma_ts(tmem, a0 + 32 * j + 8 * kk,
                           ptx::sdesc_sw128(b0 + j * p.nv * 128 + kk * 32, 16, 1024), id,
-                          (k > 0 || q >= C) ? 1u : 0u);
+                          (k > 0 || j > 0 || kk > 0) ? 1u : 0u);
             }
           }
           ptx::tc_commit(bars.empty(s));
@@ -298,21 +296,15 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
       for (int cb = 0; cb < p.nv; cb += 32) {
         float val[32];
         if (p.nv - cb >= 32) {
-          for (int c = 0; c < C; ++c) {
-            uint32_t raw[32];
-            ptx::tmem_ld32_sync(lane_addr + (uint32_t)(c * p.nvp + cb), raw);
+          uint32_t raw[32];
+          ptx::tmem_ld32_sync(lane_addr + (uint32_t)cb, raw);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              val[j] = c ? val[j] + __uint_as_float(raw[j]) : __uint_as_float(raw[j]);
-          }
+          for (int j = 0; j < 32; ++j) val[j] = __uint_as_float(raw[j]);
         } else {  // the last 16 columns (nv is a multiple of 16)
-          for (int c = 0; c < C; ++c) {
-            uint32_t raw[16];
-            ptx::tmem_ld16_sync(lane_addr + (uint32_t)(c * p.nvp + cb), raw);
+          uint32_t raw[16];
+          ptx::tmem_ld16_sync(lane_addr + (uint32_t)cb, raw);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              val[j] = c ? val[j] + __uint_as_float(raw[j]) : __uint_as_float(raw[j]);
-          }
+          for (int j = 0; j < 16; ++j) val[j] = __uint_as_float(raw[j]);
 #pragma unroll
           for (int j = 16; j < 32; ++j) val[j] = -INFINITY;
         }
@@ -487,11 +479,9 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
   p.w_bytes = p.kb * p.nv * 128;
   p.stage_bytes = p.w_bytes + p.kb * p.hb;
   p.stages = kRingBudget / p.stage_bytes < kMaxStages ? kRingBudget / p.stage_bytes : kMaxStages;
-  // TMEM: the accumulator, then the ring of h slices (32 columns each).  One
-  // chain: a deep slice ring (8 at nv = 208) lets the copying warps run ahead
-  // of the MMAs, which a second chain's columns would take away.
-  p.chains = 1;
-  p.a_col = p.chains * p.nvp;
+  // TMEM: the accumulator (nv columns, 32-aligned), then the ring of h slices
+  // (32 columns per box)
+  p.a_col = p.nvp;
   p.aslots = (kTmemCols - p.a_col) / (32 * p.kb) < kMaxASlots
                  ? (kTmemCols - p.a_col) / (32 * p.kb) : kMaxASlots;
   char* ws = static_cast<char*>(workspace);
