@@ -66,6 +66,26 @@ def config_dict():
             "l2": "inputs larger than L2: 1.21 GB KV cache, 2.46 GB of K/V streamed per round"}
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank device times (ms) over every rank of
+    the initialised process group (identity without one): a multi-GPU number
+    is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(world, steps, ms):
+    """Units per second completed by all ranks together: every rank runs
+    `steps` units of its own (weak scaling), in at most `ms` milliseconds."""
+    return world * steps / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -614,17 +634,14 @@ def main():
     step_ms = [e[0].elapsed_time(e[4]) for e in ev]
     attn_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev]
     total_ms = ev[0][0].elapsed_time(ev[-1][4])
-    t = torch.tensor([total_ms, sum(attn_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, attn_total_ms = float(t[0]), float(t[1])
+    total_ms, attn_total_ms = max_over_ranks([total_ms, sum(attn_ms)], dev)
 
     launches_attn = 2 * w["layers"] * args.steps
     attn_launch_us = attn_total_ms * 1e3 / launches_attn
     bytes_per_launch = rnd.attn_bytes_per_launch()
     hbm, src = peaks()
     achieved = bytes_per_launch / (attn_launch_us * 1e-6) / 1e9
-    rounds_per_s = world * args.steps / (total_ms * 1e-3)
+    rounds_per_s = whole_job_rate(world, args.steps, total_ms)
     gpu_launches = rnd.kernels_per_round() * args.steps
 
     # ---- end to end: per-round inputs from pinned host memory, results back
@@ -642,10 +659,8 @@ def main():
         bo = rnd.d2h(h_out)
     e1.record()
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_rounds = world * args.steps / (float(te[0]) * 1e-3)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
+    e2e_rounds = whole_job_rate(world, args.steps, e2e_ms)
     assert np.array_equal(h_out["n_emit"].numpy(), expect_ne)
 
     cpu = None
