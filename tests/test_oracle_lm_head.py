@@ -87,3 +87,22 @@ def test_gap_and_magnitude_bound_the_logits(oracle_mod):
     assert (np.abs(logits).max(axis=1) <= mag + 1e-12).all()
     srt = np.sort(logits, axis=1)
     np.testing.assert_allclose(gap, srt[:, -1] - srt[:, -2], rtol=0, atol=1e-12)
+
+
+def test_every_row_can_win_under_any_slicing(oracle_mod):
+    """The maximum planted at each vocabulary row in turn, for slice sizes that
+    put it first, last and inside a slice: the product over slices must not
+    drop or move any row."""
+    g = np.random.default_rng(26)
+    V, d = 23, 8
+    h = g.normal(0, 1, (1, d))
+    base = g.normal(0, 0.1, (V, d))
+    for v in range(V):
+        w = base.copy()
+        w[v] = 10 * h[0] / np.linalg.norm(h[0])
+        want = float(h[0] @ w[v])
+        for chunk in (1, 2, 5, 7, V, 64):
+            idx, mx, _, _ = oracle_mod.lm_head_argmax(h, w, chunk=chunk)
+            assert int(idx[0]) == v, (v, chunk)
+            # float64 summation order of the library product depends on the slice
+            assert abs(mx[0] - want) <= 1e-12 * abs(want), (v, chunk)
