@@ -9,22 +9,24 @@
 //
 // tcgen05 GEMM, D[hidden row, vocab row] = h w^T, one CTA per SM over a
 // contiguous range of vocabulary tiles of nv rows (nv chosen on the host so
-// the tiles spread evenly over the SMs; 208 at vocabulary 151936):
+// the tiles spread evenly over the SMs: at vocabulary 151936, 176 rows when
+// four boxes per stage fit, else 208):
 //   warp 0     TMA producer: per stage kb consecutive 64-column boxes of the
 //              w slice (nv rows each, K-major, 128-byte swizzle) -- the HBM
 //              stream -- and the matching columns of h (L2-resident) into a
 //              ring of stages; more boxes per stage mean fewer handshakes per
 //              byte (4 where two such stages fit, else 2)
-//   warp 1     MMA issuer (one thread): per stage 4 MMAs of K = 16 with A =
-//              the stage's 64 columns of h from TMEM (128 lanes = hidden rows,
-//              zero past R) and B = the w slice from shared memory, N = nv,
-//              into one TMEM accumulator (the rest of TMEM holds the h ring)
+//   warp 1     MMA issuer (one thread): per stage 4 kb MMAs of K = 16 with
+//              A = the stage's 64 kb columns of h from TMEM (128 lanes = hidden
+//              rows, zero past R) and B = the w slice from shared memory,
+//              N = nv, into one TMEM accumulator (the rest of TMEM holds the
+//              h ring)
 //   warps 2-5  per warp quadrant holding hidden rows: copy each stage's h
-//              slice from shared memory into a small TMEM ring ahead of the
+//              columns from shared memory into a small TMEM ring ahead of the
 //              MMAs, then for each finished tile scan the thread's row of D
-//              for its best (value, index), kept across
-//              the CTA's tiles; a stage's slot is free once the MMAs and the
-//              copying warps are done with it
+//              for its best (value, index), kept across the CTA's tiles; a
+//              stage's slot is free once the MMAs and the copying warps are
+//              done with it
 // Operand A from TMEM leaves shared memory to the w stream: with A in shared
 // memory as well, the MMA issue rate, not HBM, bounded the kernel.
 // At the end each hidden row's CTA best goes to a 64-bit slot (value order,
@@ -50,7 +52,7 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kRowsMax = 128;           // hidden rows per call (UMMA M, TMEM lanes)
-constexpr int kStepK = 64;              // d elements per stage (one 128-byte swizzle row)
+constexpr int kStepK = 64;              // d elements per box (one 128-byte swizzle row)
 constexpr int kMaxStages = 12;
 constexpr int kRingBudget = 212 * 1024; // shared memory for the stage ring
 constexpr int kTmemCols = 512;
