@@ -2,9 +2,12 @@
 // explainer of "Orthrus", §四: for sampling with a temperature the framework
 // aligns the two views' distributions by strict rejection sampling).
 // Declared in orthrus.h:
-//   orthrus_vocab_sample      draft tokens d_j ~ softmax(z_diff[j] / T) by Gumbel-max
-//   orthrus_token_logprob     log p(d_j), log q(d_j) and the rows' log-sum-exp at T
-//   orthrus_consensus_sample  accept while u_j < p/q, correction ~ normalize(max(0, p - q))
+//   orthrus_vocab_sample      draft tokens d_j ~ softmax(z_diff[j] / T) by Gumbel-max,
+//                             with log q(d_j) and the rows' log-sum-exp from the same pass
+//   orthrus_consensus_sample  log p(d_j), accept while u_j < p/q, then the correction
+//                             ~ normalize(max(0, p - q))
+//   orthrus_token_logprob     log-probability of given tokens at T (the precision
+//                             study; drafts that do not come from the sampler)
 // Random numbers: Philox4x32-10 (philox.cuh), counter layout in orthrus.h.
 #include "common.cuh"
 #include "philox.cuh"
@@ -118,9 +121,9 @@ __device__ __forceinline__ unsigned long long warp_max64(unsigned long long v) {
 // (value, index) pair replaced only by a strictly larger value (NaN never
 // wins; equal values keep the lower index) and forms the 64-bit order key
 // once.  The best (key, index) of the CTA goes to the row's slot by
-// atomicMax; with kLse
-// the CTA also stores its chunk pair.  The row's last CTA (ticket) writes
-// idx, lse and logprob and returns slot and ticket to zero.
+// atomicMax; with kLse the CTA also stores its chunk pair.  The row's last
+// CTA (ticket) writes idx, lse and logprob and returns slot and ticket to
+// zero.
 template <typename T, bool kLse>
 __global__ void __launch_bounds__(kThreads, 8)  // 8 CTAs (2048 threads) per SM
 vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, float inv_t,
@@ -239,9 +242,9 @@ token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
 // right, and writes every output except the correction.
 // Launch 2, grid (kResChunk-element chunks, B): one group of four per thread,
 // so the two rows' work spreads over about one wave; Gumbel-max over the
-// rejected row's residual
-// max(0, p - q) (the AR row's argmax as the fallback), folded per sequence
-// with atomicMax; the last CTA writes the correction.
+// rejected row's residual max(0, p - q) (the AR row's argmax as the
+// fallback), folded per sequence with atomicMax; the last CTA writes the
+// correction.
 // Workspace: SeqSlot [B], row tickets [B*blk], chunk pairs [B*blk][chunks].
 constexpr int kResChunk = kThreads * 4;
 
