@@ -69,8 +69,12 @@ int main(void) {
   printf("orthrus_sample_args size %zu\n", sizeof(orthrus_sample_args));
   F(orthrus_sample_args, row_stride); F(orthrus_sample_args, temperature);
   F(orthrus_sample_args, step); F(orthrus_sample_args, seed); F(orthrus_sample_args, draft);
-  F(orthrus_sample_args, logits_diff); F(orthrus_sample_args, next_anchor);
-  F(orthrus_sample_args, workspace_bytes);
+  F(orthrus_sample_args, logq); F(orthrus_sample_args, lse_diff);
+  F(orthrus_sample_args, logits_ar); F(orthrus_sample_args, logits_diff);
+  F(orthrus_sample_args, logp); F(orthrus_sample_args, lse_ar);
+  F(orthrus_sample_args, accept_len); F(orthrus_sample_args, n_emit);
+  F(orthrus_sample_args, emitted); F(orthrus_sample_args, next_anchor);
+  F(orthrus_sample_args, workspace); F(orthrus_sample_args, workspace_bytes);
   return 0;
 }''')
     exe = tmp_path / "layout"
@@ -85,6 +89,17 @@ int main(void) {
     for (t, m), v in got.items():
         c = cls[t]
         assert (ctypes.sizeof(c) if m == "size" else getattr(c, m).offset) == v, (t, m)
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c99"), ("g++", "-std=c++17")])
+def test_headers_compile_as_strict_c_and_cpp(tmp_path, compiler, std):
+    """Both public headers stand alone in C99 and C++17 (the ABI is plain C:
+    no C++ types leak into the declarations)."""
+    src = tmp_path / ("hdr.c" if compiler == "gcc" else "hdr.cpp")
+    src.write_text('#include "orthrus.h"\n#include "orthrus_decoder.h"\n'
+                   'int main(void) { return orthrus_version() > 0 ? 0 : 1; }\n')
+    subprocess.run([compiler, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                    "-I", os.path.join(ROOT, "include"), str(src)], check=True)
 
 
 def _args(**kw):
