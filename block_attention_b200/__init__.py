@@ -84,6 +84,7 @@ EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_vocab_sample", "orthrus_vocab_sample_workspace", "orthrus_token_logprob", "orthrus_token_logprob_workspace",
            "orthrus_consensus_sample", "orthrus_consensus_sample_workspace",
            "orthrus_lm_head_argmax", "orthrus_lm_head_argmax_workspace",
+           "orthrus_lm_head_argmax_plan",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
            "orthrus_swiglu", "orthrus_block_tokens")
@@ -134,6 +135,7 @@ def lib() -> ctypes.CDLL:
         L.orthrus_vocab_sample.argtypes = [i32, vp, i32, i32, i64, c.c_float, c.c_uint64,
                                            c.c_uint32, vp, vp, vp, vp, sz, vp]
         L.orthrus_consensus_sample.argtypes = [c.POINTER(SampleArgs), vp]
+        L.orthrus_lm_head_argmax_plan.argtypes = [i32, i32, i32, i32, vp]
         L.orthrus_lm_head_argmax_workspace.argtypes = [i32]
         L.orthrus_lm_head_argmax_workspace.restype = sz
         L.orthrus_lm_head_argmax.argtypes = [i32, vp, i32, i32, i64, vp, i32, vp, vp, vp, vp,

@@ -407,6 +407,7 @@ bool prepare() {
 
 size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
 
+
 // Vocabulary rows per tile (a multiple of 16 in [128, 256], the UMMA N
 // range used): the one that minimises the rows of the busiest CTA, ties
 // going to the larger tile (fewer MMAs).
@@ -425,38 +426,9 @@ int choose_nv(int vocab, int sms, int max_nv) {
   return best;
 }
 
-}  // namespace
-}  // namespace orthrus
-
-using namespace orthrus;
-
-extern "C" {
-
-size_t orthrus_lm_head_argmax_workspace(int32_t rows) {
-  if (rows < 0) return 0;
-  return round256((int64_t)rows * 8) + 256;
-}
-
-int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d,
-                           int64_t h_row_stride, const void* w, int32_t vocab, int32_t* idx,
-                           float* maxval, int32_t* err, void* workspace, size_t workspace_bytes,
-                           orthrus_stream_t stream) {
-  if (dtype != ORTHRUS_F32 && dtype != ORTHRUS_BF16) return ORTHRUS_EINVAL;
-  if (rows < 0 || d <= 0 || vocab <= 0 || h_row_stride < d) return ORTHRUS_EINVAL;
-  if (dtype != ORTHRUS_BF16) return ORTHRUS_EUNSUPPORTED;
-  if (rows == 0) return ORTHRUS_OK;
-  if (rows > kRowsMax || d % kStepK != 0 || h_row_stride % 8 != 0 || vocab > (1 << 30))
-    return ORTHRUS_EUNSUPPORTED;
-  if (!h || !w || !idx) return ORTHRUS_EINVAL;
-  if (reinterpret_cast<uintptr_t>(h) % 16 || reinterpret_cast<uintptr_t>(w) % 16)
-    return ORTHRUS_EINVAL;
-  if (!workspace || workspace_bytes < orthrus_lm_head_argmax_workspace(rows) ||
-      reinterpret_cast<uintptr_t>(workspace) % 16)
-    return ORTHRUS_EWORKSPACE;
-  const int sms = sm_count();
-  if (sms <= 0) return ORTHRUS_ECUDA;
-
-  LmParams p;
+// The launch's shape for rows x d x vocab on `sms` SMs (host only): tile rows,
+// boxes per stage, the stage ring, the TMEM slice ring.
+void plan(LmParams& p, int rows, int d, int vocab, int sms) {
   p.R = rows;
   p.V = vocab;
   p.ksteps = d / kStepK;
@@ -486,6 +458,59 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
   p.a_col = p.nvp;
   p.aslots = (kTmemCols - p.a_col) / (32 * p.kb) < kMaxASlots
                  ? (kTmemCols - p.a_col) / (32 * p.kb) : kMaxASlots;
+}
+
+}  // namespace
+}  // namespace orthrus
+
+using namespace orthrus;
+
+extern "C" {
+
+int orthrus_lm_head_argmax_plan(int32_t rows, int32_t d, int32_t vocab, int32_t sms,
+                                int32_t* out) {
+  if (!out || rows < 1 || rows > kRowsMax || d <= 0 || d % kStepK != 0 || vocab <= 0 ||
+      vocab > (1 << 30) || sms <= 0)
+    return ORTHRUS_EINVAL;
+  LmParams p;
+  plan(p, rows, d, vocab, sms);
+  out[0] = p.nv;
+  out[1] = p.kb;
+  out[2] = p.stages;
+  out[3] = p.aslots;
+  out[4] = layout(p.stages, p.stage_bytes).total + 1024;
+  out[5] = p.tiles < sms ? p.tiles : sms;
+  out[6] = p.tiles;
+  out[7] = kTmemCols;
+  return ORTHRUS_OK;
+}
+
+size_t orthrus_lm_head_argmax_workspace(int32_t rows) {
+  if (rows < 0) return 0;
+  return round256((int64_t)rows * 8) + 256;
+}
+
+int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d,
+                           int64_t h_row_stride, const void* w, int32_t vocab, int32_t* idx,
+                           float* maxval, int32_t* err, void* workspace, size_t workspace_bytes,
+                           orthrus_stream_t stream) {
+  if (dtype != ORTHRUS_F32 && dtype != ORTHRUS_BF16) return ORTHRUS_EINVAL;
+  if (rows < 0 || d <= 0 || vocab <= 0 || h_row_stride < d) return ORTHRUS_EINVAL;
+  if (dtype != ORTHRUS_BF16) return ORTHRUS_EUNSUPPORTED;
+  if (rows == 0) return ORTHRUS_OK;
+  if (rows > kRowsMax || d % kStepK != 0 || h_row_stride % 8 != 0 || vocab > (1 << 30))
+    return ORTHRUS_EUNSUPPORTED;
+  if (!h || !w || !idx) return ORTHRUS_EINVAL;
+  if (reinterpret_cast<uintptr_t>(h) % 16 || reinterpret_cast<uintptr_t>(w) % 16)
+    return ORTHRUS_EINVAL;
+  if (!workspace || workspace_bytes < orthrus_lm_head_argmax_workspace(rows) ||
+      reinterpret_cast<uintptr_t>(workspace) % 16)
+    return ORTHRUS_EWORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return ORTHRUS_ECUDA;
+
+  LmParams p;
+  plan(p, rows, d, vocab, sms);
   char* ws = static_cast<char*>(workspace);
   p.slots = reinterpret_cast<unsigned long long*>(ws);
   p.ticket = reinterpret_cast<unsigned*>(ws + round256((int64_t)rows * 8));

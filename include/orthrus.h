@@ -326,6 +326,13 @@ int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stre
  * zeroed once; every call leaves it zero.  One launch, one CTA per SM.
  * ---------------------------------------------------------------------- */
 size_t orthrus_lm_head_argmax_workspace(int32_t rows);
+/* The launch orthrus_lm_head_argmax would make for these sizes on a GPU with
+ * `sms` SMs (host only, no device needed): out[0..8) = vocabulary rows per
+ * tile, 64-column boxes per stage, stages, TMEM h slots, dynamic shared
+ * memory bytes, grid, tiles, TMEM columns.  ORTHRUS_EINVAL outside the
+ * limits above. */
+int orthrus_lm_head_argmax_plan(int32_t rows, int32_t d, int32_t vocab, int32_t sms,
+                                int32_t* out);
 int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d,
                            int64_t h_row_stride, const void* w, int32_t vocab, int32_t* idx,
                            float* maxval, int32_t* err, void* workspace,

@@ -259,3 +259,34 @@ def test_lm_head_argmax_host_checks(L):
     assert L.orthrus_lm_head_argmax(*args(w=520)) == -1            # w not 16-byte aligned
     assert L.orthrus_lm_head_argmax(*args(wsb=ws - 1)) == -3
     assert L.orthrus_lm_head_argmax(*args(wsp=2056)) == -3         # workspace alignment
+
+
+def test_lm_head_plan_respects_hardware_limits(L):
+    """The LM head's launch shape over a sweep of sizes and SM counts (host
+    only): tiles within the UMMA N range and the TMA box limit, the stage ring
+    and TMEM within the SM's 227 KB and 512 columns, at least one slot of look
+    ahead, every vocabulary row covered, the grid within the SMs."""
+    out = (ctypes.c_int32 * 8)()
+    for sms in (148, 132, 16, 1):
+        for rows in (1, 7, 32, 33, 64, 96, 128):
+            for d in (64, 128, 192, 256, 1024, 4096, 8192):
+                for V in (1, 100, 128, 3001, 32000, 151936, 262144, 1 << 20):
+                    assert L.orthrus_lm_head_argmax_plan(rows, d, V, sms, out) == 0
+                    nv, kb, stages, aslots, smem, grid, tiles, tmem = list(out)
+                    assert nv % 16 == 0 and 128 <= nv <= 256, (rows, d, V, nv)
+                    assert kb in (1, 2, 4) and (d // 64) % kb == 0
+                    assert stages >= 2 and aslots >= 1 and min(aslots, stages) >= 1
+                    assert smem <= 227 * 1024, (rows, d, V, smem)
+                    nvp = (nv + 31) // 32 * 32
+                    assert nvp + aslots * 32 * kb <= tmem == 512
+                    assert tiles * nv >= V > (tiles - 1) * nv
+                    assert 1 <= grid <= min(sms, tiles)
+    # the Qwen3-8B LM head as measured: 176-row tiles, four boxes per stage for
+    # one block; 208-row tiles, two boxes for four blocks
+    assert L.orthrus_lm_head_argmax_plan(32, 4096, 151936, 148, out) == 0
+    assert list(out)[:4] == [176, 4, 2, 2]
+    assert L.orthrus_lm_head_argmax_plan(128, 4096, 151936, 148, out) == 0
+    assert list(out)[:4] == [208, 2, 2, 4]
+    for bad in ((0, 4096, 100, 148), (129, 4096, 100, 148), (32, 100, 100, 148),
+                (32, 4096, 0, 148), (32, 4096, 100, 0)):
+        assert L.orthrus_lm_head_argmax_plan(*bad, out) == -1
