@@ -290,3 +290,23 @@ def test_lm_head_plan_respects_hardware_limits(L):
     for bad in ((0, 4096, 100, 148), (129, 4096, 100, 148), (32, 100, 100, 148),
                 (32, 4096, 0, 148), (32, 4096, 100, 0)):
         assert L.orthrus_lm_head_argmax_plan(*bad, out) == -1
+
+
+def test_tensor_core_split_count_stays_within_the_combine(L):
+    """Splits per (sequence, kv-head) read back from the bf16 tensor-core
+    path's workspace (B * Hkv * S partials of 128 * D / 2 + 256 words): at
+    least one, never more than the 24 the combine holds in registers or than
+    the tiles there are, and no split longer than 64 tiles unless capped."""
+    for D in (64, 128):
+        for Hq, Hkv, blk in ((32, 8, 32), (16, 8, 32), (8, 8, 16), (32, 8, 4), (64, 2, 2)):
+            for B in (1, 2, 8, 16, 64, 512):
+                for max_ctx in (0, 1, 100, 8192, 32768, 131072):
+                    a = _args(dtype=1, B=B, Hq=Hq, Hkv=Hkv, D=D, blk=blk, max_ctx=max_ctx,
+                              cap=max_ctx + blk, scale=D ** -0.5)
+                    ws = L.orthrus_block_attn_workspace(ctypes.byref(a))
+                    part = (128 * D // 2 + 256) * 4
+                    assert ws > 0 and ws % (B * Hkv * part) == 0, (D, Hq, Hkv, blk, B, max_ctx)
+                    S = ws // (B * Hkv * part)
+                    tiles = -(-max_ctx // 128) + 1
+                    assert 1 <= S <= min(24, tiles), (D, Hq, Hkv, blk, B, max_ctx, S)
+                    assert -(-tiles // S) <= 64 or S == 24
