@@ -11,9 +11,12 @@
 // which order CTAs finish.  Each CTA folds its key into the row's slot with
 // atomicMax; the last CTA of the row (ticket counter) decodes the key, writes
 // idx/maxval and returns the slot and the ticket to zero for the next call.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace orthrus {
 
@@ -45,6 +48,11 @@ argmax_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
               int nchunks, unsigned long long* keys, unsigned* tickets,
               int32_t* idx, float* maxval) {
   const int c = blockIdx.x, r = blockIdx.y;
+  // Launched with programmatic stream serialization: the launch overlaps the
+  // tail of the preceding kernel; nothing is read before that kernel has
+  // completed (it may be the one writing the logits).
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
   const T* row = logits + (int64_t)r * stride;
   const int beg = c * kArgmaxChunk;
   const int end = min(beg + kArgmaxChunk, vocab);
@@ -112,24 +120,30 @@ cudaError_t launch_argmax(int dtype, const void* logits, int rows, int vocab,
   unsigned long long* keys = static_cast<unsigned long long*>(ws);
   unsigned* tickets = reinterpret_cast<unsigned*>(keys + rows);
   const int nchunks = ceil_div(vocab, kArgmaxChunk);
-  dim3 grid(nchunks, rows);
   const size_t es = dtype == ORTHRUS_F32 ? 4 : 2;
   const bool vec = (reinterpret_cast<uintptr_t>(logits) % 16 == 0) &&
                    ((stride * (int64_t)es) % 16 == 0);
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nchunks, rows);
+  cfg.blockDim = dim3(kArgmaxThreads);
+  cfg.stream = st;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
   if (dtype == ORTHRUS_F32) {
     auto p = static_cast<const float*>(logits);
-    if (vec)
-      argmax_kernel<float, true><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
-    else
-      argmax_kernel<float, false><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
-  } else {
-    auto p = static_cast<const __nv_bfloat16*>(logits);
-    if (vec)
-      argmax_kernel<__nv_bfloat16, true><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
-    else
-      argmax_kernel<__nv_bfloat16, false><<<grid, kArgmaxThreads, 0, st>>>(p, vocab, stride, nchunks, keys, tickets, idx, maxval);
+    return vec ? cudaLaunchKernelEx(&cfg, argmax_kernel<float, true>, p, vocab, stride, nchunks,
+                                    keys, tickets, idx, maxval)
+               : cudaLaunchKernelEx(&cfg, argmax_kernel<float, false>, p, vocab, stride, nchunks,
+                                    keys, tickets, idx, maxval);
   }
-  return cudaGetLastError();
+  auto p = static_cast<const __nv_bfloat16*>(logits);
+  return vec ? cudaLaunchKernelEx(&cfg, argmax_kernel<__nv_bfloat16, true>, p, vocab, stride,
+                                  nchunks, keys, tickets, idx, maxval)
+             : cudaLaunchKernelEx(&cfg, argmax_kernel<__nv_bfloat16, false>, p, vocab, stride,
+                                  nchunks, keys, tickets, idx, maxval);
 }
 
 }  // namespace orthrus
@@ -152,10 +166,28 @@ constexpr size_t kNoAllocBytes = (size_t)kNoAllocMaxRows * 12;
 
 static __device__ __align__(256) unsigned char g_argmax_scratch[kNoAllocBytes];
 
-// Device address of g_argmax_scratch, looked up once per device (in host
-// code the symbol itself is only a host-side stand-in, never a device address).
+// Device address of g_argmax_scratch per device, together with the context it
+// was looked up in (in host code the symbol itself is only a host-side
+// stand-in, never a device address).  A device reset or a new primary context
+// reloads the module at another address, so the cached address is reused only
+// while the current context is the one it came from.
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[64] = {nullptr};
+CUcontext g_scratch_ctx[64] = {nullptr};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
 
 }  // namespace
 }  // namespace orthrus
@@ -175,12 +207,17 @@ extern "C" int orthrus_vocab_argmax_noalloc(int32_t dtype, const void* logits, i
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ORTHRUS_ECUDA;
   void* ws = nullptr;
   {
+    CtxGetCurrentFn get_ctx = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return ORTHRUS_ECUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
       void* ptr = nullptr;
       if (cudaGetSymbolAddress(&ptr, g_argmax_scratch) != cudaSuccess || !ptr)
         return ORTHRUS_ECUDA;
+      if (!ctx && (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)) return ORTHRUS_ECUDA;
       g_scratch_ptr[dev] = ptr;
+      g_scratch_ctx[dev] = ctx;
     }
     ws = g_scratch_ptr[dev];
   }

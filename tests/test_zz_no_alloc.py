@@ -60,6 +60,47 @@ def test_noalloc_argmax_matches_workspace_argmax_twice(dtype):
         assert torch.equal(max_a, max_b), call
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_noalloc_argmax_unaligned_row_stride(dtype):
+    """Rows that do not start on a 16-byte boundary take the kernel's scalar
+    path: vocab 100003 with a row stride of 100003 elements."""
+    fn = _noalloc()
+    rows, vocab = 24, 100003
+    x = synth.logits(synth.rng(410, len(dtype)), rows, vocab, dtype=dtype)
+    if dtype == "bf16":
+        t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    else:
+        t = torch.from_numpy(x).cuda()
+    assert t.stride(0) == vocab
+    for _ in range(2):
+        idx_a = torch.full((rows,), -7, dtype=torch.int32, device="cuda")
+        max_a = torch.empty(rows, dtype=torch.float32, device="cuda")
+        assert _call_noalloc(fn, t, idx_a, max_a) == 0
+        max_b = torch.empty(rows, dtype=torch.float32, device="cuda")
+        idx_b = ba.vocab_argmax(t, maxval=max_b)
+        torch.cuda.synchronize()
+        assert torch.equal(idx_a, idx_b)
+        assert torch.equal(max_a, max_b)
+
+
+def test_noalloc_argmax_allocates_no_device_memory():
+    """After a first call (which looks up the static array), further calls
+    leave the device's free memory unchanged."""
+    fn = _noalloc()
+    rows, vocab = 64, 151936
+    t = torch.from_numpy(synth.logits(synth.rng(420, 3), rows, vocab, dtype="f32")).cuda()
+    idx = torch.empty(rows, dtype=torch.int32, device="cuda")
+    mx = torch.empty(rows, dtype=torch.float32, device="cuda")
+    assert _call_noalloc(fn, t, idx, mx) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        assert _call_noalloc(fn, t, idx, mx) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
 def test_noalloc_argmax_refuses_rows_beyond_its_scratch():
     fn = _noalloc()
     t = torch.zeros(MAX_ROWS + 1, 16, device="cuda")
