@@ -47,7 +47,8 @@ class AttnArgs(ctypes.Structure):
                 ("v_blk", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
                 ("v_cache", ctypes.c_void_p), ("ctx_lens", ctypes.c_void_p),
                 ("out", ctypes.c_void_p), ("err", ctypes.c_void_p),
-                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("next_k_cache", ctypes.c_void_p), ("next_v_cache", ctypes.c_void_p)]
 
 
 class CommitArgs(ctypes.Structure):
@@ -78,7 +79,7 @@ class SampleArgs(ctypes.Structure):
 
 
 EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
-           "orthrus_block_attn_launches", "orthrus_vocab_argmax",
+           "orthrus_block_attn_launches", "orthrus_block_attn_plan", "orthrus_vocab_argmax",
            "orthrus_vocab_argmax_workspace", "orthrus_consensus", "orthrus_kv_commit",
            "orthrus_kv_commit_workspace", "orthrus_status_str", "orthrus_version",
            "orthrus_vocab_sample", "orthrus_vocab_sample_workspace", "orthrus_token_logprob", "orthrus_token_logprob_workspace",
@@ -107,6 +108,8 @@ def lib() -> ctypes.CDLL:
         L.orthrus_block_attn_workspace.restype = sz
         L.orthrus_block_attn_launches.argtypes = [c.POINTER(AttnArgs)]
         L.orthrus_block_attn_launches.restype = c.c_int
+        L.orthrus_block_attn_plan.argtypes = [c.POINTER(AttnArgs), i32, vp]
+        L.orthrus_block_attn_plan.restype = c.c_int
         L.orthrus_vocab_argmax.argtypes = [i32, vp, i32, i32, i64, vp, vp, vp, sz, vp]
         L.orthrus_vocab_argmax_workspace.argtypes = [i32]
         L.orthrus_vocab_argmax_workspace.restype = sz
@@ -207,16 +210,23 @@ ATTN_EARLY_KV = 1
 
 
 def attn_args(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, out=None,
-              scale=None, max_ctx=None, err=None, flags=0) -> AttnArgs:
+              scale=None, max_ctx=None, err=None, flags=0, next_kv=None) -> AttnArgs:
     B, blk, Hq, D = q.shape
     Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    nk = nv = None
+    if next_kv is not None:
+        nk, nv = next_kv
+        if nk.shape != k_cache.shape or nv.shape != v_cache.shape or nk.dtype != k_cache.dtype \
+                or nv.dtype != v_cache.dtype or not (nk.is_contiguous() and nv.is_contiguous()):
+            raise ValueError("next_kv must be two caches shaped like k_cache and v_cache")
+        nk, nv = nk.data_ptr(), nv.data_ptr()
     return AttnArgs(_dtype(q), int(mask_mode), B, Hq, Hkv, D, blk, cap,
                     cap if max_ctx is None else int(max_ctx),
                     float(D ** -0.5 if scale is None else scale), int(flags),
                     q.data_ptr(), k_blk.data_ptr(), v_blk.data_ptr(), k_cache.data_ptr(),
                     v_cache.data_ptr(), ctx_lens.data_ptr(),
                     out.data_ptr() if out is not None else None,
-                    err.data_ptr() if err is not None else None, None, 0)
+                    err.data_ptr() if err is not None else None, None, 0, nk, nv)
 
 
 def block_attn_workspace_bytes(args: AttnArgs) -> int:
@@ -224,19 +234,22 @@ def block_attn_workspace_bytes(args: AttnArgs) -> int:
 
 
 def block_attn(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, *, out=None,
-               scale=None, max_ctx=None, err=None, workspace=None, stream=None, flags=0):
+               scale=None, max_ctx=None, err=None, workspace=None, stream=None, flags=0,
+               next_kv=None):
     """Attention of one layer for one round (see orthrus.h for the definition).
 
     q [B, blk, Hq, D]; k_blk/v_blk [B, blk, Hkv, D]; k_cache/v_cache
     [B, Hkv, cap, D]; ctx_lens int32 [B] on the device.  max_ctx bounds every
-    ctx_lens entry (default: cap).  Returns out [B, blk, Hq, D] (q's dtype)."""
+    ctx_lens entry (default: cap).  next_kv = (k_cache, v_cache) of the call
+    that follows on the stream: warmed into L2 while this one runs (a hint;
+    results unchanged).  Returns out [B, blk, Hq, D] (q's dtype)."""
     _dev(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, out, err)
     if ctx_lens.dtype != torch.int32:
         raise TypeError("ctx_lens must be int32")
     if out is None:
         out = torch.empty_like(q)
     a = attn_args(q, k_blk, v_blk, k_cache, v_cache, ctx_lens, mask_mode, out, scale,
-                  max_ctx, err, flags)
+                  max_ctx, err, flags, next_kv)
     need = block_attn_workspace_bytes(a)
     if need:
         # scratch for the split partials; one default buffer per device

@@ -168,11 +168,16 @@ __global__ void __launch_bounds__(D) attn_simt_combine_kernel(const SimtParams p
   static_cast<T*>(p.out)[(int64_t)row * D + d] = from_f32<T>(O / L);
 }
 
+// The first kSimtSkipBytes bytes of the caller's buffer are left alone: the
+// tensor-core path keeps its merge counters there, and one buffer may serve
+// both paths.
+constexpr int64_t kSimtSkipBytes = 2048;
+
 size_t simt_workspace_bytes(int B, int Hq, int D, int blk, int max_ctx) {
   const int64_t nsplit = ceil_div(max_ctx + blk, kSimtChunk);
   const int64_t parts = (int64_t)B * Hq * blk * nsplit;
   auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
-  return (size_t)(up(parts * D * 4) + 2 * up(parts * 4));
+  return (size_t)(kSimtSkipBytes + up(parts * D * 4) + 2 * up(parts * 4));
 }
 
 template <typename T, int D>
@@ -196,7 +201,7 @@ cudaError_t launch_attn_simt(const orthrus_attn_args& a, cudaStream_t st) {
   p.nsplit = ceil_div(a.max_ctx + a.blk, kSimtChunk);
   const int64_t parts = (int64_t)a.B * a.Hq * a.blk * p.nsplit;
   auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
-  char* ws = static_cast<char*>(a.workspace);
+  char* ws = static_cast<char*>(a.workspace) + kSimtSkipBytes;
   p.ws_o = reinterpret_cast<float*>(ws);
   p.ws_m = reinterpret_cast<float*>(ws + up(parts * a.D * 4));
   p.ws_l = reinterpret_cast<float*>(ws + up(parts * a.D * 4) + up(parts * 4));

@@ -82,6 +82,9 @@ int orthrus_block_attn(const orthrus_attn_args* a, orthrus_stream_t stream) {
   for (const void* p : ptrs)
     if (!p || !aligned(p, vec)) return ORTHRUS_EINVAL;
   if (!a->ctx_lens) return ORTHRUS_EINVAL;
+  if ((a->next_k_cache && !aligned(a->next_k_cache, vec)) ||
+      (a->next_v_cache && !aligned(a->next_v_cache, vec)))
+    return ORTHRUS_EINVAL;
   const size_t need = orthrus_block_attn_workspace(a);
   if (need > 0 && (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256)))
     return ORTHRUS_EWORKSPACE;
@@ -93,6 +96,24 @@ int orthrus_block_attn(const orthrus_attn_args* a, orthrus_stream_t stream) {
 int orthrus_block_attn_launches(const orthrus_attn_args* a) {
   if (check_attn_shape(a) != ORTHRUS_OK || a->B == 0) return 0;
   return use_tc_path(a) ? tc_launches(*a) : 2;  // split + combine
+}
+
+int orthrus_block_attn_plan(const orthrus_attn_args* a, int32_t sms, int32_t* out) {
+  if (!out || sms < 1) return ORTHRUS_EINVAL;
+  const int rc = check_attn_shape(a);
+  if (rc != ORTHRUS_OK) return rc;
+  if (!use_tc_path(a)) return ORTHRUS_EUNSUPPORTED;
+  const int S = tc_plan_splits(*a, sms);
+  const int tiles = (a->max_ctx + 127) / 128 + 1;  // 128-key cache tiles + the block tile
+  out[0] = S;
+  out[1] = S;
+  out[2] = a->Hkv;
+  out[3] = a->B;
+  out[4] = tc_threads();
+  out[5] = tc_smem_bytes();
+  out[6] = (tiles + S - 1) / S;
+  out[7] = tc_plan_fused(*a, sms, S) ? 1 : 0;
+  return ORTHRUS_OK;
 }
 
 size_t orthrus_vocab_argmax_workspace(int32_t rows) {

@@ -25,12 +25,12 @@
  *     device can see (a device-resident length out of range) set the optional
  *     device error word `err` (first error code wins) and skip the affected
  *     sequence's writes; kernels never trap.
- *   - Workspaces: query the size and allocate it once.  Argmax and commit
- *     workspaces hold ticket counters: zero them once (cudaMemset 0); the
- *     kernels leave the counters at zero again, so the buffer serves every
- *     later call on the same stream (zero it again after a call that reported
- *     an error).  The block-attention workspace is scratch only.  Calls that
- *     may run at the same time (different streams) need separate workspaces.
+ *   - Workspaces: query the size and allocate it once.  Workspaces hold
+ *     ticket or arrival counters: zero them once (cudaMemset 0); the kernels
+ *     leave the counters at zero again, so the buffer serves every later call
+ *     on the same stream (zero it again after a call that reported an
+ *     error).  Calls that may run at the same time (different streams) need
+ *     separate workspaces.
  *   - Tensors are dense, row-major, with the layouts written next to each
  *     field.  dtype applies to every floating-point tensor of a call.
  */
@@ -116,15 +116,32 @@ typedef struct orthrus_attn_args {
   void* out;           /* [B, blk, Hq, D], same dtype as q */
   int32_t* err;        /* optional device int32 error word (NULL = none) */
   void* workspace;     /* >= orthrus_block_attn_workspace() bytes, 256-byte aligned,
-                          scratch (see below) */
+                          zeroed once (see below) */
   size_t workspace_bytes; /* size of the caller's buffer */
+  /* Optional L2 warm-up for the call that follows this one on the stream
+   * (the next layer of the same view, say): its K and V caches, with this
+   * call's B, Hkv, cap, D and lengths.  NULL = none.  The BF16 tensor-core
+   * path then prefetches, while it runs, the rows [0, ctx_lens[b]) of those
+   * caches into L2 (each CTA its own tiles' rows, after issuing its last load
+   * of this call's cache), so HBM keeps streaming across the boundary between
+   * the two calls.  A hint only: the results of both calls are unchanged, and
+   * the FP32 path ignores it.  16-byte aligned. */
+  const void* next_k_cache;
+  const void* next_v_cache;
 } orthrus_attn_args;
 
-/* Workspace of orthrus_block_attn: scratch for the per-split partial results
- * of the split-KV reduction (unnormalised O plus row max and row sum), written
- * and read back within the call; it needs no initialisation and carries
- * nothing from one call to the next.  One buffer may serve any sequence of
- * FP32 and BF16 calls on one stream whose sizes fit it. */
+/* Workspace of orthrus_block_attn: the per-split partial results of the
+ * split-KV reduction (unnormalised O plus row max and row sum), written and
+ * read back within the call.  The BF16 tensor-core path also keeps, in the
+ * buffer's first 2048 bytes, the counters of its in-launch merge:
+ * zero the buffer once (cudaMemset 0); every call leaves the counters at
+ * zero, so one buffer serves any later FP32 and BF16 calls on one stream
+ * whose sizes fit it (zero it again after a call that reported an error).
+ * A BF16 call whose grid fits one wave (see orthrus_block_attn_plan) counts
+ * on all of its CTAs being resident together: do not run it concurrently
+ * with kernels (other streams) that could hold SMs until it ends -- the
+ * merge's wait would give up after about a second and report
+ * ORTHRUS_ETIMEOUT. */
 
 /* Bytes of workspace orthrus_block_attn needs for these arguments (0 if none).
  * Pointers in `a` are not read.  Returns 0 for invalid shapes as well. */
@@ -135,6 +152,18 @@ int orthrus_block_attn(const orthrus_attn_args* a, orthrus_stream_t stream);
 /* Number of kernel launches one orthrus_block_attn call with these arguments
  * issues (for launch accounting); 0 for invalid shapes or B == 0. */
 int orthrus_block_attn_launches(const orthrus_attn_args* a);
+
+/* Launch plan of the BF16 tensor-core path for a GPU with `sms` SMs (host
+ * only; pointers in `a` are not read).  The keys of each (sequence, kv-head)
+ * -- cache[0, max_ctx) in 128-key tiles, then one tile of block rows -- are
+ * dealt over S splits, one CTA each; the splits' partial results are merged
+ * in split order.  out[0..8) = S, grid x, y, z (S, Hkv, B), threads per CTA,
+ * dynamic shared memory bytes, most tiles one split streams, and 1 if the
+ * merge runs inside the one launch (the grid fits one wave of one CTA per SM:
+ * B * Hkv * S <= sms and B * Hkv <= 256) or 0 if a second, PDL-chained
+ * kernel merges.  ORTHRUS_EUNSUPPORTED when the call would take the FP32
+ * path. */
+int orthrus_block_attn_plan(const orthrus_attn_args* a, int32_t sms, int32_t* out);
 
 /* ------------------------------------------------------------------------
  * Vocab-row argmax (explainer §四: "the token that should most appear here").
@@ -163,6 +192,9 @@ int orthrus_vocab_argmax(int32_t dtype, const void* logits, int32_t rows,
  *     uses with cudaMemsetAsync on `stream`, then launches the argmax kernel.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is kept with the context it came from and looked up again
+ *     when the current context differs (after a device reset, for example);
+ *     that later lookup is again a call to make outside stream capture.
  *   - Every call shares the one array: calls that overlap on the GPU (other
  *     streams, other threads) race and give wrong indices; serialise them. */
 #define ORTHRUS_NOALLOC_ARGMAX_MAX_ROWS 4096

@@ -62,6 +62,7 @@ int main(void) {
   F(orthrus_attn_args, scale); F(orthrus_attn_args, flags); F(orthrus_attn_args, q);
   F(orthrus_attn_args, ctx_lens);
   F(orthrus_attn_args, err); F(orthrus_attn_args, workspace_bytes);
+  F(orthrus_attn_args, next_k_cache); F(orthrus_attn_args, next_v_cache);
   printf("orthrus_commit_args size %zu\n", sizeof(orthrus_commit_args));
   F(orthrus_commit_args, k_cache); F(orthrus_commit_args, cache_layer_stride);
   F(orthrus_commit_args, blk_layer_stride); F(orthrus_commit_args, n_emit);
@@ -292,11 +293,16 @@ def test_lm_head_plan_respects_hardware_limits(L):
         assert L.orthrus_lm_head_argmax_plan(*bad, out) == -1
 
 
-def test_tensor_core_split_count_stays_within_the_combine(L):
-    """Splits per (sequence, kv-head) read back from the bf16 tensor-core
-    path's workspace (B * Hkv * S partials of 128 * D / 2 + 256 words): at
-    least one, never more than the 24 the combine holds in registers or than
-    the tiles there are, and no split longer than 64 tiles unless capped."""
+def test_tensor_core_attention_plan(L):
+    """Launch plan of the bf16 tensor-core path over a sweep of shapes and SM
+    counts: S splits per (sequence, kv-head) with 1 <= S <= min(24, tiles)
+    (24: the merge keeps every split's loads in registers), one wave of CTAs
+    when the batch is small, no split longer than 64 tiles unless S is
+    capped, the shared memory within the 227 KB a CTA may use, the merge
+    inside the launch exactly when the grid fits one wave, and a workspace
+    that holds the 2048-byte counter head plus every split's fp32 partial for
+    any GPU of up to 256 SMs."""
+    out = (ctypes.c_int32 * 8)()
     for D in (64, 128):
         for Hq, Hkv, blk in ((32, 8, 32), (16, 8, 32), (8, 8, 16), (32, 8, 4), (64, 2, 2)):
             for B in (1, 2, 8, 16, 64, 512):
@@ -304,9 +310,33 @@ def test_tensor_core_split_count_stays_within_the_combine(L):
                     a = _args(dtype=1, B=B, Hq=Hq, Hkv=Hkv, D=D, blk=blk, max_ctx=max_ctx,
                               cap=max_ctx + blk, scale=D ** -0.5)
                     ws = L.orthrus_block_attn_workspace(ctypes.byref(a))
-                    part = (128 * D // 2 + 256) * 4
-                    assert ws > 0 and ws % (B * Hkv * part) == 0, (D, Hq, Hkv, blk, B, max_ctx)
-                    S = ws // (B * Hkv * part)
-                    tiles = -(-max_ctx // 128) + 1
-                    assert 1 <= S <= min(24, tiles), (D, Hq, Hkv, blk, B, max_ctx, S)
-                    assert -(-tiles // S) <= 64 or S == 24
+                    assert L.orthrus_block_attn_plan(ctypes.byref(a), 256, out) == 0
+                    part = (128 + 24) * (D // 2 + 4) * 4  # bf16 O + fp32 (max, sum) per row
+                    assert ws == 2048 + B * Hkv * out[0] * part, (D, Hq, Hkv, blk, B, max_ctx)
+                    assert L.orthrus_block_attn_launches(ctypes.byref(a)) in (1, 2)
+                    for sms in (132, 148, 160, 256):
+                        key = (D, Hq, Hkv, blk, B, max_ctx, sms)
+                        assert L.orthrus_block_attn_plan(ctypes.byref(a), sms, out) == 0, key
+                        S, gx, gy, gz, thr, smem, most, fused = list(out)
+                        tiles = -(-max_ctx // 128) + 1
+                        heads = B * Hkv
+                        assert 1 <= S <= min(24, tiles), key
+                        assert 2048 + heads * S * part <= ws, key  # fits the sized buffer
+                        assert (gx, gy, gz) == (S, Hkv, B), key
+                        assert most == -(-tiles // S), key
+                        assert most <= 64 or S == 24, key
+                        if heads < sms:  # a small batch fills the SMs as far as it can
+                            assert S >= min(24, tiles, sms // heads), key
+                        # more CTAs than SMs only where long sequences need the splits
+                        assert heads * S <= sms or S == min(24, tiles, -(-tiles // 64)), key
+                        assert fused == int(heads * S <= sms and heads <= 256), key
+                        assert thr % 32 == 0 and 0 < smem <= 227 * 1024, key
+    # the fp32 path has no such plan
+    a = _args(dtype=0, B=1, Hq=32, Hkv=8, D=128, blk=32, max_ctx=64, cap=96, scale=0.1)
+    assert L.orthrus_block_attn_plan(ctypes.byref(a), 148, out) == -2
+    a = _args(dtype=1, B=1, Hq=32, Hkv=8, D=128, blk=32, max_ctx=8192, cap=8224, scale=0.1)
+    assert L.orthrus_block_attn_plan(ctypes.byref(a), 0, out) == -1
+    # the Qwen3-8B round shape on 148 SMs: 18 splits per kv-head, 144 CTAs,
+    # at most 4 of the 65 tiles each, merged inside the launch
+    assert L.orthrus_block_attn_plan(ctypes.byref(a), 148, out) == 0
+    assert list(out)[:4] == [18, 18, 8, 1] and out[6] == 4 and out[7] == 1

@@ -141,8 +141,10 @@ def test_device_length_over_bound_sets_error_word(oracle_mod, dtype):
 
 
 def test_one_workspace_reused_across_shapes(oracle_mod):
-    """One bf16 workspace serves calls of different shapes in any order: its
-    ticket counters (kept at the end of the buffer) stay valid."""
+    """One bf16 workspace serves calls of different shapes in any order: the
+    merge's arrival counts (the buffer's first 1024 bytes; the generations
+    follow, and no partial is ever written there) are back at zero after
+    every call."""
     ws = ba.Workspace("cuda")
     shapes = [(2, 32, 8, 128, 32, [3000, 500]), (1, 4, 1, 64, 32, [100]),
               (1, 16, 8, 128, 32, [2048]), (1, 8, 8, 128, 4, [0]),
@@ -158,6 +160,7 @@ def test_one_workspace_reused_across_shapes(oracle_mod):
                                         inp["v_cache"], inp["ctx_lens"], mode)
             e = rel_err_rows(to_host(out), ref)
             assert e.max() <= TOL["bf16"], (k, mode, e.max())
+            assert int(ws.buf[:1024].count_nonzero()) == 0, (k, mode)
 
 
 @pytest.mark.parametrize("mode", [0, 1])
@@ -181,3 +184,24 @@ def test_block_size_variants(oracle_mod, dtype, mode, blk):
     Qwen3-8B head layout, with a ragged pair of contexts."""
     inp = synth.attn_inputs(2, 32, 8, 128, blk, [2000, 333], 2000 + blk, dtype, seed=150 + blk)
     check(inp, mode, dtype, oracle_mod=oracle_mod)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_next_call_l2_prefetch_same_result(oracle_mod, mode):
+    """Naming the next call's caches (an L2 warm-up hint) leaves the output
+    bit-identical, for a one-wave grid (merge inside the launch) and a larger
+    one (separate merge kernel)."""
+    for B, lens in ((1, [8192]), (8, [3000, 500, 8000, 1, 0, 4096, 2048, 7777])):
+        inp = synth.attn_inputs(B, 32, 8, 128, 32, lens, max(lens) + 32, "bf16", seed=160 + B)
+        t = {k: to_dev(v) for k, v in inp.items()}
+        nk, nv = torch.randn_like(t["k_cache"]), torch.randn_like(t["v_cache"])
+        a = ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                          t["ctx_lens"], mode)
+        b = ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                          t["ctx_lens"], mode, next_kv=(nk, nv), flags=ba.ATTN_EARLY_KV)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b), B
+        if B == 1:
+            ref = oracle_mod.block_attn(inp["q"], inp["k_blk"], inp["v_blk"], inp["k_cache"],
+                                        inp["v_cache"], inp["ctx_lens"], mode)
+            assert rel_err_rows(to_host(b), ref).max() <= TOL["bf16"]
