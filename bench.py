@@ -36,9 +36,8 @@ WORKLOAD = dict(name="qwen3_8b_round", layers=36, B=1, Hq=32, Hkv=8, D=128, ctx=
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20  # written between cold timings: twice the 126 MB L2
 # DRAM bytes (read + write) of one block-attention call at this workload, from
-# the ncu capture summarised in profiles/attn_tc_partial_b8_ctx8192_full.md
-# (8-sequence case scaled to one sequence).  Valid only for the kernel source
-# it was measured on: reported as null once attn_tc.cu changes.
+# an ncu capture of the benchmarked call.  Valid only for the kernel source it
+# was measured on: reported as null once attn_tc.cu changes.
 TRAFFIC = {"attn_tc_sha256_prefix": "7b738b971b3b616f", "bytes_per_call": 34630624}
 
 
@@ -97,8 +96,9 @@ class ClockSampler:
         self.uuid, self.proc, self.path = uuid, None, None
 
     def start(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="orthrus_clocks_", suffix=".csv")
+        os.close(fd)
         try:
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                    "-lms", "100"]
@@ -115,10 +115,15 @@ class ClockSampler:
         self.proc.terminate()
         self.proc.wait()
         rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 10:
-                rows.append(parts)
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
@@ -445,6 +450,123 @@ def batched_ragged_leg(dev, hbm, launches=10):
             "frac": gbs / hbm, "launches": launches, "l2": "inputs larger than L2"}
 
 
+def attn_flops(Hq, blk, lens, D, mode):
+    """Multiply-adds x 2 of one block-attention call: Q K^T and P V over the
+    visible keys of every query row (bidir: n + blk keys per row; causal:
+    n + i + 1 for block row i)."""
+    keys = 0
+    for n in lens:
+        keys += blk * (n + blk) if mode == 0 else blk * n + blk * (blk + 1) // 2
+    return 4 * Hq * keys * D
+
+
+def ffma_peak_tflops(sm_mhz):
+    """FP32 fused multiply-add peak: 148 SMs x 4 sub-partitions x 32 FP32
+    lanes, 2 FLOP per FMA, at the given SM clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def small_config_legs(dev, hbm, sm_max_mhz=1965.0, reps=4):
+    """Block attention of the two smaller configurations, both views chained
+    layer after layer as in a round:
+      tiny: B 1, Hq 4, Hkv 2, D 64, ctx 256, block 32, FP32, one layer (its
+            0.3 MB of K/V stay in L2; the number is launch-bound);
+      qwen3_1p7b: B 1, Hq 16, Hkv 8, D 128, ctx 2048, block 32, 28 layers
+            (Qwen3-1.7B depth) so the caches (238 MB bf16, 477 MB FP32)
+            exceed the L2; bf16 (tensor cores) and FP32 (CUDA cores).
+    FP32 runs are reported as a fraction of the FP32 FMA peak, bf16 runs as a
+    fraction of the measured HBM bandwidth."""
+    import torch
+    import block_attention_b200 as ba
+    out = {}
+    cases = (("tiny_f32", 1, 4, 2, 64, 256, 32, 1, torch.float32),
+             ("qwen3_1p7b_bf16", 1, 16, 8, 128, 2048, 32, 28, torch.bfloat16),
+             ("qwen3_1p7b_f32", 1, 16, 8, 128, 2048, 32, 28, torch.float32))
+    for name, B, Hq, Hkv, D, ctx, blk, layers, dt in cases:
+        g = torch.Generator(device=dev).manual_seed(1001)
+        rnd = lambda *shape: torch.randn(*shape, generator=g, device=dev).to(dt)
+        cap = ctx + blk
+        kc, vc = rnd(layers, B, Hkv, cap, D), rnd(layers, B, Hkv, cap, D)
+        q = rnd(2, layers, B, blk, Hq, D)
+        kb, vb = rnd(2, layers, B, blk, Hkv, D), rnd(2, layers, B, blk, Hkv, D)
+        o = torch.empty_like(q)
+        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        ws = ba.Workspace(dev)
+
+        def seq():
+            for view in (0, 1):
+                for l in range(layers):
+                    ba.block_attn(q[view, l], kb[view, l], vb[view, l], kc[l], vc[l], lens, view,
+                                  out=o[view, l], max_ctx=ctx, workspace=ws,
+                                  flags=ba.ATTN_EARLY_KV)
+        seq()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            seq()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        calls = reps * 2 * layers
+        us = e0.elapsed_time(e1) * 1e3 / calls
+        es = 4 if dt == torch.float32 else 2
+        nbytes = 2 * B * ctx * Hkv * D * es + 2 * B * blk * Hq * D * es + 2 * B * blk * Hkv * D * es
+        flops = (attn_flops(Hq, blk, [ctx] * B, D, 0) + attn_flops(Hq, blk, [ctx] * B, D, 1)) / 2
+        rec = {"us_per_call": us, "bytes_per_call": nbytes, "gbs": nbytes / us / 1e3,
+               "tflops": flops / us / 1e6, "calls_timed": calls,
+               "l2": "L2-resident" if layers == 1 else "inputs larger than L2"}
+        if dt == torch.float32:
+            peak = ffma_peak_tflops(sm_max_mhz)
+            rec.update(bound="fp32 FMA", peak_tflops=peak, frac=rec["tflops"] / peak,
+                       peak_note=f"148 SMs x 128 FP32 lanes x 2 FLOP x {sm_max_mhz:.0f} MHz")
+        else:
+            rec.update(bound="hbm", peak_gbs=hbm, frac=rec["gbs"] / hbm)
+        out[name] = rec
+        del graph
+    return out
+
+
+def argmax_leg(dev, hbm, buffers=8, reps=5):
+    """The vocabulary argmax of one view at the Qwen3-8B shape (32 rows x
+    151936 fp32 logits = 19.45 MB), alone: `buffers` distinct logit matrices
+    (156 MB together, beyond the L2) read in turn, buffers x reps launches in
+    one CUDA graph.  Algorithmic bytes: the logits once."""
+    import torch
+    import block_attention_b200 as ba
+    rows, V = WORKLOAD["B"] * WORKLOAD["blk"], WORKLOAD["vocab"]
+    g = torch.Generator(device=dev).manual_seed(1007)
+    logits = [torch.randn(rows, V, generator=g, device=dev) * 3 for _ in range(buffers)]
+    idx = torch.empty(rows, dtype=torch.int32, device=dev)
+    ws = ba.Workspace(dev)
+    calls = lambda: [ba.vocab_argmax(x, idx=idx, workspace=ws) for x in logits]
+    for _ in range(3):
+        calls()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            calls()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (buffers * reps)
+    nbytes = rows * V * 4
+    del graph
+    return {"workload": f"{rows} rows x vocab {V}, fp32 logits, {buffers} buffers in turn "
+                        "(inputs larger than L2)",
+            "us_per_launch": us, "bytes_per_launch": nbytes, "gbs": nbytes / us / 1e3,
+            "peak": hbm, "frac": nbytes / us / 1e3 / hbm}
+
+
 def stochastic_round_leg(dev, hbm, iters=20):
     """The stochastic consensus step of one round at the Qwen3-8B shape (B = 1,
     block 32, vocab 151936, fp32 logits of both views): draft sampling with the
@@ -547,7 +669,47 @@ def decoder_report():
     rep["bf16_loop_vs_fp32_greedy_by_reference_perplexity"] = perplexity_report(
         out["bf16_loop"], out["fp32_greedy"], out["fp32_logprob"])
     rep["seconds"] = time.perf_counter() - t0
-    return rep
+    return rep, {"prompts": prompts, "weights": W, "fp32_greedy": out["fp32_greedy"]}
+
+
+def oracle_decoder_leg(dec_raw, prompts_n=8, n_new=64):
+    """CPU baseline of the end-to-end configuration: the float64 oracle's
+    greedy AR decoding of the first `prompts_n` prompts (`n_new` tokens each)
+    and its consensus loop on the first two, timed on this host's cores, and
+    the GPU FP32 greedy trajectories' match against the oracle's on that
+    subset (different summation orders may flip a true near-tie, so the match
+    is reported, not assumed)."""
+    import oracle
+    E = synth_workload("e2e_decoder")
+    cfg = oracle.model_cfg(E["V"], E["d"], E["L"], E["Hq"], E["Hkv"], E["hd"], E["ffn"])
+    wflat = oracle.pack_weights(cfg, dec_raw["weights"])
+    nthreads = os.cpu_count() or 1
+    sub = dec_raw["prompts"][:prompts_n]
+    t0 = time.perf_counter()
+    ref = [oracle.greedy_ar(cfg, wflat, p, n_new, nthreads=nthreads) for p in sub]
+    t_greedy = time.perf_counter() - t0
+    gpu = dec_raw["fp32_greedy"][:prompts_n, :n_new]
+    exact = [bool(np.array_equal(gpu[b], ref[b])) for b in range(len(sub))]
+    tok = [float(np.mean(gpu[b] == ref[b])) for b in range(len(sub))]
+    n_cons = 32
+    t0 = time.perf_counter()
+    cons, _ = oracle.consensus_decode(cfg, wflat, sub[-1], n_cons, blk=E["blk"],
+                                      nthreads=nthreads)
+    t_cons = time.perf_counter() - t0
+    return {"subset": f"first {len(sub)} prompts (lengths {[len(p) for p in sub]}), "
+                      f"{n_new} greedy tokens each; consensus loop on the last of them, "
+                      f"{n_cons} tokens",
+            "cores": nthreads,
+            "greedy_tokens_per_s": len(sub) * n_new / t_greedy,
+            "consensus_tokens_per_s": n_cons / t_cons,
+            "consensus_equals_greedy": bool(np.array_equal(cons, ref[-1][:n_cons])),
+            "gpu_fp32_greedy_vs_oracle_exact_match_rate": float(np.mean(exact)),
+            "gpu_fp32_greedy_vs_oracle_token_match_rate": float(np.mean(tok))}
+
+
+def synth_workload(name):
+    from block_attention_b200 import synth
+    return synth.WORKLOADS[name]
 
 
 def main():
@@ -608,6 +770,21 @@ def main():
     expect_ne = np.minimum(rnd.accept + 1, w["blk"])
     assert np.array_equal(rnd.n_emit.cpu().numpy(), expect_ne), "round result mismatch"
     assert int(rnd.err.item()) == 0
+    # The kernels are deterministic: a sampled layer's attention output of both
+    # views, poisoned before each measured loop, must come back bit-identical.
+    probe_layer = w["layers"] // 2
+    attn_ref = rnd.out[:, probe_layer].clone()
+
+    def poison_probe():
+        rnd.out[:, probe_layer].fill_(float("nan"))
+        torch.cuda.synchronize()
+
+    def check_probe(where):
+        torch.cuda.synchronize()
+        assert int(rnd.err.item()) == 0, f"device error word set during the {where}"
+        assert torch.equal(rnd.out[:, probe_layer], attn_ref), \
+            f"layer {probe_layer} attention differs after the {where}"
+    poison_probe()
 
     # ---- timed region: K rounds from the graphs, inputs resident in HBM
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
@@ -631,6 +808,7 @@ def main():
     time.sleep(0.2)
     clk = clocks.stop()
 
+    check_probe("timed rounds")
     step_ms = [e[0].elapsed_time(e[4]) for e in ev]
     attn_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev]
     total_ms = ev[0][0].elapsed_time(ev[-1][4])
@@ -649,6 +827,7 @@ def main():
     for _ in range(2):
         rnd.h2d(h_in); rnd.replay(); rnd.d2h(h_out)
     torch.cuda.synchronize()
+    poison_probe()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -662,18 +841,43 @@ def main():
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
     e2e_rounds = whole_job_rate(world, args.steps, e2e_ms)
     assert np.array_equal(h_out["n_emit"].numpy(), expect_ne)
+    check_probe("end-to-end rounds")
+
+    dec = dec_raw = None
+    if rank == 0 and world == 1 and not args.no_e2e_decoder:
+        dec, dec_raw = decoder_report()
+
+    # ---- the same rounds without the next-layer L2 warm-up (for comparison)
+    nopf = None
+    if not args.no_batched:
+        rnd.prefetch = False
+        rnd.capture()
+        for _ in range(args.warmup):
+            rnd.replay()
+        poison_probe()
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+        for k in range(args.steps):
+            rnd.replay(ev2[k])
+        check_probe("rounds without prefetch")
+        a2 = max_over_ranks([sum(e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev2),
+                             ev2[0][0].elapsed_time(ev2[-1][4])], dev)
+        us2 = a2[0] * 1e3 / launches_attn
+        nopf = {"us_per_launch": us2, "gbs": bytes_per_launch / us2 / 1e3,
+                "pct_of_peak": 100.0 * bytes_per_launch / us2 / 1e3 / hbm,
+                "rounds_per_s": whole_job_rate(world, args.steps, a2[1])}
+        rnd.prefetch = True
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = oracle_round_sample(heads=WORKLOAD["Hkv"], layers_timed=4)
         cpu = {"value": v, "unit": "rounds/s", "cores": cores, "kind": "oracle",
                "sample": sample}
-
-    dec = None
-    if rank == 0 and world == 1 and not args.no_e2e_decoder:
-        dec = decoder_report()
-    batched = stochastic = lm_head = None
+        if dec_raw is not None:
+            cpu["e2e_decoder"] = oracle_decoder_leg(dec_raw)
+    batched = stochastic = lm_head = small = amax = None
     if rank == 0 and world == 1 and not args.no_batched:
+        small = small_config_legs(dev, hbm)
+        amax = argmax_leg(dev, hbm)
         batched = batched_ragged_leg(dev, hbm)
         stochastic = stochastic_round_leg(dev, hbm)
         lm_head = lm_head_leg(dev)
@@ -692,7 +896,9 @@ def main():
         "data": "synthetic", "config": config_dict(),
         "block_attn": {"gbs": achieved, "pct_of_peak": 100.0 * achieved / hbm,
                        "us_per_launch": attn_launch_us, "bytes_per_launch": bytes_per_launch,
-                       "launches_per_round": 2 * w["layers"]},
+                       "launches_per_round": 2 * w["layers"],
+                       "next_layer_l2_prefetch": True},
+        "block_attn_without_prefetch": nopf,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "peak_source": src, "traffic": measured_traffic(),
                      "kernel": "block_attn (both views, per-layer launches)"},
@@ -705,6 +911,8 @@ def main():
         "clocks": clk,
         "cpu_baseline": cpu,
         "e2e_decoder": dec,
+        "block_attn_small_configs": small,
+        "vocab_argmax": amax,
         "block_attn_batched_ragged": batched,
         "stochastic_consensus": stochastic,
         "lm_head_argmax": lm_head,

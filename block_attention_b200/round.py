@@ -37,7 +37,7 @@ def _dev(a: np.ndarray, device) -> torch.Tensor:
 class DecodeRound:
     def __init__(self, *, layers, B, Hq, Hkv, D, blk, vocab, ctx_lens, cap=None,
                  dtype="bf16", logits_dtype="f32", accept_mean=5.4, seed=0,
-                 device="cuda"):
+                 device="cuda", prefetch=True):
         self.dev = torch.device(device)
         self.L, self.B, self.Hq, self.Hkv, self.D, self.blk, self.V = (
             layers, B, Hq, Hkv, D, blk, vocab)
@@ -83,19 +83,27 @@ class DecodeRound:
         self.err = torch.zeros(1, **i32)
         self.ws = {k: Workspace(dev) for k in ("attn0", "attn1", "argmax", "commit")}
         self.graphs = None
+        self.prefetch = prefetch
 
     # ------------------------------------------------------------ segments
     def _attn(self, view):
-        # Within a view the kernel before each attention call is the previous
-        # layer's attention (or, for layer 0, the length reset copy / the
-        # diffusion argmax): none of them writes a cache or the lengths, so the
-        # cache may start streaming before that kernel has finished.
+        # ATTN_EARLY_KV promises that the work right before the call writes
+        # neither a cache nor the lengths.  It holds for every layer after the
+        # first (the previous layer's attention) and for the verify view's
+        # first layer (the diffusion argmax).  The diffusion view's first
+        # layer follows the copy that resets ctx_lens, so it waits for it.
+        # With `prefetch`, each call warms L2 with the cache the next
+        # attention call reads: the next layer's, and after the last layer
+        # the first layer's (the other view's pass, or the next round's).
         mode = BIDIR_BLOCK if view == 0 else CAUSAL_VERIFY
         for l in range(self.L):
+            early = not (view == 0 and l == 0)
+            nxt = (l + 1) % self.L
             block_attn(self.q[view, l], self.k_blk[view, l], self.v_blk[view, l],
                        self.k_cache[l], self.v_cache[l], self.ctx_lens, mode,
                        out=self.out[view, l], max_ctx=self.max_ctx, err=self.err,
-                       workspace=self.ws[f"attn{view}"], flags=ATTN_EARLY_KV)
+                       workspace=self.ws[f"attn{view}"], flags=ATTN_EARLY_KV if early else 0,
+                       next_kv=(self.k_cache[nxt], self.v_cache[nxt]) if self.prefetch else None)
 
     def seg_a(self):
         self.ctx_lens.copy_(self.ctx_base)  # same round every step
