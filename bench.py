@@ -207,15 +207,17 @@ def reference_arm(args, rank, world):
 # ---------------------------------------------------------------- one kernel alone
 
 def kernel_alone(args):
-    """Block attention alone at the Qwen3-8B layer shape, B=8 sequences of
-    context 8192 (269 MB of K/V, over twice the L2), bidirectional view:
+    """Block attention alone at the Qwen3-8B layer shape, bidirectional view:
+    B sequences of context 8192 (--attn-batch; 8 by default: 269 MB of K/V,
+    over twice the L2; 1: the call the round makes, whose 34 MB stay in L2
+    across launches, so only a cold-cache profile reads them from HBM).
     W warm-up launches, then K launches captured in one CUDA graph."""
     import torch
     import block_attention_b200 as ba
     from block_attention_b200.round import _dev
     from block_attention_b200 import synth
     w = WORKLOAD
-    B, ctx = 8, w["ctx"]
+    B, ctx = args.attn_batch, w["ctx"]
     cap = ctx + w["blk"]
     dev = torch.device("cuda", 0)
     inp = synth.attn_inputs(B, w["Hq"], w["Hkv"], w["D"], w["blk"], [ctx] * B, cap, "bf16",
@@ -567,6 +569,73 @@ def argmax_leg(dev, hbm, buffers=8, reps=5):
             "peak": hbm, "frac": nbytes / us / 1e3 / hbm}
 
 
+def projected_round_leg(dev, hbm, steps=10, warmup=3):
+    """A round with the attention block's projections and the LM head on the
+    path (block_attention_b200.projected): Qwen3-8B shape, 36 layers, both
+    views each computing Q and the block K/V from the hidden states (RMSNorm,
+    QKV projection, RoPE), attending, projecting back with the residual,
+    then the LM head with the argmax fused; consensus and commit.  Reported:
+    rounds/s of the captured round, its algorithmic bytes, and the projection
+    kernels alone (36 layers' weights in turn, beyond the L2) against the
+    measured HBM bandwidth."""
+    import torch
+    import block_attention_b200 as ba
+    from block_attention_b200.projected import ProjectedRound
+    rnd = ProjectedRound(layers=WORKLOAD["layers"], ctx=WORKLOAD["ctx"], seed=1009,
+                         device=dev)
+    rnd.capture()
+    for _ in range(warmup):
+        rnd.replay()
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    e0, e1 = ev(), ev()
+    e0.record()
+    for _ in range(steps):
+        rnd.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    assert int(rnd.err.item()) == 0
+    ms = e0.elapsed_time(e1) / steps
+    rb = rnd.bytes_per_round()
+    out = {"workload": "Qwen3-8B attention path: 36 layers x 2 views of RMSNorm, QKV "
+                       "projection (4096 -> 6144), RoPE, block attention (ctx 8192), output "
+                       "projection (4096 -> 4096) with residual; LM head (vocab 151936) with "
+                       "the argmax fused; bf16 random weights",
+           "rounds_per_s": 1e3 / ms, "ms_per_round": ms, "bytes_per_round": rb,
+           "round_gbs": sum(rb.values()) / (ms * 1e-3) / 1e9,
+           "kernels_per_round": rnd.kernels_per_round()}
+    # the projections alone, each layer's weights in turn (graph of 36 calls)
+    x = torch.randn(WORKLOAD["blk"], rnd.d, device=dev).to(torch.bfloat16)
+    for name, W, N in (("qkv_projection", rnd.wqkv[1], rnd.wqkv.shape[2]),
+                       ("output_projection", rnd.wo[1], rnd.d)):
+        y = torch.empty(WORKLOAD["blk"], N, dtype=torch.bfloat16, device=dev)
+        ws = ba.Workspace(dev)
+        # (the output projection's input is [blk, Hq * D] = [blk, 4096], like x)
+        seq = lambda: [ba.linear_tc(x, W[l], out=y, workspace=ws) for l in range(rnd.L)]
+        seq()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            seq()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(3):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (3 * rnd.L)
+        nbytes = N * rnd.d * 2 + WORKLOAD["blk"] * (rnd.d + N) * 2
+        out[name] = {"us_per_call": us, "bytes_per_call": nbytes, "gbs": nbytes / us / 1e3,
+                     "frac": nbytes / us / 1e3 / hbm,
+                     "shape": f"{WORKLOAD['blk']} x {rnd.d} -> {N}"}
+        del g
+    del rnd
+    torch.cuda.empty_cache()
+    return out
+
+
 def stochastic_round_leg(dev, hbm, iters=20):
     """The stochastic consensus step of one round at the Qwen3-8B shape (B = 1,
     block 32, vocab 151936, fp32 logits of both views): draft sampling with the
@@ -724,6 +793,9 @@ def main():
     ap.add_argument("--no-batched", action="store_true",
                     help="skip the batched ragged attention, stochastic consensus and LM-head "
                          "legs (they run after the timing)")
+    ap.add_argument("--attn-batch", type=int, default=8,
+                    help="sequences of the --kernel attn case (8: larger than L2; 1: the "
+                         "round's call)")
     ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
                          "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
@@ -874,10 +946,11 @@ def main():
                "sample": sample}
         if dec_raw is not None:
             cpu["e2e_decoder"] = oracle_decoder_leg(dec_raw)
-    batched = stochastic = lm_head = small = amax = None
+    batched = stochastic = lm_head = small = amax = proj = None
     if rank == 0 and world == 1 and not args.no_batched:
         small = small_config_legs(dev, hbm)
         amax = argmax_leg(dev, hbm)
+        proj = projected_round_leg(dev, hbm)
         batched = batched_ragged_leg(dev, hbm)
         stochastic = stochastic_round_leg(dev, hbm)
         lm_head = lm_head_leg(dev)
@@ -913,6 +986,7 @@ def main():
         "e2e_decoder": dec,
         "block_attn_small_configs": small,
         "vocab_argmax": amax,
+        "projected_round": proj,
         "block_attn_batched_ragged": batched,
         "stochastic_consensus": stochastic,
         "lm_head_argmax": lm_head,

@@ -86,6 +86,7 @@ EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_consensus_sample", "orthrus_consensus_sample_workspace",
            "orthrus_lm_head_argmax", "orthrus_lm_head_argmax_workspace",
            "orthrus_lm_head_argmax_plan",
+           "orthrus_linear_tc", "orthrus_linear_tc_workspace", "orthrus_linear_tc_plan",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
            "orthrus_swiglu", "orthrus_block_tokens")
@@ -138,6 +139,11 @@ def lib() -> ctypes.CDLL:
         L.orthrus_vocab_sample.argtypes = [i32, vp, i32, i32, i64, c.c_float, c.c_uint64,
                                            c.c_uint32, vp, vp, vp, vp, sz, vp]
         L.orthrus_consensus_sample.argtypes = [c.POINTER(SampleArgs), vp]
+        L.orthrus_linear_tc_workspace.argtypes = [i32, i32, i32]
+        L.orthrus_linear_tc_workspace.restype = sz
+        L.orthrus_linear_tc_plan.argtypes = [i32, i32, i32, i32, vp]
+        L.orthrus_linear_tc.argtypes = [i32, vp, i32, i32, i64, vp, i32, vp, vp, i64, vp, vp, sz,
+                                        vp]
         L.orthrus_lm_head_argmax_plan.argtypes = [i32, i32, i32, i32, vp]
         L.orthrus_lm_head_argmax_workspace.argtypes = [i32]
         L.orthrus_lm_head_argmax_workspace.restype = sz
@@ -475,3 +481,30 @@ def lm_head_argmax(h, w, *, idx=None, maxval=None, err=None, workspace=None, str
         _dtype(h), _ptr(h), rows, d, h.stride(0), _ptr(w), w.shape[0], _ptr(idx),
         _ptr(maxval), _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
     return idx
+
+
+def linear_tc(x, w, *, residual=None, out=None, err=None, workspace=None, stream=None):
+    """bf16 [rows, N] = x @ w.T on the tensor cores (plus the residual, each
+    sum rounded to bf16 first; see orthrus.h).  x bf16 [rows, K] (unit
+    column stride), w bf16 [N, K] contiguous, residual/out bf16 [rows, N]
+    with unit column stride (out may be the residual)."""
+    _dev(w, residual, out, err)
+    if not x.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (no CPU path)")
+    if x.dim() != 2 or w.dim() != 2 or x.stride(1) != 1 or not w.is_contiguous():
+        raise ValueError("x must be 2-D with unit column stride, w 2-D contiguous")
+    rows, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("x and w disagree on K")
+    if out is None:
+        out = torch.empty(rows, N, dtype=x.dtype, device=x.device)
+    if out.shape != (rows, N) or out.stride(1) != 1:
+        raise ValueError("out must be [rows, N] with unit column stride")
+    if residual is not None and (residual.shape != (rows, N) or residual.stride() != out.stride()):
+        raise ValueError("residual must be laid out like out")
+    buf = _ws(workspace, x.device, "linear").get(lib().orthrus_linear_tc_workspace(rows, K, N))
+    _check("orthrus_linear_tc", lib().orthrus_linear_tc(
+        _dtype(x), _ptr(x), rows, K, x.stride(0), _ptr(w), N, _ptr(residual), _ptr(out),
+        out.stride(0), _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
+    return out

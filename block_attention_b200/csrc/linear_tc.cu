@@ -1,0 +1,446 @@
+// linear_tc.cu -- the attention block's projections on the tensor cores:
+//   y[r, n] = bf16( sum_k x[r, k] w[n, k] )              (residual == NULL)
+//   y[r, n] = bf16( residual[r, n] + bf16(sum_k ...) )    (otherwise)
+// for a handful of rows (the 32 rows of a decoding block) against a large
+// weight matrix w [N, K] (the QKV and output projections around the round's
+// attention -- cjcn.com.cn explainer of "Orthrus", §二: the diffusion view
+// has its own copy of these projections, everything else is shared).
+//
+// With 32 rows the product is weight-streaming: every weight byte is used
+// 32 times, so the bound is HBM.  tcgen05 GEMM with the weights as the A
+// operand (M = 128 output features per tile, from shared memory) and the
+// rows as the B operand (N = rows rounded up to 16), so one MMA of K = 16
+// consumes 4 KB of weights.  A tile's K range is split over `ksplit` CTAs so
+// the 32-48 tiles of a projection fill the SMs; each writes its fp32 partial
+// to the workspace and the tile's last CTA (ticket) sums the partials in
+// split order -- the result does not depend on timing -- and writes y.  Per
+// CTA:
+//   warp 0     TMA producer: per 64-wide K step one box of 128 weight rows
+//              (16 KB, 128-byte swizzle) and one box of the x rows, through
+//              a ring of stages.  The weights never depend on the preceding
+//              kernel, so the first stages' weight boxes are requested before
+//              the programmatic-dependency wait; x only after it.
+//   warp 1     MMA issuer (one thread): 4 MMAs per K step into one TMEM
+//              accumulator (128 lanes = output features, rows in columns).
+//   warps 2-5  epilogue: each thread owns one output feature (TMEM lane) and
+//              reads its row of results 32 columns at a time.
+// Every mbarrier wait is bounded: on a timeout the kernel records
+// ORTHRUS_ETIMEOUT, stops issuing, drains what it issued and still takes its
+// ticket, so it always terminates.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "orthrus.h"
+#include "tc_ptx.cuh"
+
+namespace orthrus {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTileN = 128;                // output features per tile (UMMA M)
+constexpr int kStepK = 64;                 // K per box: one 128-byte swizzle row
+constexpr int kMaxRows = 128;              // x rows per call (UMMA N)
+constexpr int kMaxStages = 16;
+constexpr int kRingBudget = 208 * 1024;
+constexpr int kWBox = kTileN * 128;        // bytes of one weight box
+constexpr int kNumBars = 2 * kMaxStages + 2;
+
+struct __align__(64) LinParams {
+  CUtensorMap tm_w;  // 2D (K, N), box (64, 128)
+  CUtensorMap tm_x;  // 2D (K, R), row pitch ldx, box (64, Rp); rows past R read as zero
+  const __nv_bfloat16* residual;  // [R] rows of pitch ldy, or null
+  __nv_bfloat16* y;               // [R] rows of pitch ldy
+  float* part;                    // [tiles][ksplit][Rp][128] fp32 split-K partials
+  unsigned* tickets;              // [tiles], zero between calls
+  int32_t* err;
+  int R, Rp, N, ldy, tiles, ksplit, ksteps, stages, stage_bytes, tmem_cols;
+};
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t at(int i) const { return base + 8 * i; }
+  __device__ uint32_t full(int s) const { return at(s); }
+  __device__ uint32_t empty(int s) const { return at(kMaxStages + s); }
+  __device__ uint32_t acc_full() const { return at(2 * kMaxStages); }
+  __device__ uint32_t red_full() const { return at(2 * kMaxStages + 1); }  // partials staged
+};
+
+__device__ __forceinline__ void record_timeout(int32_t* err, volatile int* abort_flag) {
+  *abort_flag = 1;
+  set_err(err, ORTHRUS_ETIMEOUT);
+}
+
+__device__ __forceinline__ float bf16_round(float v) {
+  return __uint_as_float(ptx::pack_bf16x2(v, 0.f) << 16);
+}
+
+// out = bf16(sum) or bf16(residual + bf16(sum))
+__device__ __forceinline__ __nv_bfloat16 finish(float sum, const __nv_bfloat16* res) {
+  float v = bf16_round(sum);
+  if (res) v = __bfloat162float(*res) + v;
+  return __float2bfloat16_rn(v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_constant__ LinParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned full_mask = 0xffffffffu;
+  const int ST = p.stages, SB = p.stage_bytes;
+  const Bars bars{sbase + (uint32_t)(ST * SB)};
+  uint8_t* misc = smem + ST * SB + kNumBars * 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 8);
+
+  const int tile = blockIdx.x / p.ksplit, ks = blockIdx.x % p.ksplit;
+  const int k_beg = (int)((int64_t)ks * p.ksteps / p.ksplit);
+  const int nk = (int)((int64_t)(ks + 1) * p.ksteps / p.ksplit) - k_beg;
+  const int n0 = tile * kTileN;
+  const uint32_t x_bytes = (uint32_t)(p.Rp * 128);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    *last_flag = 0;
+    for (int s = 0; s < ST; ++s) {
+      ptx::mbar_init(bars.full(s), 1);
+      ptx::mbar_init(bars.empty(s), 1);
+    }
+    ptx::mbar_init(bars.acc_full(), 1);
+    ptx::mbar_init(bars.red_full(), 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::tma_prefetch_desc(&p.tm_w);
+    ptx::tma_prefetch_desc(&p.tm_x);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), (uint32_t)p.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  ptx::griddep_launch_dependents();
+
+  // the weights are constant: their first boxes stream before the wait for
+  // the preceding kernel (which may be writing x or the residual)
+  const int early = min(nk, ST);
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < early; ++i) {
+      ptx::mbar_expect_tx(bars.full(i), (uint32_t)kWBox + x_bytes);
+      ptx::tma_load_2d(sbase + (uint32_t)(i * SB), &p.tm_w, bars.full(i), (k_beg + i) * kStepK,
+                       n0);
+    }
+  }
+  ptx::griddep_wait();
+
+  if (warp == 0) {
+    // ================================================== TMA producer
+    if (lane == 0) {
+      // the x boxes of the early stages first: with them every stage whose
+      // weights are in flight can complete
+      for (int i = 0; i < early; ++i)
+        ptx::tma_load_2d(sbase + (uint32_t)(i * SB + kWBox), &p.tm_x, bars.full(i),
+                         (k_beg + i) * kStepK, 0);
+      int issued = early;
+      for (int i = early; i < nk; ++i) {
+        if (*abort_flag) break;
+        const int s = i % ST;
+        const uint32_t dst = sbase + (uint32_t)(s * SB);
+        if (!ptx::mbar_wait(bars.empty(s), ((i / ST) & 1) ^ 1)) {
+          record_timeout(p.err, abort_flag);
+          break;
+        }
+        ptx::mbar_expect_tx(bars.full(s), (uint32_t)kWBox + x_bytes);
+        ptx::tma_load_2d(dst, &p.tm_w, bars.full(s), (k_beg + i) * kStepK, n0);
+        ptx::tma_load_2d(dst + kWBox, &p.tm_x, bars.full(s), (k_beg + i) * kStepK, 0);
+        issued = i + 1;
+      }
+      // every issued load lands before the CTA can exit
+      for (int u = max(0, issued - ST); u < issued; ++u)
+        if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(p.err, abort_flag);
+    }
+  } else if (warp == 1) {
+    // ================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t id = ptx::idesc_bf16(kTileN, p.Rp, false, false);
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % ST;
+        if (*abort_flag || !ptx::mbar_wait(bars.full(s), (i / ST) & 1)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t wa = sbase + (uint32_t)(s * SB);
+#pragma unroll
+        for (int kk = 0; kk < kStepK / 16; ++kk)
+          ptx::mma_ss(tmem, ptx::sdesc_sw128(wa + kk * 32, 16, 1024),
+                      ptx::sdesc_sw128(wa + kWBox + kk * 32, 16, 1024), id,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        ptx::tc_commit(bars.empty(s));
+      }
+      if (!ok) record_timeout(p.err, abort_flag);
+      ptx::tc_commit(bars.acc_full());  // also: every MMA has finished
+      if (!ptx::mbar_wait(bars.acc_full(), 0)) record_timeout(p.err, abort_flag);
+    }
+  } else {
+    // ================================================== epilogue
+    const int quad = warp & 3;
+    const int n = quad * 32 + lane;  // output feature within the tile (TMEM lane)
+    const int ng = n0 + n;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    bool ok = nk > 0 && __all_sync(full_mask, ptx::mbar_wait(bars.acc_full(), 0));
+    if (nk > 0 && !ok) record_timeout(p.err, abort_flag);
+    ok = ok && !__any_sync(full_mask, *abort_flag != 0);
+    if (ok) ptx::tc_fence_after();
+    float* part = p.part + ((int64_t)tile * p.ksplit + ks) * p.Rp * kTileN;
+    for (int cb = 0; cb < p.Rp; cb += 32) {
+      uint32_t d[32];
+      if (ok) {
+        if (p.Rp - cb >= 32) {
+          ptx::tmem_ld32_sync(lane_addr + (uint32_t)cb, d);
+        } else {  // the last 16 columns (Rp is a multiple of 16)
+          uint32_t d16[16];
+          ptx::tmem_ld16_sync(lane_addr + (uint32_t)cb, d16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) d[j] = d16[j];
+#pragma unroll
+          for (int j = 16; j < 32; ++j) d[j] = 0u;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) d[j] = 0u;
+      }
+      if (p.ksplit == 1) {
+        if (ng < p.N) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int r = cb + j;
+            if (r < p.R && ok) {
+              const int64_t o = (int64_t)r * p.ldy + ng;
+              p.y[o] = finish(__uint_as_float(d[j]), p.residual ? p.residual + o : nullptr);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (cb + j < p.Rp) __stcg(part + (int64_t)(cb + j) * kTileN + n, __uint_as_float(d[j]));
+      }
+    }
+  }
+
+  // ---- teardown; with split K, the tile's last CTA sums the partials
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+  }
+  if (p.ksplit == 1) return;
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's partial is visible before its ticket
+    *last_flag = atomicAdd(p.tickets + tile, 1u) == (unsigned)p.ksplit - 1u;
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  // the tile's partials (one contiguous Rp x 128 block per split) come into
+  // the idle ring by bulk copies, all in flight at once, then are summed in
+  // split order
+  const float* base = p.part + (int64_t)tile * p.ksplit * p.Rp * kTileN;
+  const uint32_t blk_bytes = (uint32_t)(p.Rp * kTileN * 4);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    ptx::fence_proxy_async_global();  // the partials were written by generic stores
+    ptx::mbar_expect_tx(bars.red_full(), blk_bytes * (uint32_t)p.ksplit);
+    for (int s = 0; s < p.ksplit; ++s)
+      ptx::bulk_g2s(sbase + (uint32_t)s * blk_bytes, base + (int64_t)s * p.Rp * kTileN, blk_bytes,
+                    bars.red_full());
+  }
+  if (!ptx::mbar_wait(bars.red_full(), 0)) {
+    set_err(p.err, ORTHRUS_ETIMEOUT);
+  } else {
+    const float* st = reinterpret_cast<const float*>(smem);
+    for (int e = threadIdx.x; e < p.R * kTileN; e += kThreads) {
+      const int r = e / kTileN, n = e % kTileN, ng = n0 + n;
+      if (ng >= p.N) continue;
+      float sum = 0.f;
+      for (int s = 0; s < p.ksplit; ++s) sum += st[((int64_t)s * p.Rp + r) * kTileN + n];
+      const int64_t o = (int64_t)r * p.ldy + ng;
+      p.y[o] = finish(sum, p.residual ? p.residual + o : nullptr);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) p.tickets[tile] = 0u;
+}
+
+// ------------------------------------------------------------------ host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t pitch_bytes,
+               int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)pitch_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)kStepK, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+struct Plan {
+  int Rp, tiles, ksplit, ksteps, stages, stage_bytes, smem, tmem_cols;
+};
+
+// Launch shape for rows x K x N on `sms` SMs: 128-feature tiles, the K range
+// of each split over enough CTAs to fill the SMs (at most one 64-wide K step
+// less than an even share each), a ring of as many stages as fit.
+Plan plan(int rows, int K, int N, int sms) {
+  Plan q;
+  q.Rp = (rows + 15) / 16 * 16;
+  q.ksteps = K / kStepK;
+  q.tiles = ceil_div(N, kTileN);
+  q.stage_bytes = kWBox + (q.Rp * 128 + 1023) / 1024 * 1024;
+  q.stages = min(kMaxStages, kRingBudget / q.stage_bytes);
+  // splits: enough to fill the SMs, at most one per K step, at most 16, and
+  // no more than the ring can stage for the last CTA's sum
+  q.ksplit = q.tiles >= sms ? 1 : sms / q.tiles;
+  q.ksplit = min(q.ksplit, min(q.ksteps, 16));
+  q.ksplit = max(1, min(q.ksplit, q.stages * q.stage_bytes / (q.Rp * kTileN * 4)));
+  q.smem = q.stages * q.stage_bytes + kNumBars * 8 + 16 + 1024;
+  q.tmem_cols = 32;
+  while (q.tmem_cols < q.Rp) q.tmem_cols *= 2;
+  return q;
+}
+
+size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
+
+size_t workspace_bytes(int rows, int K, int N) {
+  // sized for any SM count up to 256
+  const Plan q = plan(rows, K, N, 256);
+  const int64_t parts = q.ksplit > 1 ? (int64_t)q.tiles * 16 * q.Rp * kTileN * 4 : 0;
+  return round256((int64_t)q.tiles * 4) + (size_t)parts;
+}
+
+bool prepare() {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64 && done[dev]) return true;
+  if (cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           227 * 1024) != cudaSuccess)
+    return false;
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return true;
+}
+
+}  // namespace
+}  // namespace orthrus
+
+using namespace orthrus;
+
+extern "C" {
+
+int orthrus_linear_tc_plan(int32_t rows, int32_t K, int32_t N, int32_t sms, int32_t* out) {
+  if (!out || rows < 1 || rows > kMaxRows || K < kStepK || K % kStepK || N < 1 || sms < 1)
+    return ORTHRUS_EINVAL;
+  const Plan q = plan(rows, K, N, sms);
+  out[0] = q.tiles;
+  out[1] = q.ksplit;
+  out[2] = q.stages;
+  out[3] = q.stage_bytes;
+  out[4] = q.smem;
+  out[5] = q.tiles * q.ksplit;  // grid
+  out[6] = q.tmem_cols;
+  out[7] = q.Rp;
+  return ORTHRUS_OK;
+}
+
+size_t orthrus_linear_tc_workspace(int32_t rows, int32_t K, int32_t N) {
+  if (rows < 1 || rows > kMaxRows || K < kStepK || K % kStepK || N < 1) return 0;
+  return workspace_bytes(rows, K, N);
+}
+
+int orthrus_linear_tc(int32_t dtype, const void* x, int32_t rows, int32_t K, int64_t ldx,
+                      const void* w, int32_t N, const void* residual, void* y, int64_t ldy,
+                      int32_t* err, void* workspace, size_t workspace_bytes_given,
+                      orthrus_stream_t stream) {
+  if (dtype != ORTHRUS_F32 && dtype != ORTHRUS_BF16) return ORTHRUS_EINVAL;
+  if (rows < 0 || K <= 0 || N <= 0 || ldx < K || ldy < N) return ORTHRUS_EINVAL;
+  if (dtype != ORTHRUS_BF16) return ORTHRUS_EUNSUPPORTED;
+  if (rows == 0) return ORTHRUS_OK;
+  if (rows > kMaxRows || K % kStepK || ldx % 8) return ORTHRUS_EUNSUPPORTED;
+  if (!x || !w || !y) return ORTHRUS_EINVAL;
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w) % 16 ||
+      reinterpret_cast<uintptr_t>(y) % 2 || reinterpret_cast<uintptr_t>(residual) % 2)
+    return ORTHRUS_EINVAL;
+  if (!workspace || workspace_bytes_given < workspace_bytes(rows, K, N) ||
+      reinterpret_cast<uintptr_t>(workspace) % 256)
+    return ORTHRUS_EWORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return ORTHRUS_ECUDA;
+  if (!prepare()) return ORTHRUS_ECUDA;
+  const Plan q = plan(rows, K, N, sms);
+  LinParams p;
+  if (!encode_2d(&p.tm_w, w, K, N, (int64_t)K * 2, kTileN) ||
+      !encode_2d(&p.tm_x, x, K, rows, ldx * 2, q.Rp))
+    return ORTHRUS_ECUDA;
+  char* ws = static_cast<char*>(workspace);
+  p.tickets = reinterpret_cast<unsigned*>(ws);
+  p.part = reinterpret_cast<float*>(ws + round256((int64_t)q.tiles * 4));
+  p.residual = static_cast<const __nv_bfloat16*>(residual);
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.err = err;
+  p.R = rows; p.Rp = q.Rp; p.N = N; p.ldy = (int)ldy;
+  p.tiles = q.tiles; p.ksplit = q.ksplit; p.ksteps = q.ksteps; p.stages = q.stages;
+  p.stage_bytes = q.stage_bytes; p.tmem_cols = q.tmem_cols;
+
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(q.tiles * q.ksplit);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = q.smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, linear_tc_kernel, p) == cudaSuccess ? ORTHRUS_OK
+                                                                        : ORTHRUS_ECUDA;
+}
+
+}  // extern "C"

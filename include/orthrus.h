@@ -370,6 +370,40 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
                            float* maxval, int32_t* err, void* workspace,
                            size_t workspace_bytes, orthrus_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Projection on the tensor cores: the attention block's QKV and output
+ * projections around the round's attention (explainer §二: the diffusion
+ * view has its own copy of the attention projections, the AR view uses the
+ * frozen model's), for the few rows of a decoding block:
+ *   y[r, n] = bf16( sum_k x[r, k] w[n, k] )                  residual == NULL
+ *   y[r, n] = bf16( residual[r, n] + bf16(sum_k x[r, k] w[n, k]) )
+ * x [rows, K] (row pitch ldx elements), w [N, K] dense (the PyTorch Linear
+ * layout), residual and y [rows, N] (row pitch ldy; y may alias residual).
+ * The sum is an fp32 accumulation of exact bf16 products on the tensor cores
+ * (128 output features per tile; a tile's K range split over several CTAs
+ * whose fp32 partials are added in a fixed order), so the result does not
+ * depend on timing but may differ from an exactly rounded product by one
+ * bf16 step.  w is read before the wait on the preceding kernel (it may not
+ * be written by the kernel right before this call on the stream); x and the
+ * residual only after it.
+ * Limits: dtype ORTHRUS_BF16 (ORTHRUS_F32: ORTHRUS_EUNSUPPORTED);
+ * 1 <= rows <= 128 (0: no-op); K a multiple of 64; ldx a multiple of 8;
+ * x, w 16-byte aligned.  err (nullable) receives ORTHRUS_ETIMEOUT if a
+ * bounded wait inside the kernel gave up.  workspace:
+ * orthrus_linear_tc_workspace(rows, K, N) bytes, 256-byte aligned, zeroed
+ * once; every call leaves its ticket counters zero.  One launch.
+ * ---------------------------------------------------------------------- */
+size_t orthrus_linear_tc_workspace(int32_t rows, int32_t K, int32_t N);
+/* The launch for these sizes on a GPU with `sms` SMs (host only): out[0..8)
+ * = 128-feature tiles, K splits per tile, ring stages, bytes per stage,
+ * dynamic shared memory, grid, TMEM columns, rows rounded up to 16.
+ * ORTHRUS_EINVAL outside the limits above. */
+int orthrus_linear_tc_plan(int32_t rows, int32_t K, int32_t N, int32_t sms, int32_t* out);
+int orthrus_linear_tc(int32_t dtype, const void* x, int32_t rows, int32_t K, int64_t ldx,
+                      const void* w, int32_t N, const void* residual, void* y, int64_t ldy,
+                      int32_t* err, void* workspace, size_t workspace_bytes,
+                      orthrus_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 const char* orthrus_status_str(int status);
 int orthrus_version(void);

@@ -182,6 +182,36 @@ def lm_head_argmax(h, w, chunk=8192):
     return idx, mx, gap, mag
 
 
+def round_bf16(x):
+    """float64 -> bf16 bit patterns (uint16), rounding once, to nearest with
+    ties to even, straight from the float64 value: x = m 2^e with
+    0.5 <= |m| < 1, and bf16 keeps 8 significant bits, so m is rounded to a
+    multiple of 2^-8.  Finite inputs of normal bf16 range only."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    y = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)  # np.rint: ties to even
+    return (y.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def projection(x, w, residual=None):
+    """A linear layer of a bf16 model (the attention block's QKV and output
+    projections around the round's attention; explainer §二: the diffusion
+    view has its own copy of them): y[r, n] = sum_k x[r, k] w[n, k] in
+    float64 over the exactly widened bf16 inputs, rounded to bf16; with a
+    residual, y = bf16(residual + that rounded product).  x [R, K], w [N, K]
+    (PyTorch Linear layout), residual [R, N], all bf16 bit patterns.  Returns
+    (y bf16 bits [R, N], exact product float64 [R, N], mag float64 [R, N] =
+    sum_k |x[r, k]| |w[n, k]|, the scale of any lower-precision summation's
+    error)."""
+    X, W = _widen64(x), _widen64(w)
+    exact = X @ W.T
+    mag = np.abs(X) @ np.abs(W).T
+    y = round_bf16(exact)
+    if residual is not None:
+        y = round_bf16(_widen64(residual) + _widen64(y))
+    return y, exact, mag
+
+
 def consensus(draft, verify):
     """(accept_len [B], n_emit [B], emitted [B, blk] (-1 padded), next_anchor [B])."""
     d = np.ascontiguousarray(draft, dtype=np.int32)

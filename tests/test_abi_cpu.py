@@ -340,3 +340,43 @@ def test_tensor_core_attention_plan(L):
     # at most 4 of the 65 tiles each, merged inside the launch
     assert L.orthrus_block_attn_plan(ctypes.byref(a), 148, out) == 0
     assert list(out)[:4] == [18, 18, 8, 1] and out[6] == 4 and out[7] == 1
+
+
+def test_linear_tc_plan_and_rejections(L):
+    """Launch plan of the tensor-core projection over a sweep: tiles of 128
+    features, K splits that fill the SMs without exceeding 16 or the K steps,
+    at least two ring stages within the shared memory a CTA may use, TMEM
+    columns a power of two holding the rows; and the host-side rejections."""
+    out = (ctypes.c_int32 * 8)()
+    for rows in (1, 16, 17, 32, 100, 128):
+        for K in (64, 640, 4096):
+            for N in (1, 128, 300, 4096, 6144, 151936):
+                for sms in (132, 148, 160):
+                    key = (rows, K, N, sms)
+                    assert L.orthrus_linear_tc_plan(rows, K, N, sms, out) == 0, key
+                    tiles, ksplit, stages, sb, smem, grid, tcols, rp = list(out)
+                    assert tiles == -(-N // 128) and grid == tiles * ksplit, key
+                    assert 1 <= ksplit <= min(16, K // 64), key
+                    assert tiles * ksplit <= max(sms, tiles), key
+                    assert stages >= 2 and smem <= 227 * 1024, key
+                    assert rp == -(-rows // 16) * 16 and sb >= 128 * 128 + rp * 128, key
+                    assert tcols >= rp and tcols & (tcols - 1) == 0 and tcols <= 512, key
+                    assert L.orthrus_linear_tc_workspace(rows, K, N) >= tiles * 4, key
+    assert L.orthrus_linear_tc_plan(129, 64, 128, 148, out) == -1
+    assert L.orthrus_linear_tc_plan(32, 100, 128, 148, out) == -1
+    vp = ctypes.c_void_p
+    ws = L.orthrus_linear_tc_workspace(32, 4096, 6144)
+    call = lambda dtype=1, x=256, rows=32, K=4096, ldx=4096, w=512, N=6144, y=1024, ldy=6144, \
+        wsp=2048, wsb=ws: L.orthrus_linear_tc(dtype, vp(x) if x else None, rows, K, ldx,
+                                              vp(w) if w else None, N, None, vp(y) if y else None,
+                                              ldy, None, vp(wsp) if wsp else None, wsb, None)
+    assert call(dtype=0) == -2           # fp32: unsupported
+    assert call(dtype=5) == -1
+    assert call(rows=0) == 0             # nothing to do
+    assert call(rows=129) == -2
+    assert call(K=100, ldx=100) == -2    # K not a multiple of 64
+    assert call(ldx=4100) == -2          # row pitch not 16-byte aligned
+    assert call(ldx=10) == -1            # pitch below K
+    assert call(x=0) == -1 and call(w=0) == -1 and call(y=0) == -1
+    assert call(x=264) == -1             # x not 16-byte aligned
+    assert call(wsp=0) == -3 and call(wsb=ws - 1) == -3 and call(wsp=2056) == -3
