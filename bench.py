@@ -349,6 +349,46 @@ def lm_head_leg(dev, steps=10, warmup=3):
             "peak": hbm, "peak_source": src, **out}
 
 
+def projection_kernels(args):
+    """The attention block's projections alone at the Qwen3-8B shape: a
+    32-row block through the QKV (4096 -> 6144) and output (4096 -> 4096)
+    weights of 36 layers in turn (beyond the L2), `steps` graph replays."""
+    import torch
+    import block_attention_b200 as ba
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(1010)
+    L, blk, d = WORKLOAD["layers"], WORKLOAD["blk"], 4096
+    hbm, src = peaks()
+    res = {}
+    for name, N in (("qkv_projection", 6144), ("output_projection", 4096)):
+        W = (torch.randn(L, N, d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        x = torch.randn(blk, d, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(blk, N, dtype=torch.bfloat16, device=dev)
+        ws = ba.Workspace(dev)
+        seq = lambda: [ba.linear_tc(x, W[l], out=y, workspace=ws) for l in range(L)]
+        for _ in range(args.warmup):
+            seq()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            seq()
+        gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (args.steps * L)
+        nbytes = N * d * 2 + blk * (d + N) * 2
+        res[name] = {"us_per_call": us, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / hbm}
+        del gr, W
+    print(json.dumps({"kernel": "linear_tc", "case": f"{blk} rows, Qwen3-8B projections, "
+                      f"{L} layers' weights in turn", "peak": hbm, "peak_source": src, **res}),
+          flush=True)
+
+
 def lm_head_kernel(args):
     import torch
     print(json.dumps(lm_head_leg(torch.device("cuda", 0), args.steps, args.warmup)), flush=True)
@@ -796,11 +836,12 @@ def main():
     ap.add_argument("--attn-batch", type=int, default=8,
                     help="sequences of the --kernel attn case (8: larger than L2; 1: the "
                          "round's call)")
-    ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead"], default=None,
+    ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead", "proj"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
                          "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
                          "the stochastic round's kernels one at a time; lmhead: the LM head "
-                         "with the argmax in its epilogue against GEMM + argmax")
+                         "with the argmax in its epilogue against GEMM + argmax; proj: the "
+                         "attention block's projections alone")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel == "attn":
@@ -811,6 +852,8 @@ def main():
         return sampling_kernels(args)
     if args.kernel == "lmhead":
         return lm_head_kernel(args)
+    if args.kernel == "proj":
+        return projection_kernels(args)
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

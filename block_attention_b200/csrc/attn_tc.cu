@@ -162,6 +162,15 @@ __device__ __forceinline__ void record_timeout(int32_t* err, volatile int* abort
   set_err(err, ORTHRUS_ETIMEOUT);
 }
 
+// 64 S values of keys [k0, k0 + 64) of a tile: those at or past nv -> -inf
+__device__ __forceinline__ void mask_keys(uint32_t (&sv)[2][32], int k0, int nv) {
+#pragma unroll
+  for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (k0 + 32 * cb + j >= nv) sv[cb][j] = __float_as_uint(-INFINITY);
+}
+
 template <int kD>
 __device__ __forceinline__ void merge_rows(const TcParams& p, int b, int g, int q, int tid,
                                            int nthreads, uint8_t* stage, uint32_t bar);
@@ -438,31 +447,28 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
         record_timeout(p.err, abort_flag); alive = false; break;
       }
       ptx::tc_fence_after();
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) ptx::tmem_ld32(lane_addr + X * kTile + cb * 32, sv[cb]);
-      ptx::tmem_wait_ld();
-      // S(u) is in registers: its TMEM buffer may take S(u + 2)
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bars.s_free(X));
       const bool blk_tile = t == Tc;
       const int nv_tile = blk_tile ? p.blk : min(kTile, n - t * kTile);
       int nv = nv_tile;
       if (blk_tile && p.mask_mode == ORTHRUS_CAUSAL_VERIFY) nv = min(i_blk + 1, p.blk);
-      // masked keys -> -inf before the max and the exponent (exactly 0 in P)
-      if (nv < kTile) {
+      const uint32_t s_addr = lane_addr + X * kTile;
+      // S(u) is read from TMEM twice, 64 columns at a time -- once for the row
+      // maximum, once for the exponentials -- so that no more than 64 of its
+      // values are live in registers; masked keys -> -inf (exactly 0 in P)
+      float mt[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb)
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[2][32];
+        ptx::tmem_ld32(s_addr + 64 * half, sv[0]);
+        ptx::tmem_ld32(s_addr + 64 * half + 32, sv[1]);
+        ptx::tmem_wait_ld();
+        if (nv < kTile) mask_keys(sv, 64 * half, nv);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (cb * 32 + j >= nv) sv[cb][j] = __float_as_uint(-INFINITY);
+        for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mt[cb] = fmaxf(mt[cb], __uint_as_float(sv[cb][j]));
       }
-      float mt[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mt[cb] = fmaxf(mt[cb], __uint_as_float(sv[cb][j]));
-      const float ms = fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3])) * c;
+      const float ms = fmaxf(mt[0], mt[1]) * c;
       const bool need = ms > m_ref + kLazyThresh;
       const bool rescale = __any_sync(full_mask, need);
       float f = 1.f;
@@ -487,12 +493,21 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       uint8_t* prow = smem + kPOff + X * kPBytes + r * 128;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
+        uint32_t sv[2][32];
+        ptx::tmem_ld32(s_addr + 64 * half, sv[0]);
+        ptx::tmem_ld32(s_addr + 64 * half + 32, sv[1]);
+        ptx::tmem_wait_ld();
+        if (half == 1) {  // S(u) is read: its TMEM buffer may take S(u + 2)
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bars.s_free(X));
+        }
+        if (nv < kTile) mask_keys(sv, 64 * half, nv);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {  // 8 keys: 64 half + 8 ch .. + 7
           uint32_t w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int k0 = 64 * half + 8 * ch + 2 * e;  // key of the pair's low half
+            const int k0 = 8 * ch + 2 * e;  // key of the pair's low half within the half
             const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[k0 >> 5][k0 & 31]), c, nm));
             const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[k0 >> 5][(k0 & 31) + 1]), c, nm));
             ls[e] += p0 + p1;

@@ -58,6 +58,7 @@ struct __align__(64) LinParams {
   unsigned* tickets;              // [tiles], zero between calls
   int32_t* err;
   int R, Rp, N, ldy, tiles, ksplit, ksteps, stages, stage_bytes, tmem_cols;
+  int kb;  // 64-wide K steps (weight box + x box each) per stage
 };
 
 struct Bars {
@@ -101,9 +102,14 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
 
   const int tile = blockIdx.x / p.ksplit, ks = blockIdx.x % p.ksplit;
   const int k_beg = (int)((int64_t)ks * p.ksteps / p.ksplit);
-  const int nk = (int)((int64_t)(ks + 1) * p.ksteps / p.ksplit) - k_beg;
+  const int nsteps = (int)((int64_t)(ks + 1) * p.ksteps / p.ksplit) - k_beg;
+  const int KB = p.kb;
+  const int nk = ceil_div(nsteps, KB);  // stages this CTA streams (the last may be short)
   const int n0 = tile * kTileN;
   const uint32_t x_bytes = (uint32_t)(p.Rp * 128);
+  const uint32_t x_off = (uint32_t)(KB * kWBox);  // the x boxes follow the stage's weight boxes
+  // K steps of stage i: [k_beg + i KB, k_beg + min(nsteps, (i + 1) KB))
+  auto steps_of = [&](int i) { return min(KB, nsteps - i * KB); };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -135,9 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
   const int early = min(nk, ST);
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < early; ++i) {
-      ptx::mbar_expect_tx(bars.full(i), (uint32_t)kWBox + x_bytes);
-      ptx::tma_load_2d(sbase + (uint32_t)(i * SB), &p.tm_w, bars.full(i), (k_beg + i) * kStepK,
-                       n0);
+      const int ns = steps_of(i);
+      ptx::mbar_expect_tx(bars.full(i), (uint32_t)ns * ((uint32_t)kWBox + x_bytes));
+      for (int j = 0; j < ns; ++j)
+        ptx::tma_load_2d(sbase + (uint32_t)(i * SB + j * kWBox), &p.tm_w, bars.full(i),
+                         (k_beg + i * KB + j) * kStepK, n0);
     }
   }
   ptx::griddep_wait();
@@ -148,20 +156,25 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
       // the x boxes of the early stages first: with them every stage whose
       // weights are in flight can complete
       for (int i = 0; i < early; ++i)
-        ptx::tma_load_2d(sbase + (uint32_t)(i * SB + kWBox), &p.tm_x, bars.full(i),
-                         (k_beg + i) * kStepK, 0);
+        for (int j = 0; j < steps_of(i); ++j)
+          ptx::tma_load_2d(sbase + (uint32_t)(i * SB) + x_off + (uint32_t)(j * x_bytes), &p.tm_x,
+                           bars.full(i), (k_beg + i * KB + j) * kStepK, 0);
       int issued = early;
       for (int i = early; i < nk; ++i) {
         if (*abort_flag) break;
-        const int s = i % ST;
+        const int s = i % ST, ns = steps_of(i);
         const uint32_t dst = sbase + (uint32_t)(s * SB);
         if (!ptx::mbar_wait(bars.empty(s), ((i / ST) & 1) ^ 1)) {
           record_timeout(p.err, abort_flag);
           break;
         }
-        ptx::mbar_expect_tx(bars.full(s), (uint32_t)kWBox + x_bytes);
-        ptx::tma_load_2d(dst, &p.tm_w, bars.full(s), (k_beg + i) * kStepK, n0);
-        ptx::tma_load_2d(dst + kWBox, &p.tm_x, bars.full(s), (k_beg + i) * kStepK, 0);
+        ptx::mbar_expect_tx(bars.full(s), (uint32_t)ns * ((uint32_t)kWBox + x_bytes));
+        for (int j = 0; j < ns; ++j) {
+          ptx::tma_load_2d(dst + (uint32_t)(j * kWBox), &p.tm_w, bars.full(s),
+                           (k_beg + i * KB + j) * kStepK, n0);
+          ptx::tma_load_2d(dst + x_off + (uint32_t)(j * x_bytes), &p.tm_x, bars.full(s),
+                           (k_beg + i * KB + j) * kStepK, 0);
+        }
         issued = i + 1;
       }
       // every issued load lands before the CTA can exit
@@ -181,11 +194,13 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
         }
         ptx::tc_fence_after();
         const uint32_t wa = sbase + (uint32_t)(s * SB);
+        for (int j = 0; j < steps_of(i); ++j) {
 #pragma unroll
-        for (int kk = 0; kk < kStepK / 16; ++kk)
-          ptx::mma_ss(tmem, ptx::sdesc_sw128(wa + kk * 32, 16, 1024),
-                      ptx::sdesc_sw128(wa + kWBox + kk * 32, 16, 1024), id,
-                      (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kStepK / 16; ++kk)
+            ptx::mma_ss(tmem, ptx::sdesc_sw128(wa + j * kWBox + kk * 32, 16, 1024),
+                        ptx::sdesc_sw128(wa + x_off + j * x_bytes + kk * 32, 16, 1024), id,
+                        (i > 0 || j > 0 || kk > 0) ? 1u : 0u);
+        }
         ptx::tc_commit(bars.empty(s));
       }
       if (!ok) record_timeout(p.err, abort_flag);
@@ -323,18 +338,22 @@ int sm_count() {
 }
 
 struct Plan {
-  int Rp, tiles, ksplit, ksteps, stages, stage_bytes, smem, tmem_cols;
+  int Rp, tiles, ksplit, ksteps, stages, stage_bytes, smem, tmem_cols, kb;
 };
 
 // Launch shape for rows x K x N on `sms` SMs: 128-feature tiles, the K range
 // of each split over enough CTAs to fill the SMs (at most one 64-wide K step
 // less than an even share each), a ring of as many stages as fit.
-Plan plan(int rows, int K, int N, int sms) {
+Plan plan(int rows, int K, int N, int sms, int kb) {
   Plan q;
   q.Rp = (rows + 15) / 16 * 16;
   q.ksteps = K / kStepK;
   q.tiles = ceil_div(N, kTileN);
-  q.stage_bytes = kWBox + (q.Rp * 128 + 1023) / 1024 * 1024;
+  // kb K steps per stage: their weight boxes, then their x boxes (each x box
+  // Rp rows of 128 bytes; kb * Rp * 128 rounded up to 1 KB keeps every box
+  // of the next stage 1 KB aligned for the 128-byte swizzle)
+  q.kb = kb;
+  q.stage_bytes = kb * kWBox + (kb * q.Rp * 128 + 1023) / 1024 * 1024;
   q.stages = min(kMaxStages, kRingBudget / q.stage_bytes);
   // splits: enough to fill the SMs, at most one per K step, at most 16, and
   // no more than the ring can stage for the last CTA's sum
@@ -346,6 +365,17 @@ Plan plan(int rows, int K, int N, int sms) {
   while (q.tmem_cols < q.Rp) q.tmem_cols *= 2;
   return q;
 }
+
+// The most K steps per stage (up to kMaxKb) that still leave two stages.
+constexpr int kMaxKb = 4;
+int choose_kb(int rows) {
+  const int Rp = (rows + 15) / 16 * 16;
+  for (int kb = kMaxKb; kb > 1; kb /= 2)
+    if (kRingBudget / (kb * kWBox + (kb * Rp * 128 + 1023) / 1024 * 1024) >= 2) return kb;
+  return 1;
+}
+
+Plan plan(int rows, int K, int N, int sms) { return plan(rows, K, N, sms, choose_kb(rows)); }
 
 size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
 
@@ -427,7 +457,7 @@ int orthrus_linear_tc(int32_t dtype, const void* x, int32_t rows, int32_t K, int
   p.err = err;
   p.R = rows; p.Rp = q.Rp; p.N = N; p.ldy = (int)ldy;
   p.tiles = q.tiles; p.ksplit = q.ksplit; p.ksteps = q.ksteps; p.stages = q.stages;
-  p.stage_bytes = q.stage_bytes; p.tmem_cols = q.tmem_cols;
+  p.stage_bytes = q.stage_bytes; p.tmem_cols = q.tmem_cols; p.kb = q.kb;
 
   cudaLaunchAttribute pdl;
   pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
