@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "orthrus_decoder.h"
+#include "tc_ptx.cuh"
 
 namespace orthrus {
 namespace {
@@ -32,45 +33,177 @@ template <typename T> __device__ __forceinline__ float rnd(float x) {
   return round_to(x, static_cast<T*>(nullptr));
 }
 
+// ------------------------------------------------ 16-byte chunk helpers
+// A row is read and written in 16-byte chunks of kW<T> elements; chunk c of a
+// row is elements c*kW .. c*kW+kW-1.  kVec: the row is 16-byte aligned and a
+// whole number of chunks (one vector access per chunk); otherwise element by
+// element, elements past the row's end reading as zero.
+template <typename T> constexpr int kW = 16 / sizeof(T);
+
+template <typename T, bool kVec>
+__device__ __forceinline__ void load_chunk(const T* row, int c, int n, float (&v)[kW<T>]) {
+  if (kVec) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row + c * kW<T>);
+    if constexpr (sizeof(T) == 4) {
+      v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+      v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+    } else {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kW<T>; ++i) {
+      const int e = c * kW<T> + i;
+      v[i] = e < n ? to_f32(row[e]) : 0.f;
+    }
+  }
+}
+
+template <typename T, bool kVec>
+__device__ __forceinline__ void store_chunk(T* row, int c, int n, const float (&v)[kW<T>]) {
+  if (kVec) {
+    uint4 u;
+    if constexpr (sizeof(T) == 4) {
+      u = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                     __float_as_uint(v[3]));
+    } else {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      u = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *reinterpret_cast<uint4*>(row + c * kW<T>) = u;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kW<T>; ++i) {
+      const int e = c * kW<T> + i;
+      if (e < n) row[e] = from_f32<T>(v[i]);
+    }
+  }
+}
+
+// Launch with programmatic stream serialization: the grid may start while
+// the preceding kernel finishes; each of these kernels lets its own
+// dependents start at once and waits for its predecessor before reading.
+template <typename... KA, typename... A>
+cudaError_t launch_pdl(void (*kernel)(KA...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, A... args) {
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KA>(args)...);
+}
+
+__device__ __forceinline__ void pdl_enter() {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
+}
+
 // ------------------------------------------------------------------ embed
-template <typename T>
+template <typename T, bool kVec>
 __global__ void __launch_bounds__(128)
 embed_kernel(const T* __restrict__ table, int V, int d, const int32_t* __restrict__ tokens,
              T* __restrict__ out, int32_t* err) {
+  pdl_enter();
   const int r = blockIdx.x;
   const int tok = tokens[r];
   const bool ok = tok >= 0 && tok < V;
   if (!ok && threadIdx.x == 0) set_err(err, ORTHRUS_EINVAL);
   const T* src = table + (int64_t)(ok ? tok : 0) * d;
   T* dst = out + (int64_t)r * d;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) dst[i] = ok ? src[i] : from_f32<T>(0.f);
+  for (int c = threadIdx.x; c < ceil_div(d, kW<T>); c += blockDim.x) {
+    float v[kW<T>];
+    load_chunk<T, kVec>(src, c, d, v);
+    if (!ok) {
+#pragma unroll
+      for (int i = 0; i < kW<T>; ++i) v[i] = 0.f;
+    }
+    store_chunk<T, kVec>(dst, c, d, v);
+  }
 }
 
 // ---------------------------------------------------------------- RMSNorm
-// One warp per row.  Lane l sums x[i]^2 for i = l, l+32, ... in order, then
-// the 32 partial sums meet in a fixed xor butterfly.
-constexpr int kNormRowsPerCta = 4;
+// One CTA per row.  Chunk c of the row belongs to thread c % kNormThreads;
+// each thread sums the squares of its chunks in order (chunk by chunk,
+// element by element), then the threads' sums meet in a fixed xor butterfly
+// within each warp and in warp order across warps.  The order depends on d
+// alone, so a row's result does not depend on the other rows of the call.
+// kChunks > 0: the thread's chunks stay in registers between the two
+// passes; kChunks == 0: the row is read again for the output.
+constexpr int kNormThreads = 256;
 
-template <typename T>
-__global__ void __launch_bounds__(32 * kNormRowsPerCta)
-rmsnorm_kernel(const T* x, const T* __restrict__ gain, int rows, int d, float eps, T* out) {
-  const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kNormRowsPerCta + (threadIdx.x >> 5);
-  if (r >= rows) return;
-  const T* xr = x + (int64_t)r * d;
-  T* yr = out + (int64_t)r * d;
+template <typename T, bool kVec, int kChunks>
+__global__ void __launch_bounds__(kNormThreads)
+rmsnorm_kernel(const T* x, const T* __restrict__ gain, int d, float eps, T* out) {
+  pdl_enter();
+  const T* xr = x + (int64_t)blockIdx.x * d;
+  T* yr = out + (int64_t)blockIdx.x * d;
+  const int nch = ceil_div(d, kW<T>);
+  constexpr int kC = kChunks > 0 ? kChunks : 1;
+  float v[kC][kW<T>];
   float ss = 0.f;
-  for (int i = lane; i < d; i += 32) {
-    const float v = to_f32(xr[i]);
-    ss = fmaf(v, v, ss);
+  if (kChunks > 0) {
+#pragma unroll
+    for (int k = 0; k < kC; ++k) {
+      const int c = threadIdx.x + k * kNormThreads;
+      if (c < nch) load_chunk<T, kVec>(xr, c, d, v[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kC; ++k) {
+      if (threadIdx.x + k * kNormThreads < nch) {
+#pragma unroll
+        for (int i = 0; i < kW<T>; ++i) ss = fmaf(v[k][i], v[k][i], ss);
+      }
+    }
+  } else {
+    for (int c = threadIdx.x; c < nch; c += kNormThreads) {
+      load_chunk<T, kVec>(xr, c, d, v[0]);
+#pragma unroll
+      for (int i = 0; i < kW<T>; ++i) ss = fmaf(v[0][i], v[0][i], ss);
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  __shared__ float warp_ss[kNormThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_ss[threadIdx.x >> 5] = ss;
+  __syncthreads();  // also: every thread has read its x before any writes (out may alias x)
+  ss = 0.f;
+#pragma unroll
+  for (int w = 0; w < kNormThreads / 32; ++w) ss += warp_ss[w];
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
-  __syncwarp();  // every lane has read its x before any lane writes (out may alias x)
-  for (int i = lane; i < d; i += 32) {
-    const float y = rnd<T>(to_f32(xr[i]) * inv);
-    yr[i] = from_f32<T>(y * to_f32(gain[i]));
+  auto emit = [&](int c, float (&xv)[kW<T>]) {
+    float g[kW<T>];
+    load_chunk<T, kVec>(gain, c, d, g);
+#pragma unroll
+    for (int i = 0; i < kW<T>; ++i) xv[i] = rnd<T>(xv[i] * inv) * g[i];
+    store_chunk<T, kVec>(yr, c, d, xv);
+  };
+  if (kChunks > 0) {
+#pragma unroll
+    for (int k = 0; k < kC; ++k) {
+      const int c = threadIdx.x + k * kNormThreads;
+      if (c < nch) emit(c, v[k]);
+    }
+  } else {
+    for (int c = threadIdx.x; c < nch; c += kNormThreads) {
+      load_chunk<T, kVec>(xr, c, d, v[0]);
+      emit(c, v[0]);
+    }
   }
 }
 
@@ -170,38 +303,94 @@ linear_kernel(const T* __restrict__ X, const T* __restrict__ W, const T* R, T* Y
 }
 
 // --------------------------------------------------------- q/k/v + RoPE
-template <typename T>
-__global__ void __launch_bounds__(128)
+// One CTA per block row.  Rotation pairs (x[i], x[i + hd/2]) of a head at the
+// row's absolute position: the angle pos * theta^(-2i/hd) and its cosine and
+// sine in double, once per row into shared memory; the rotation itself in
+// float.  Work units: a 16-byte chunk of x[i..] together with the matching
+// chunk of x[i + hd/2] (q and k heads), and 16-byte chunks of v (copied).
+// kVec: hd/2 is a whole number of chunks and every row is 16-byte aligned;
+// otherwise a unit is a single pair or a single element.  Each thread reads
+// all of its units before the table is built, so the loads of a row are in
+// flight together.
+constexpr int kRopeThreads = 256;
+constexpr int kRopeUnits = 4;  // units per thread held in registers per batch
+
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kRopeThreads)
 qkv_rope_kernel(const T* __restrict__ qkv, int blk, int Hq, int Hkv, int hd,
                 const int32_t* __restrict__ ctx_lens, double theta, T* __restrict__ q,
                 T* __restrict__ k, T* __restrict__ v) {
   extern __shared__ float cs[];  // [hd/2] cos, then [hd/2] sin
+  pdl_enter();
+  constexpr int W = kVec ? kW<T> : 1;
   const int r = blockIdx.x, b = r / blk, j = r % blk;
-  const int half = hd / 2;
-  const int64_t pos = (int64_t)ctx_lens[b] + j;
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double ang = (double)pos * pow(theta, -2.0 * i / hd);
-    double s, c;
-    sincos(ang, &s, &c);
-    cs[i] = (float)c;
-    cs[half + i] = (float)s;
-  }
-  __syncthreads();
+  const int half = hd / 2, hc = half / W;  // chunks per half head
   const int width = (Hq + 2 * Hkv) * hd;
   const T* src = qkv + (int64_t)r * width;
-  const int pairs = (Hq + Hkv) * half;
-  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
-    const int h = p / half, i = p % half;
-    const float c = cs[i], s = cs[half + i];
-    const float x1 = to_f32(src[h * hd + i]), x2 = to_f32(src[h * hd + i + half]);
-    const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
-    T* dst = h < Hq ? q + ((int64_t)r * Hq + h) * hd : k + ((int64_t)r * Hkv + h - Hq) * hd;
-    dst[i] = from_f32<T>(y1);
-    dst[i + half] = from_f32<T>(y2);
+  const int rot_units = (Hq + Hkv) * hc, copy_units = Hkv * hd / W;
+  const int units = rot_units + copy_units;
+  const int64_t pos = (int64_t)ctx_lens[b] + j;
+  bool table = false;
+  for (int base = 0; base < units; base += kRopeThreads * kRopeUnits) {
+    float a[kRopeUnits][W], c2[kRopeUnits][W];
+#pragma unroll
+    for (int u = 0; u < kRopeUnits; ++u) {
+      const int id = base + u * kRopeThreads + threadIdx.x;
+      if (id < rot_units) {
+        const int h = id / hc, i0 = (id % hc) * W;
+        if constexpr (kVec) {
+          load_chunk<T, true>(src + h * hd, i0 / W, hd, a[u]);
+          load_chunk<T, true>(src + h * hd + half, i0 / W, hd, c2[u]);
+        } else {
+          a[u][0] = to_f32(src[h * hd + i0]);
+          c2[u][0] = to_f32(src[h * hd + half + i0]);
+        }
+      } else if (id < units) {
+        const int e0 = (id - rot_units) * W;
+        if constexpr (kVec) load_chunk<T, true>(src + (Hq + Hkv) * hd, e0 / W, Hkv * hd, a[u]);
+        else a[u][0] = to_f32(src[(Hq + Hkv) * hd + e0]);
+      }
+    }
+    if (!table) {
+      for (int i = threadIdx.x; i < half; i += kRopeThreads) {
+        const double ang = (double)pos * pow(theta, -2.0 * i / hd);
+        double sn, cn;
+        sincos(ang, &sn, &cn);
+        cs[i] = (float)cn;
+        cs[half + i] = (float)sn;
+      }
+      __syncthreads();
+      table = true;
+    }
+#pragma unroll
+    for (int u = 0; u < kRopeUnits; ++u) {
+      const int id = base + u * kRopeThreads + threadIdx.x;
+      if (id < rot_units) {
+        const int h = id / hc, i0 = (id % hc) * W;
+        float y1[W], y2[W];
+#pragma unroll
+        for (int e = 0; e < W; ++e) {
+          const float c = cs[i0 + e], s = cs[half + i0 + e];
+          const float x1 = a[u][e], x2 = c2[u][e];
+          y1[e] = x1 * c - x2 * s;
+          y2[e] = x2 * c + x1 * s;
+        }
+        T* dst = h < Hq ? q + ((int64_t)r * Hq + h) * hd : k + ((int64_t)r * Hkv + h - Hq) * hd;
+        if constexpr (kVec) {
+          store_chunk<T, true>(dst, i0 / W, hd, y1);
+          store_chunk<T, true>(dst + half, i0 / W, hd, y2);
+        } else {
+          dst[i0] = from_f32<T>(y1[0]);
+          dst[half + i0] = from_f32<T>(y2[0]);
+        }
+      } else if (id < units) {
+        const int e0 = (id - rot_units) * W;
+        T* vd = v + (int64_t)r * Hkv * hd;
+        if constexpr (kVec) store_chunk<T, true>(vd, e0 / W, Hkv * hd, a[u]);
+        else vd[e0] = from_f32<T>(a[u][0]);
+      }
+    }
   }
-  const T* vs = src + (Hq + Hkv) * hd;
-  T* vd = v + (int64_t)r * Hkv * hd;
-  for (int e = threadIdx.x; e < Hkv * hd; e += blockDim.x) vd[e] = vs[e];
 }
 
 // ----------------------------------------------------------------- SwiGLU
@@ -227,6 +416,19 @@ block_tokens_kernel(const int32_t* __restrict__ anchor, const int32_t* __restric
       j == 0 ? anchor[b] : (draft ? draft[(int64_t)b * blk + j - 1] : mask_id);
 }
 
+template <typename T, bool kVec>
+cudaError_t launch_rmsnorm(const T* x, const T* gain, int rows, int d, float eps, T* out,
+                           cudaStream_t st) {
+  const int per_thread = ceil_div(ceil_div(d, kW<T>), kNormThreads);
+  auto go = [&](auto kernel) {
+    return launch_pdl(kernel, rows, kNormThreads, 0, st, x, gain, d, eps, out);
+  };
+  if (per_thread <= 1) return go(rmsnorm_kernel<T, kVec, 1>);
+  if (per_thread <= 2) return go(rmsnorm_kernel<T, kVec, 2>);
+  if (per_thread <= 4) return go(rmsnorm_kernel<T, kVec, 4>);
+  return go(rmsnorm_kernel<T, kVec, 0>);
+}
+
 }  // namespace
 }  // namespace orthrus
 
@@ -241,14 +443,22 @@ int orthrus_embed(int32_t dtype, const void* table, int32_t V, int32_t d,
   if (rows == 0) return ORTHRUS_OK;
   if (!table || !tokens || !out) return ORTHRUS_EINVAL;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == ORTHRUS_F32)
-    embed_kernel<float><<<rows, 128, 0, st>>>(static_cast<const float*>(table), V, d, tokens,
-                                              static_cast<float*>(out), err);
-  else
-    embed_kernel<__nv_bfloat16><<<rows, 128, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(table), V, d, tokens,
-        static_cast<__nv_bfloat16*>(out), err);
-  return status(cudaGetLastError());
+  const bool vec = (d * esize(dtype)) % 16 == 0 && aligned_to(table, 16) && aligned_to(out, 16);
+  cudaError_t e;
+  if (dtype == ORTHRUS_F32) {
+    auto t = static_cast<const float*>(table);
+    auto o = static_cast<float*>(out);
+    e = vec ? launch_pdl(embed_kernel<float, true>, rows, 128, 0, st, t, V, d, tokens, o, err)
+            : launch_pdl(embed_kernel<float, false>, rows, 128, 0, st, t, V, d, tokens, o, err);
+  } else {
+    auto t = static_cast<const __nv_bfloat16*>(table);
+    auto o = static_cast<__nv_bfloat16*>(out);
+    e = vec ? launch_pdl(embed_kernel<__nv_bfloat16, true>, rows, 128, 0, st, t, V, d, tokens,
+                         o, err)
+            : launch_pdl(embed_kernel<__nv_bfloat16, false>, rows, 128, 0, st, t, V, d, tokens,
+                         o, err);
+  }
+  return status(e);
 }
 
 int orthrus_rmsnorm(int32_t dtype, const void* x, const void* gain, int32_t rows, int32_t d,
@@ -257,16 +467,21 @@ int orthrus_rmsnorm(int32_t dtype, const void* x, const void* gain, int32_t rows
   if (rows == 0) return ORTHRUS_OK;
   if (!x || !gain || !out) return ORTHRUS_EINVAL;
   auto st = reinterpret_cast<cudaStream_t>(stream);
-  const int grid = ceil_div(rows, kNormRowsPerCta);
-  if (dtype == ORTHRUS_F32)
-    rmsnorm_kernel<float><<<grid, 32 * kNormRowsPerCta, 0, st>>>(
-        static_cast<const float*>(x), static_cast<const float*>(gain), rows, d, eps,
-        static_cast<float*>(out));
-  else
-    rmsnorm_kernel<__nv_bfloat16><<<grid, 32 * kNormRowsPerCta, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gain), rows,
-        d, eps, static_cast<__nv_bfloat16*>(out));
-  return status(cudaGetLastError());
+  const bool vec = (d * esize(dtype)) % 16 == 0 && aligned_to(x, 16) && aligned_to(gain, 16) &&
+                   aligned_to(out, 16);
+  cudaError_t e;
+  if (dtype == ORTHRUS_F32) {
+    auto X = static_cast<const float*>(x), G = static_cast<const float*>(gain);
+    auto Y = static_cast<float*>(out);
+    e = vec ? launch_rmsnorm<float, true>(X, G, rows, d, eps, Y, st)
+            : launch_rmsnorm<float, false>(X, G, rows, d, eps, Y, st);
+  } else {
+    auto X = static_cast<const __nv_bfloat16*>(x), G = static_cast<const __nv_bfloat16*>(gain);
+    auto Y = static_cast<__nv_bfloat16*>(out);
+    e = vec ? launch_rmsnorm<__nv_bfloat16, true>(X, G, rows, d, eps, Y, st)
+            : launch_rmsnorm<__nv_bfloat16, false>(X, G, rows, d, eps, Y, st);
+  }
+  return status(e);
 }
 
 int orthrus_linear(int32_t dtype, const void* x, const void* w, const void* residual,
@@ -311,16 +526,28 @@ int orthrus_qkv_rope(int32_t dtype, const void* qkv, int32_t B, int32_t blk, int
   if (rows > 2147483647LL) return ORTHRUS_EUNSUPPORTED;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   const size_t smem = sizeof(float) * hd;
-  if (dtype == ORTHRUS_F32)
-    qkv_rope_kernel<float><<<(unsigned)rows, 128, smem, st>>>(
-        static_cast<const float*>(qkv), blk, Hq, Hkv, hd, ctx_lens, theta,
-        static_cast<float*>(q), static_cast<float*>(k), static_cast<float*>(v));
-  else
-    qkv_rope_kernel<__nv_bfloat16><<<(unsigned)rows, 128, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(qkv), blk, Hq, Hkv, hd, ctx_lens, theta,
-        static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
-        static_cast<__nv_bfloat16*>(v));
-  return status(cudaGetLastError());
+  const size_t es = esize(dtype);
+  const bool vec = (hd / 2) % (16 / es) == 0 && aligned_to(qkv, 16) && aligned_to(q, 16) &&
+                   aligned_to(k, 16) && aligned_to(v, 16);
+  cudaError_t e;
+  const unsigned g = (unsigned)rows;
+  if (dtype == ORTHRUS_F32) {
+    auto src = static_cast<const float*>(qkv);
+    auto Q = static_cast<float*>(q), K = static_cast<float*>(k), Vv = static_cast<float*>(v);
+    e = vec ? launch_pdl(qkv_rope_kernel<float, true>, g, kRopeThreads, smem, st, src, blk, Hq,
+                         Hkv, hd, ctx_lens, theta, Q, K, Vv)
+            : launch_pdl(qkv_rope_kernel<float, false>, g, kRopeThreads, smem, st, src, blk,
+                         Hq, Hkv, hd, ctx_lens, theta, Q, K, Vv);
+  } else {
+    auto src = static_cast<const __nv_bfloat16*>(qkv);
+    auto Q = static_cast<__nv_bfloat16*>(q), K = static_cast<__nv_bfloat16*>(k),
+         Vv = static_cast<__nv_bfloat16*>(v);
+    e = vec ? launch_pdl(qkv_rope_kernel<__nv_bfloat16, true>, g, kRopeThreads, smem, st, src,
+                         blk, Hq, Hkv, hd, ctx_lens, theta, Q, K, Vv)
+            : launch_pdl(qkv_rope_kernel<__nv_bfloat16, false>, g, kRopeThreads, smem, st, src,
+                         blk, Hq, Hkv, hd, ctx_lens, theta, Q, K, Vv);
+  }
+  return status(e);
 }
 
 int orthrus_swiglu(int32_t dtype, const void* gu, int32_t rows, int32_t F, void* out,
