@@ -54,7 +54,7 @@ struct __align__(64) LinParams {
   CUtensorMap tm_x;  // 2D (K, R), row pitch ldx, box (64, Rp); rows past R read as zero
   const __nv_bfloat16* residual;  // [R] rows of pitch ldy, or null
   __nv_bfloat16* y;               // [R] rows of pitch ldy
-  float* part;                    // [tiles][ksplit][Rp][128] fp32 split-K partials
+  float* part;                    // [tiles][ksplit][128][Rp + 4] fp32 split-K partials
   unsigned* tickets;              // [tiles], zero between calls
   int32_t* err;
   int R, Rp, N, ldy, tiles, ksplit, ksteps, stages, stage_bytes, tmem_cols;
@@ -79,34 +79,89 @@ __device__ __forceinline__ float bf16_round(float v) {
   return __uint_as_float(ptx::pack_bf16x2(v, 0.f) << 16);
 }
 
-// out = bf16(sum) or bf16(residual + bf16(sum))
-__device__ __forceinline__ __nv_bfloat16 finish(float sum, const __nv_bfloat16* res) {
-  float v = bf16_round(sum);
-  if (res) v = __bfloat162float(*res) + v;
-  return __float2bfloat16_rn(v);
+// The scalars of LinParams, read from the parameter space once at the start
+// of the kernel (while the first loads are in flight) and kept in registers:
+// left to the compiler, the epilogue's first reads of them are constant-cache
+// misses on the critical path after the last MMA.
+struct Scalars {
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* y;
+  float* part;
+  unsigned* tickets;
+  int32_t* err;
+  int R, Rp, N, ldy, ksplit, ksteps, stages, stage_bytes, tmem_cols, kb;
+};
+
+template <typename T> __device__ __forceinline__ T* keep(T* v) {
+  uint64_t u = reinterpret_cast<uint64_t>(v);
+  asm volatile("" : "+l"(u));
+  return reinterpret_cast<T*>(u);
+}
+__device__ __forceinline__ int keep(int v) {
+  asm volatile("" : "+r"(v));
+  return v;
+}
+
+__device__ __forceinline__ Scalars load_scalars(const LinParams& p) {
+  Scalars c;
+  c.residual = keep(p.residual); c.y = keep(p.y); c.part = keep(p.part);
+  c.tickets = keep(p.tickets); c.err = keep(p.err);
+  c.R = keep(p.R); c.Rp = keep(p.Rp); c.N = keep(p.N); c.ldy = keep(p.ldy);
+  c.ksplit = keep(p.ksplit); c.ksteps = keep(p.ksteps); c.stages = keep(p.stages);
+  c.stage_bytes = keep(p.stage_bytes); c.tmem_cols = keep(p.tmem_cols); c.kb = keep(p.kb);
+  return c;
+}
+
+// The residual of rows cb .. cb + 31 of feature ng (zero past the rows, or
+// without a residual), all loads in flight together.
+__device__ __forceinline__ void load_residual(const Scalars& c, int cb, int ng,
+                                              float (&res)[32]) {
+  const int nr = min(32, c.R - cb);
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    res[j] = c.residual && j < nr
+                 ? __bfloat162float(c.residual[(int64_t)(cb + j) * c.ldy + ng]) : 0.f;
+}
+
+// y[cb + j, ng] = bf16(bf16(v[j]) + res[j]) for the rows j < 32 of this chunk
+// that exist (bf16(v[j]) without a residual).  The caller reads the residual
+// before any y is written: the residual may be y itself.
+__device__ __forceinline__ void store_rows(const Scalars& c, int cb, int ng, const float (&v)[32],
+                                           const float (&res)[32]) {
+  const int nr = min(32, c.R - cb);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j < nr) {
+      float o = bf16_round(v[j]);
+      if (c.residual) o += res[j];
+      c.y[(int64_t)(cb + j) * c.ldy + ng] = __float2bfloat16_rn(o);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_constant__ LinParams p) {
+  const Scalars c = load_scalars(p);
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1 KB aligned for the 128-byte swizzle; offset from smem_raw itself so
+  // the compiler keeps the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned full_mask = 0xffffffffu;
-  const int ST = p.stages, SB = p.stage_bytes;
+  const int ST = c.stages, SB = c.stage_bytes;
   const Bars bars{sbase + (uint32_t)(ST * SB)};
   uint8_t* misc = smem + ST * SB + kNumBars * 8;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 8);
 
-  const int tile = blockIdx.x / p.ksplit, ks = blockIdx.x % p.ksplit;
-  const int k_beg = (int)((int64_t)ks * p.ksteps / p.ksplit);
-  const int nsteps = (int)((int64_t)(ks + 1) * p.ksteps / p.ksplit) - k_beg;
-  const int KB = p.kb;
+  const int tile = blockIdx.x / c.ksplit, ks = blockIdx.x % c.ksplit;
+  const int k_beg = (int)((int64_t)ks * c.ksteps / c.ksplit);
+  const int nsteps = (int)((int64_t)(ks + 1) * c.ksteps / c.ksplit) - k_beg;
+  const int KB = c.kb;
   const int nk = ceil_div(nsteps, KB);  // stages this CTA streams (the last may be short)
   const int n0 = tile * kTileN;
-  const uint32_t x_bytes = (uint32_t)(p.Rp * 128);
+  const uint32_t x_bytes = (uint32_t)(c.Rp * 128);
   const uint32_t x_off = (uint32_t)(KB * kWBox);  // the x boxes follow the stage's weight boxes
   // K steps of stage i: [k_beg + i KB, k_beg + min(nsteps, (i + 1) KB))
   auto steps_of = [&](int i) { return min(KB, nsteps - i * KB); };
@@ -127,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
     ptx::tma_prefetch_desc(&p.tm_x);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), (uint32_t)p.tmem_cols);
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), (uint32_t)c.tmem_cols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -165,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
         const int s = i % ST, ns = steps_of(i);
         const uint32_t dst = sbase + (uint32_t)(s * SB);
         if (!ptx::mbar_wait(bars.empty(s), ((i / ST) & 1) ^ 1)) {
-          record_timeout(p.err, abort_flag);
+          record_timeout(c.err, abort_flag);
           break;
         }
         ptx::mbar_expect_tx(bars.full(s), (uint32_t)ns * ((uint32_t)kWBox + x_bytes));
@@ -179,12 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
       }
       // every issued load lands before the CTA can exit
       for (int u = max(0, issued - ST); u < issued; ++u)
-        if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(p.err, abort_flag);
+        if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(c.err, abort_flag);
     }
   } else if (warp == 1) {
     // ================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t id = ptx::idesc_bf16(kTileN, p.Rp, false, false);
+      const uint32_t id = ptx::idesc_bf16(kTileN, c.Rp, false, false);
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
         const int s = i % ST;
@@ -203,9 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
         }
         ptx::tc_commit(bars.empty(s));
       }
-      if (!ok) record_timeout(p.err, abort_flag);
+      if (!ok) record_timeout(c.err, abort_flag);
       ptx::tc_commit(bars.acc_full());  // also: every MMA has finished
-      if (!ptx::mbar_wait(bars.acc_full(), 0)) record_timeout(p.err, abort_flag);
+      if (!ptx::mbar_wait(bars.acc_full(), 0)) record_timeout(c.err, abort_flag);
     }
   } else {
     // ================================================== epilogue
@@ -214,16 +269,18 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
     const int ng = n0 + n;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     bool ok = nk > 0 && __all_sync(full_mask, ptx::mbar_wait(bars.acc_full(), 0));
-    if (nk > 0 && !ok) record_timeout(p.err, abort_flag);
+    if (nk > 0 && !ok) record_timeout(c.err, abort_flag);
     ok = ok && !__any_sync(full_mask, *abort_flag != 0);
     if (ok) ptx::tc_fence_after();
-    float* part = p.part + ((int64_t)tile * p.ksplit + ks) * p.Rp * kTileN;
-    for (int cb = 0; cb < p.Rp; cb += 32) {
+    const int RP4 = c.Rp + 4;  // padded column of the partials: conflict-free reads
+    float* part = c.part + (((int64_t)tile * c.ksplit + ks) * kTileN + n) * RP4;
+    for (int cb = 0; cb < c.Rp; cb += 32) {
+      const int nc = min(32, c.Rp - cb);  // 32, or the last 16 (Rp is a multiple of 16)
       uint32_t d[32];
       if (ok) {
-        if (p.Rp - cb >= 32) {
+        if (nc == 32) {
           ptx::tmem_ld32_sync(lane_addr + (uint32_t)cb, d);
-        } else {  // the last 16 columns (Rp is a multiple of 16)
+        } else {
           uint32_t d16[16];
           ptx::tmem_ld16_sync(lane_addr + (uint32_t)cb, d16);
 #pragma unroll
@@ -235,21 +292,23 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
 #pragma unroll
         for (int j = 0; j < 32; ++j) d[j] = 0u;
       }
-      if (p.ksplit == 1) {
-        if (ng < p.N) {
+      if (c.ksplit == 1) {
+        float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int r = cb + j;
-            if (r < p.R && ok) {
-              const int64_t o = (int64_t)r * p.ldy + ng;
-              p.y[o] = finish(__uint_as_float(d[j]), p.residual ? p.residual + o : nullptr);
-            }
-          }
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(d[j]);
+        if (ok && ng < c.N) {
+          float res[32];
+          load_residual(c, cb, ng, res);
+          store_rows(c, cb, ng, v, res);
         }
       } else {
+        // this feature's partial sums of rows cb .. cb + nc - 1, contiguous
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (cb + j < p.Rp) __stcg(part + (int64_t)(cb + j) * kTileN + n, __uint_as_float(d[j]));
+        for (int j = 0; j < 32; j += 4)
+          if (j < nc)
+            __stcg(reinterpret_cast<float4*>(part + cb + j),
+                   make_float4(__uint_as_float(d[j]), __uint_as_float(d[j + 1]),
+                               __uint_as_float(d[j + 2]), __uint_as_float(d[j + 3])));
       }
     }
   }
@@ -260,43 +319,59 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+    ptx::tmem_dealloc(tmem, (uint32_t)c.tmem_cols);
   }
-  if (p.ksplit == 1) return;
+  if (c.ksplit == 1) return;
   if (threadIdx.x == 0) {
     __threadfence();  // this CTA's partial is visible before its ticket
-    *last_flag = atomicAdd(p.tickets + tile, 1u) == (unsigned)p.ksplit - 1u;
+    *last_flag = atomicAdd(c.tickets + tile, 1u) == (unsigned)c.ksplit - 1u;
   }
   __syncthreads();
   if (!*last_flag) return;
-  // the tile's partials (one contiguous Rp x 128 block per split) come into
-  // the idle ring by bulk copies, all in flight at once, then are summed in
-  // split order
-  const float* base = p.part + (int64_t)tile * p.ksplit * p.Rp * kTileN;
-  const uint32_t blk_bytes = (uint32_t)(p.Rp * kTileN * 4);
+  // the tile's partials (one contiguous 128 x (Rp + 4) block per split) come
+  // into the idle ring by bulk copies, all in flight at once; thread n then
+  // sums feature n's rows in split order
+  const int RP4 = c.Rp + 4;
+  const float* base = c.part + (int64_t)tile * c.ksplit * kTileN * RP4;
+  const uint32_t blk_bytes = (uint32_t)(kTileN * RP4 * 4);
   if (threadIdx.x == 0) {
     __threadfence();
     ptx::fence_proxy_async_global();  // the partials were written by generic stores
-    ptx::mbar_expect_tx(bars.red_full(), blk_bytes * (uint32_t)p.ksplit);
-    for (int s = 0; s < p.ksplit; ++s)
-      ptx::bulk_g2s(sbase + (uint32_t)s * blk_bytes, base + (int64_t)s * p.Rp * kTileN, blk_bytes,
+    ptx::mbar_expect_tx(bars.red_full(), blk_bytes * (uint32_t)c.ksplit);
+    for (int s = 0; s < c.ksplit; ++s)
+      ptx::bulk_g2s(sbase + (uint32_t)s * blk_bytes, base + (int64_t)s * kTileN * RP4, blk_bytes,
                     bars.red_full());
   }
+  // the first rows' residual comes in while the partials do
+  const int n = threadIdx.x, ng = n0 + n;
+  float res[32];
+  if (n < kTileN && ng < c.N) load_residual(c, 0, ng, res);
   if (!ptx::mbar_wait(bars.red_full(), 0)) {
-    set_err(p.err, ORTHRUS_ETIMEOUT);
-  } else {
-    const float* st = reinterpret_cast<const float*>(smem);
-    for (int e = threadIdx.x; e < p.R * kTileN; e += kThreads) {
-      const int r = e / kTileN, n = e % kTileN, ng = n0 + n;
-      if (ng >= p.N) continue;
-      float sum = 0.f;
-      for (int s = 0; s < p.ksplit; ++s) sum += st[((int64_t)s * p.Rp + r) * kTileN + n];
-      const int64_t o = (int64_t)r * p.ldy + ng;
-      p.y[o] = finish(sum, p.residual ? p.residual + o : nullptr);
+    set_err(c.err, ORTHRUS_ETIMEOUT);
+  } else if (n < kTileN) {
+    const float* st = reinterpret_cast<const float*>(smem) + n * RP4;
+    if (ng < c.N) {
+      for (int cb = 0; cb < c.Rp; cb += 32) {
+        if (cb > 0) load_residual(c, cb, ng, res);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        for (int sp = 0; sp < c.ksplit; ++sp) {
+          const float* src = st + (int64_t)sp * kTileN * RP4 + cb;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            if (cb + j < c.Rp) {
+              const float4 f = *reinterpret_cast<const float4*>(src + j);
+              v[j] += f.x; v[j + 1] += f.y; v[j + 2] += f.z; v[j + 3] += f.w;
+            }
+          }
+        }
+        store_rows(c, cb, ng, v, res);
+      }
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) p.tickets[tile] = 0u;
+  if (threadIdx.x == 0) c.tickets[tile] = 0u;
 }
 
 // ------------------------------------------------------------------ host
@@ -359,7 +434,7 @@ Plan plan(int rows, int K, int N, int sms, int kb) {
   // no more than the ring can stage for the last CTA's sum
   q.ksplit = q.tiles >= sms ? 1 : sms / q.tiles;
   q.ksplit = min(q.ksplit, min(q.ksteps, 16));
-  q.ksplit = max(1, min(q.ksplit, q.stages * q.stage_bytes / (q.Rp * kTileN * 4)));
+  q.ksplit = max(1, min(q.ksplit, q.stages * q.stage_bytes / ((q.Rp + 4) * kTileN * 4)));
   q.smem = q.stages * q.stage_bytes + kNumBars * 8 + 16 + 1024;
   q.tmem_cols = 32;
   while (q.tmem_cols < q.Rp) q.tmem_cols *= 2;
@@ -382,7 +457,7 @@ size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
 size_t workspace_bytes(int rows, int K, int N) {
   // sized for any SM count up to 256
   const Plan q = plan(rows, K, N, 256);
-  const int64_t parts = q.ksplit > 1 ? (int64_t)q.tiles * 16 * q.Rp * kTileN * 4 : 0;
+  const int64_t parts = q.ksplit > 1 ? (int64_t)q.tiles * 16 * (q.Rp + 4) * kTileN * 4 : 0;
   return round256((int64_t)q.tiles * 4) + (size_t)parts;
 }
 
