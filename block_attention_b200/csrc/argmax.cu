@@ -8,9 +8,13 @@
 // values, the smallest index.  NaN maps to key 0 and never wins; -0.0 is
 // canonicalised to +0.0 so the two zeros tie.  Because max is associative
 // and commutative, the result does not depend on how the row is split or in
-// which order CTAs finish.  Each CTA folds its key into the row's slot with
-// atomicMax; the last CTA of the row (ticket counter) decodes the key, writes
-// idx/maxval and returns the slot and the ticket to zero for the next call.
+// which order CTAs finish.  When a row takes at most 16 chunks, its CTAs form
+// one thread-block cluster: each stores its key into the rank-0 CTA's shared
+// memory, and after the cluster barrier rank 0 folds them and writes
+// idx/maxval -- no global atomics, the workspace is not touched.  Longer rows
+// fold each CTA's key into the row's slot with atomicMax; the last CTA of the
+// row (ticket counter) decodes the key, writes idx/maxval and returns the slot
+// and the ticket to zero for the next call.
 #include <cuda.h>
 
 #include <mutex>
@@ -22,6 +26,7 @@ namespace orthrus {
 
 constexpr int kArgmaxThreads = 256;
 constexpr int kArgmaxChunk = 16384;  // elements per CTA (multiple of 8)
+constexpr int kArgmaxMaxCluster = 16;  // most chunks of a row one cluster takes (non-portable)
 
 __device__ __forceinline__ unsigned long long argmax_key(float v, int j) {
   if (v != v) return 0ull;  // NaN
@@ -42,6 +47,119 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a,
   return a > b ? a : b;
 }
 
+// Running (value, index) best of one thread, over elements it visits in
+// increasing index order.  A group of consecutive elements is folded by its
+// NaN-ignoring maximum m; only when m beats the best so far (strictly: an
+// equal value keeps the earlier index) is the group searched for the first
+// element equal to m.  -0.0 == +0.0, so the two zeros tie and the earlier
+// one stays; NaN never wins; a group of NaNs only is skipped.
+struct RunningBest {
+  float v = -INFINITY;
+  int j = -1;  // -1: nothing but NaN seen yet
+  template <int N>
+  __device__ __forceinline__ void fold(const float (&e)[N], int j0) {
+    float m = e[0];
+#pragma unroll
+    for (int u = 1; u < N; ++u) m = fmaxf(m, e[u]);
+    if (m > v || (j < 0 && m == m)) {
+      int k = N - 1;
+#pragma unroll
+      for (int u = N - 2; u >= 0; --u) k = e[u] == m ? u : k;
+      v = m;
+      j = j0 + k;
+    }
+  }
+  __device__ __forceinline__ unsigned long long key() const {
+    return j < 0 ? 0ull : argmax_key(v, j);
+  }
+};
+
+// The key of the best element of chunk c of `row` (elements
+// [c * kArgmaxChunk, min((c + 1) * kArgmaxChunk, vocab))) seen by this thread.
+template <typename T, bool kVec>
+__device__ __forceinline__ unsigned long long scan_chunk(const T* __restrict__ row, int vocab,
+                                                         int c) {
+  const int beg = c * kArgmaxChunk;
+  const int end = min(beg + kArgmaxChunk, vocab);
+  RunningBest rb;
+  if (kVec) {
+    // 4 elements per vector load for f32 (16 B), 8 for bf16 (16 B), all of
+    // the thread's loads in flight before the first is used
+    constexpr int kV = 16 / sizeof(T);
+    constexpr int kIters = kArgmaxChunk / (kV * kArgmaxThreads);
+    uint4 buf[kIters];
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int j = beg + (it * kArgmaxThreads + threadIdx.x) * kV;
+      if (j + kV <= end) buf[it] = __ldcs(reinterpret_cast<const uint4*>(row + j));
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int j = beg + (it * kArgmaxThreads + threadIdx.x) * kV;
+      float e[kV];
+      if (j + kV <= end) {
+        const T* t = reinterpret_cast<const T*>(&buf[it]);
+#pragma unroll
+        for (int u = 0; u < kV; ++u) e[u] = to_f32(t[u]);
+        rb.fold(e, j);
+      } else {
+        for (int u = 0; u < kV && j + u < end; ++u) {
+          const float one[1] = {to_f32(row[j + u])};
+          rb.fold(one, j + u);
+        }
+      }
+    }
+  } else {
+    for (int j = beg + threadIdx.x; j < end; j += kArgmaxThreads) {
+      const float one[1] = {to_f32(row[j])};
+      rb.fold(one, j);
+    }
+  }
+  return rb.key();
+}
+
+// The CTA's best key (valid in thread 0).
+__device__ __forceinline__ unsigned long long cta_best(unsigned long long best) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    best = umax64(best, __shfl_xor_sync(0xffffffffu, best, off));
+  __shared__ unsigned long long warp_best[kArgmaxThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int w = 1; w < kArgmaxThreads / 32; ++w) best = umax64(best, warp_best[w]);
+  return best;
+}
+
+// One cluster of gridDim.x CTAs per row (grid (nchunks, rows), cluster
+// (nchunks, 1, 1)): CTA c scans chunk c and stores its key into slot c of the
+// rank-0 CTA's shared memory; after the cluster barrier rank 0 folds them.
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kArgmaxThreads)
+argmax_cluster_kernel(const T* __restrict__ logits, int vocab, int64_t stride, int32_t* idx,
+                      float* maxval) {
+  __shared__ unsigned long long cta_keys[kArgmaxMaxCluster];
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
+  const int c = blockIdx.x, r = blockIdx.y;
+  const T* row = logits + (int64_t)r * stride;
+  const unsigned long long best = cta_best(scan_chunk<T, kVec>(row, vocab, c));
+  if (threadIdx.x == 0)
+    ptx::st_cluster_u64(ptx::map_rank(ptx::smem_u32(&cta_keys[c]), 0), best);
+  ptx::cluster_sync();  // release / acquire: every CTA's key is in rank 0's slots
+  if (c == 0 && threadIdx.x == 0) {
+    unsigned long long k = 0ull;
+    for (int q = 0; q < (int)gridDim.x; ++q) k = umax64(k, cta_keys[q]);
+    if (k == 0ull) {  // every element was NaN
+      idx[r] = 0;
+      if (maxval) maxval[r] = to_f32(row[0]);
+    } else {
+      idx[r] = (int32_t)(0xFFFFFFFFu - (unsigned)(k & 0xFFFFFFFFull));
+      if (maxval) maxval[r] = key_value(k);
+    }
+  }
+}
+
 template <typename T, bool kVec>
 __global__ void __launch_bounds__(kArgmaxThreads)
 argmax_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
@@ -54,44 +172,9 @@ argmax_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
   ptx::griddep_launch_dependents();
   ptx::griddep_wait();
   const T* row = logits + (int64_t)r * stride;
-  const int beg = c * kArgmaxChunk;
-  const int end = min(beg + kArgmaxChunk, vocab);
-  unsigned long long best = 0ull;
-  if (kVec) {
-    // 4 elements per vector load for f32 (16 B), 8 for bf16 (16 B)
-    constexpr int kV = 16 / sizeof(T);
-    constexpr int kIters = kArgmaxChunk / (kV * kArgmaxThreads);
-    uint4 buf[kIters];
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int j = beg + (it * kArgmaxThreads + threadIdx.x) * kV;
-      if (j + kV <= end) buf[it] = __ldcs(reinterpret_cast<const uint4*>(row + j));
-    }
-#pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-      const int j = beg + (it * kArgmaxThreads + threadIdx.x) * kV;
-      if (j + kV <= end) {
-        const T* e = reinterpret_cast<const T*>(&buf[it]);
-#pragma unroll
-        for (int u = 0; u < kV; ++u) best = umax64(best, argmax_key(to_f32(e[u]), j + u));
-      } else {
-        for (int u = 0; u < kV && j + u < end; ++u)
-          best = umax64(best, argmax_key(to_f32(row[j + u]), j + u));
-      }
-    }
-  } else {
-    for (int j = beg + threadIdx.x; j < end; j += kArgmaxThreads)
-      best = umax64(best, argmax_key(to_f32(row[j]), j));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1)
-    best = umax64(best, __shfl_xor_sync(0xffffffffu, best, off));
-  __shared__ unsigned long long warp_best[kArgmaxThreads / 32];
+  const unsigned long long best = cta_best(scan_chunk<T, kVec>(row, vocab, c));
   __shared__ bool last;
-  if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = best;
-  __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < kArgmaxThreads / 32; ++w) best = umax64(best, warp_best[w]);
     atomicMax(&keys[r], best);
     __threadfence();
     last = atomicAdd(&tickets[r], 1u) == (unsigned)nchunks - 1u;
@@ -123,15 +206,36 @@ cudaError_t launch_argmax(int dtype, const void* logits, int rows, int vocab,
   const size_t es = dtype == ORTHRUS_F32 ? 4 : 2;
   const bool vec = (reinterpret_cast<uintptr_t>(logits) % 16 == 0) &&
                    ((stride * (int64_t)es) % 16 == 0);
-  cudaLaunchAttribute pdl;
-  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nchunks, rows);
   cfg.blockDim = dim3(kArgmaxThreads);
   cfg.stream = st;
-  cfg.attrs = &pdl;
+  cfg.attrs = attrs;
   cfg.numAttrs = 1;
+  if (nchunks <= kArgmaxMaxCluster) {
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = (unsigned)nchunks;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    auto go = [&](auto kernel, auto p) -> cudaError_t {
+      const cudaError_t e =
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      return cudaLaunchKernelEx(&cfg, kernel, p, vocab, stride, idx, maxval);
+    };
+    if (dtype == ORTHRUS_F32) {
+      auto p = static_cast<const float*>(logits);
+      return vec ? go(argmax_cluster_kernel<float, true>, p)
+                 : go(argmax_cluster_kernel<float, false>, p);
+    }
+    auto p = static_cast<const __nv_bfloat16*>(logits);
+    return vec ? go(argmax_cluster_kernel<__nv_bfloat16, true>, p)
+               : go(argmax_cluster_kernel<__nv_bfloat16, false>, p);
+  }
   if (dtype == ORTHRUS_F32) {
     auto p = static_cast<const float*>(logits);
     return vec ? cudaLaunchKernelEx(&cfg, argmax_kernel<float, true>, p, vocab, stride, nchunks,

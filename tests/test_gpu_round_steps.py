@@ -24,7 +24,7 @@ def gpu_argmax(x, stride=None):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("vocab", [1024, 8192, 151936, 100003])
+@pytest.mark.parametrize("vocab", [1024, 8192, 151936, 100003, 300007])
 def test_argmax_random_rows(oracle_mod, dtype, vocab):
     x = synth.logits(synth.rng(201, vocab), 32, vocab, std=3.0, dtype=dtype)
     idx, mx = gpu_argmax(x)
@@ -34,9 +34,9 @@ def test_argmax_random_rows(oracle_mod, dtype, vocab):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_argmax_ties_nan_zero_and_strides(oracle_mod, dtype):
+@pytest.mark.parametrize("V", [151936, 300007])  # one cluster per row; atomics across CTAs
+def test_argmax_ties_nan_zero_and_strides(oracle_mod, dtype, V):
     g = synth.rng(202)
-    V = 151936
     x = synth.logits(g, 24, V, dtype=dtype)
     top = synth.cast(np.array([60.0], np.float32), dtype)[0]
     for r in range(0, 8):  # planted ties across chunk boundaries
@@ -50,19 +50,22 @@ def test_argmax_ties_nan_zero_and_strides(oracle_mod, dtype):
     x[10, 9] = synth.cast(np.array([0.0], np.float32), dtype)[0]   # -0 == +0 -> 5
     x[11, :] = synth.cast(np.array([2.5], np.float32), dtype)[0]   # all equal -> 0
     x[12, -1] = top                     # max in the last element (ragged tail)
+    x[13, :] = synth.cast(np.array([-np.inf], np.float32), dtype)[0]
+    x[13, :3] = nan                     # -inf everywhere else: the first -inf wins
     ref = oracle_mod.vocab_argmax(x)
     for stride in (None, V + 8, V + 3):  # aligned and unaligned row strides
         idx, _ = gpu_argmax(x, stride)
         np.testing.assert_array_equal(idx, ref)
-    assert ref[8] == 0 and ref[10] == 5 and ref[11] == 0 and ref[12] == V - 1
+    assert ref[8] == 0 and ref[10] == 5 and ref[11] == 0 and ref[12] == V - 1 and ref[13] == 3
 
 
 def test_argmax_repeated_calls_reuse_workspace(oracle_mod):
     """The workspace's slots return to zero: many calls in a row agree."""
     for s in range(5):
-        x = synth.logits(synth.rng(203, s), 7, 5000)
-        idx, _ = gpu_argmax(x)
-        np.testing.assert_array_equal(idx, oracle_mod.vocab_argmax(x))
+        for V in (5000, 300007):
+            x = synth.logits(synth.rng(203, s), 7, V)
+            idx, _ = gpu_argmax(x)
+            np.testing.assert_array_equal(idx, oracle_mod.vocab_argmax(x))
 
 
 def _gpu_consensus(d, a):
