@@ -11,12 +11,35 @@
 // Random numbers: Philox4x32-10 (philox.cuh), counter layout in orthrus.h.
 #include "common.cuh"
 #include "philox.cuh"
+#include "tc_ptx.cuh"
 
 namespace orthrus {
 namespace {
 
 bool dtype_ok(int32_t t) { return t == ORTHRUS_F32 || t == ORTHRUS_BF16; }
 int status(cudaError_t e) { return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA; }
+
+// Every kernel here is launched with programmatic stream serialization: it
+// may start while the preceding kernel finishes, lets its own dependents
+// start at once, and waits for its predecessor before reading anything.
+template <typename... KA, typename... A>
+cudaError_t launch_pdl(void (*kernel)(KA...), dim3 grid, cudaStream_t st, A... args) {
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KA>(args)...);
+}
+
+__device__ __forceinline__ void pdl_enter() {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
+}
 
 // Keys ordering (value, lowest index first) as one unsigned 64-bit number.
 __device__ __forceinline__ unsigned long long order_key(float v, int j) {
@@ -40,18 +63,46 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int e) {
 // ------------------------------------------------------------ shared pieces
 // Every kernel here cuts rows into chunks of kChunk elements, one CTA per
 // (chunk, row), kPer elements per thread held in registers.
+// 24 elements per thread (six Philox groups of four): a 151936-entry row is
+// 25 chunks, so 32 rows are 800 CTAs -- one wave at six CTAs per SM.
 constexpr int kThreads = 256;
-constexpr int kPer = 16;
+constexpr int kPer = 24;
 constexpr int kChunk = kThreads * kPer;
 constexpr int kWarps = kThreads / 32;
+static_assert(kThreads == 256, "launch_pdl launches 256-thread CTAs");
+constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ float qnan() { return __int_as_float(0x7fc00000); }
 
-// Gumbel noise -log(-log u).  The inner log keeps full relative accuracy
-// (near u = 1, -log u ~ 1 - u is tiny and its relative error becomes the
-// noise's absolute error); the outer one needs only absolute accuracy.
+// The hardware base-2 logarithm and exponential (MUFU; absolute error of
+// lg2 about 2^-22, relative error of ex2 about 2^-22).
+__device__ __forceinline__ float hw_lg2(float x) {
+  float y;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float hw_ex2(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Gumbel noise -ln(E) of the exponential variate E = -ln u, u =
+// philox_uniform(w) = ((w >> 9) + 1/2) 2^-23, to a few parts in 10^6:
+//   E: for u <= 15/16 from lg2 (|log2 u| >= 0.093, so its absolute error is
+//      under 3e-6 relative); above, from the series
+//      -ln(1 - v) = v (1 + v/2 + v^2/3 + v^3/4 + v^4/5 + ...) with
+//      v = 1 - u = ((~w >> 9) + 1/2) 2^-23 formed exactly from the bits
+//      (truncation below v^5/6 < 2e-7 relative for v < 1/16).
+//   -ln E from lg2: absolute error a few 10^-6 over E's whole range.
+// The argmax over keys x/T + g then agrees with exact arithmetic wherever
+// the two best keys are more than ~1e-5 apart.
 __device__ __forceinline__ float gumbel(uint32_t w) {
-  return -__logf(-logf(philox_uniform(w)));
+  const float u = philox_uniform(w);
+  const float v = (float)((~w) >> 9) * 0x1p-23f + 0x1p-24f;
+  const float series = v * fmaf(v, fmaf(v, fmaf(v, fmaf(v, 0.2f, 0.25f), 1.f / 3.f), 0.5f), 1.f);
+  const float e = v < 0.0625f ? series : -kLn2 * hw_lg2(u);
+  return -kLn2 * hw_lg2(e);
 }
 
 // Block-wide max or sum in a fixed tree; every thread gets the result.
@@ -83,9 +134,18 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) 
 __device__ __forceinline__ float2 chunk_pair(const float (&x)[kPer], float m, float* red) {
   m = block_reduce(m, true, red);
   float s = 0.f;
+  const float mb = m * kLog2e;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) s += expf(x[e] - m);  // exp(-inf) = 0 past the row
+  for (int e = 0; e < kPer; ++e) s += hw_ex2(fmaf(x[e], kLog2e, -mb));  // 0 past the row
   return make_float2(m, block_reduce(s, false, red));
+}
+
+// The same from per-thread running pairs (m, s): s = sum exp(x - m) over the
+// thread's elements.
+__device__ __forceinline__ float2 merge_thread_pairs(float m, float s, float* red) {
+  const float M = block_reduce(m, true, red);
+  s = m == -INFINITY ? 0.f : s * hw_ex2((m - M) * kLog2e);
+  return make_float2(M, block_reduce(s, false, red));
 }
 
 // One warp merges a row's chunk pairs -- lane i takes chunks i, i + 32, ...,
@@ -116,16 +176,17 @@ __device__ __forceinline__ unsigned long long warp_max64(unsigned long long v) {
 
 // ------------------------------------------------------------ draft sample
 // Thread t of chunk c takes the groups g = c * kChunk/4 + i * kThreads + t
-// (i < kPer/4), each the 4 consecutive elements one Philox call covers.  A
-// thread visits its elements in increasing index, so it keeps its best as a
-// (value, index) pair replaced only by a strictly larger value (NaN never
-// wins; equal values keep the lower index) and forms the 64-bit order key
-// once.  The best (key, index) of the CTA goes to the row's slot by
-// atomicMax; with kLse the CTA also stores its chunk pair.  The row's last
-// CTA (ticket) writes idx, lse and logprob and returns slot and ticket to
-// zero.
-template <typename T, bool kLse>
-__global__ void __launch_bounds__(kThreads, 8)  // 8 CTAs (2048 threads) per SM
+// (i < kPer/4), each the 4 consecutive elements one Philox call covers (one
+// 16-byte load when the row allows).  A thread visits its elements in
+// increasing index, so it keeps its best as a (value, index) pair replaced
+// only by a strictly larger value (NaN never wins; equal values keep the
+// lower index) and forms the 64-bit order key once; with kLse it also keeps
+// a running (max, sum of exp(x - max)) pair.  The best key of the CTA goes
+// to the row's slot by atomicMax; with kLse the CTA also stores its chunk
+// pair.  The row's last CTA (ticket) writes idx, lse and logprob and returns
+// slot and ticket to zero.
+template <typename T, bool kLse, bool kVec>
+__global__ void __launch_bounds__(kThreads, 6)  // 6 CTAs per SM: 800 fill one wave
 vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, float inv_t,
                     uint32_t k0, uint32_t k1, uint32_t step, int nchunks,
                     unsigned long long* keys, unsigned* tickets, float2* pairs,
@@ -134,33 +195,72 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
   __shared__ float red[kWarps + 1];
   __shared__ unsigned long long wbest[kWarps];
   __shared__ bool last;
+  pdl_enter();
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, lane = t & 31;
   const T* row = logits + (int64_t)r * stride;
-  float x[kPer];
-  float m = -INFINITY, bv = -INFINITY;
+  float bv = -INFINITY, m = -INFINITY, sum = 0.f;
   int bi = -1;
+  // two batches of three groups: a batch's loads first, then its arithmetic
+  constexpr int kB = kPer / 8;
 #pragma unroll
-  for (int i = 0; i < kPer / 4; ++i) {
+  for (int half = 0; half < 2; ++half) {
+  float xs[4 * kB];
+#pragma unroll
+  for (int ii = 0; ii < kB; ++ii) {
+    const int i = half * kB + ii;
+    const int j0 = 4 * (c * (kChunk / 4) + i * kThreads + t);
+    if (kVec && j0 + 3 < vocab) {
+      if constexpr (sizeof(T) == 4) {
+        const float4 f = __ldcs(reinterpret_cast<const float4*>(row + j0));
+        xs[4 * ii] = f.x; xs[4 * ii + 1] = f.y; xs[4 * ii + 2] = f.z; xs[4 * ii + 3] = f.w;
+      } else {
+        const uint2 u = __ldcs(reinterpret_cast<const uint2*>(row + j0));
+        xs[4 * ii] = __uint_as_float(u.x << 16);
+        xs[4 * ii + 1] = __uint_as_float(u.x & 0xffff0000u);
+        xs[4 * ii + 2] = __uint_as_float(u.y << 16);
+        xs[4 * ii + 3] = __uint_as_float(u.y & 0xffff0000u);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xs[4 * ii + e] = j0 + e < vocab ? to_f32(row[j0 + e]) : 0.f;
+    }
+  }
+#pragma unroll
+  for (int ii = 0; ii < kB; ++ii) {
+    const int i = half * kB + ii;
     const int g = c * (kChunk / 4) + i * kThreads + t;
     const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step),
                                   k0, k1);
+    float x[4];
+    float gm = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int j = 4 * g + e;
-      const bool in = j < vocab;
-      x[4 * i + e] = in ? to_f32(row[j]) * inv_t : -INFINITY;
-      m = fmaxf(m, x[4 * i + e]);
-      const float key = x[4 * i + e] + gumbel(word(w, e));
-      if (in && (key > bv || bi < 0)) {
+      x[e] = j < vocab ? xs[4 * ii + e] * inv_t : -INFINITY;
+      gm = fmaxf(gm, x[e]);
+      const float key = x[e] + gumbel(word(w, e));
+      if (j < vocab && (key > bv || bi < 0)) {
         if (key == key) { bv = key; bi = j; }
       }
     }
+    if constexpr (kLse) {
+      if (gm > m) {
+        sum = m == -INFINITY ? 0.f : sum * hw_ex2((m - gm) * kLog2e);
+        m = gm;
+      }
+      if (m != -INFINITY) {
+        const float mb = m * kLog2e;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sum += hw_ex2(fmaf(x[e], kLog2e, -mb));
+      }
+    }
+  }
   }
   unsigned long long best = bi < 0 ? 0ull : order_key(bv, bi);
   best = warp_max64(best);
   if (lane == 0) wbest[t >> 5] = best;
   float2 pr = make_float2(0.f, 0.f);
-  if constexpr (kLse) pr = chunk_pair(x, m, red);  // its barriers publish wbest
+  if constexpr (kLse) pr = merge_thread_pairs(m, sum, red);  // its barriers publish wbest
   else __syncthreads();
   if (t == 0) {
     for (int w = 1; w < kWarps; ++w) best = umax64(best, wbest[w]);
@@ -213,6 +313,7 @@ token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
                      float* __restrict__ lse) {
   __shared__ float red[kWarps + 1];
   __shared__ bool last;
+  pdl_enter();
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x;
   const T* row = logits + (int64_t)r * stride;
   float x[kPer];
@@ -254,11 +355,12 @@ struct SeqSlot {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 6)
 consensus_verify_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, float inv_t,
                         int nchunks, SeqSlot* seq, unsigned* row_tickets, float2* pairs) {
   __shared__ float red[kWarps + 1];
   __shared__ bool last;
+  pdl_enter();
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, blk = p.blk, b = r / blk;
   const T* row = static_cast<const T*>(p.logits_ar) + (int64_t)r * p.row_stride;
   float x[kPer];
@@ -310,6 +412,7 @@ __global__ void __launch_bounds__(kThreads)
 consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, float inv_t,
                           int nchunks, SeqSlot* seq) {
   __shared__ unsigned long long wres[kWarps], wmax[kWarps];
+  pdl_enter();
   const int c = blockIdx.x, b = blockIdx.y, t = threadIdx.x, blk = p.blk;
   const int L = p.accept_len[b];
   if (L >= blk) return;  // every draft accepted: no correction
@@ -394,19 +497,34 @@ int orthrus_vocab_sample(int32_t dtype, const void* logits, int32_t rows, int32_
   const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
   const float inv_t = 1.f / temperature;
   const bool want = logprob || lse;
+  // one 16-byte (f32) or 8-byte (bf16) load per group of four: the base
+  // aligned to a group and every row starting on a group boundary
+  const size_t gbytes = dtype == ORTHRUS_F32 ? 16 : 8;
+  const bool vec = reinterpret_cast<uintptr_t>(logits) % gbytes == 0 && row_stride % 4 == 0;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid(nchunks, rows);
-#define ORTHRUS_SAMPLE(T, L)                                                              \
-  vocab_sample_kernel<T, L><<<grid, kThreads, 0, st>>>(                                   \
-      static_cast<const T*>(logits), vocab, row_stride, inv_t, k0, k1, step, nchunks, keys, \
-      tickets, pairs, idx, logprob, lse)
+  cudaError_t e;
+#define ORTHRUS_SAMPLE(T, L, V)                                                              \
+  e = launch_pdl(vocab_sample_kernel<T, L, V>, grid, st, static_cast<const T*>(logits), vocab, \
+                 row_stride, inv_t, k0, k1, step, nchunks, keys, tickets, pairs, idx, logprob, \
+                 lse)
   if (dtype == ORTHRUS_F32) {
-    if (want) ORTHRUS_SAMPLE(float, true); else ORTHRUS_SAMPLE(float, false);
+    if (vec) {
+      if (want) ORTHRUS_SAMPLE(float, true, true); else ORTHRUS_SAMPLE(float, false, true);
+    } else {
+      if (want) ORTHRUS_SAMPLE(float, true, false); else ORTHRUS_SAMPLE(float, false, false);
+    }
   } else {
-    if (want) ORTHRUS_SAMPLE(__nv_bfloat16, true); else ORTHRUS_SAMPLE(__nv_bfloat16, false);
+    if (vec) {
+      if (want) ORTHRUS_SAMPLE(__nv_bfloat16, true, true);
+      else ORTHRUS_SAMPLE(__nv_bfloat16, false, true);
+    } else {
+      if (want) ORTHRUS_SAMPLE(__nv_bfloat16, true, false);
+      else ORTHRUS_SAMPLE(__nv_bfloat16, false, false);
+    }
   }
 #undef ORTHRUS_SAMPLE
-  return status(cudaGetLastError());
+  return status(e);
 }
 
 size_t orthrus_token_logprob_workspace(int32_t rows, int32_t vocab) {
@@ -437,14 +555,12 @@ int orthrus_token_logprob(int32_t dtype, const void* logits, int32_t rows, int32
   auto st = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid(nchunks, rows);
   if (dtype == ORTHRUS_F32)
-    token_logprob_kernel<float><<<grid, kThreads, 0, st>>>(
-        static_cast<const float*>(logits), vocab, row_stride, idx, inv_t, nchunks, tickets,
-        pairs, logprob, lse);
-  else
-    token_logprob_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(logits), vocab, row_stride, idx, inv_t, nchunks,
-        tickets, pairs, logprob, lse);
-  return status(cudaGetLastError());
+    return status(launch_pdl(token_logprob_kernel<float>, grid, st,
+                             static_cast<const float*>(logits), vocab, row_stride, idx, inv_t,
+                             nchunks, tickets, pairs, logprob, lse));
+  return status(launch_pdl(token_logprob_kernel<__nv_bfloat16>, grid, st,
+                           static_cast<const __nv_bfloat16*>(logits), vocab, row_stride, idx,
+                           inv_t, nchunks, tickets, pairs, logprob, lse));
 }
 
 size_t orthrus_consensus_sample_workspace(int32_t B, int32_t blk, int32_t vocab) {
@@ -480,17 +596,21 @@ int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stre
   auto st = reinterpret_cast<cudaStream_t>(stream);
   const int nres = ceil_div(a->vocab, kResChunk);
   const dim3 g1(nchunks, (unsigned)rows), g2(nres, a->B);
+  const orthrus_sample_args args = *a;
+  cudaError_t e;
   if (a->dtype == ORTHRUS_F32) {
-    consensus_verify_kernel<float><<<g1, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks, seq,
-                                                             row_tickets, pairs);
-    consensus_residual_kernel<float><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t, nres, seq);
+    e = launch_pdl(consensus_verify_kernel<float>, g1, st, args, k0, k1, inv_t, nchunks, seq,
+                   row_tickets, pairs);
+    if (e == cudaSuccess)
+      e = launch_pdl(consensus_residual_kernel<float>, g2, st, args, k0, k1, inv_t, nres, seq);
   } else {
-    consensus_verify_kernel<__nv_bfloat16><<<g1, kThreads, 0, st>>>(*a, k0, k1, inv_t, nchunks,
-                                                                     seq, row_tickets, pairs);
-    consensus_residual_kernel<__nv_bfloat16><<<g2, kThreads, 0, st>>>(*a, k0, k1, inv_t,
-                                                                      nres, seq);
+    e = launch_pdl(consensus_verify_kernel<__nv_bfloat16>, g1, st, args, k0, k1, inv_t,
+                   nchunks, seq, row_tickets, pairs);
+    if (e == cudaSuccess)
+      e = launch_pdl(consensus_residual_kernel<__nv_bfloat16>, g2, st, args, k0, k1, inv_t,
+                     nres, seq);
   }
-  return status(cudaGetLastError());
+  return status(e);
 }
 
 }  // extern "C"

@@ -187,14 +187,38 @@ class DecodeRound:
                 "commit": commit}
 
     # ------------------------------------------------------------ host I/O
+    INPUTS = ("q", "k_blk", "v_blk", "logits")
+
     def pinned_inputs(self):
         """Pinned host copies of one round's inputs (for the end-to-end path)."""
-        return {k: getattr(self, k).cpu().pin_memory() for k in ("q", "k_blk", "v_blk", "logits")}
+        return {k: getattr(self, k).cpu().pin_memory() for k in self.INPUTS}
 
-    def h2d(self, host):
+    def h2d(self, host, into=None):
+        """Copy a round's inputs from (pinned) host memory into the current
+        input set, or into input set `into` (see add_input_set)."""
+        bufs = self.input_sets[into][0] if into is not None else {
+            k: getattr(self, k) for k in self.INPUTS}
         for k, t in host.items():
-            getattr(self, k).copy_(t, non_blocking=True)
+            bufs[k].copy_(t, non_blocking=True)
         return sum(t.numel() * t.element_size() for t in host.values())
+
+    def add_input_set(self):
+        """A second set of per-round input buffers with graphs of its own
+        (after capture()), so that one set's inputs can be copied in while
+        the round on the other set runs.  Caches, lengths, outputs and
+        workspaces stay shared: rounds still run one after another."""
+        first = ({k: getattr(self, k) for k in self.INPUTS}, self.graphs)
+        for k in self.INPUTS:
+            setattr(self, k, first[0][k].clone())
+        self.capture()
+        self.input_sets = [first, ({k: getattr(self, k) for k in self.INPUTS}, self.graphs)]
+        self.use_set(0)
+
+    def use_set(self, s):
+        bufs, graphs = self.input_sets[s]
+        for k, t in bufs.items():
+            setattr(self, k, t)
+        self.graphs = graphs
 
     def pinned_outputs(self):
         return {k: torch.empty(getattr(self, k).shape, dtype=torch.int32).pin_memory()

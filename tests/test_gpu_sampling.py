@@ -21,7 +21,8 @@ pytestmark = pytest.mark.gpu
 SAFE = 1e-3  # margin (in log units) beyond FP32 rounding of the keys
 
 
-@pytest.mark.parametrize("dtype,rows,vocab,T", [("f32", 32, 151936, 0.8), ("bf16", 7, 1000, 1.3)])
+@pytest.mark.parametrize("dtype,rows,vocab,T", [("f32", 32, 151936, 0.8), ("bf16", 7, 1000, 1.3),
+                                                ("f32", 5, 1001, 1.0), ("bf16", 3, 6, 0.7)])
 def test_vocab_sample_matches_oracle(oracle_mod, dtype, rows, vocab, T):
     for step in (0, 3):
         x = synth.logits(synth.rng(600 + step, len(dtype)), rows, vocab, dtype=dtype)
