@@ -70,39 +70,47 @@ constexpr int kPer = 24;
 constexpr int kChunk = kThreads * kPer;
 constexpr int kWarps = kThreads / 32;
 static_assert(kThreads == 256, "launch_pdl launches 256-thread CTAs");
-constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float qnan() { return __int_as_float(0x7fc00000); }
 
 // The hardware base-2 logarithm and exponential (MUFU; absolute error of
-// lg2 about 2^-22, relative error of ex2 about 2^-22).
+// lg2 about 2^-22, relative error of ex2 about 2^-22), flushing subnormals:
+// lg2 only ever sees normal arguments here (uniforms >= 2^-24, exponential
+// variates >= 8e-8), and an ex2 result below 2^-126 adds nothing to a sum
+// that holds at least exp(0) = 1.
 __device__ __forceinline__ float hw_lg2(float x) {
   float y;
-  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ float hw_ex2(float x) {
   float y;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-// Gumbel noise -ln(E) of the exponential variate E = -ln u, u =
-// philox_uniform(w) = ((w >> 9) + 1/2) 2^-23, to a few parts in 10^6:
-//   E: for u <= 15/16 from lg2 (|log2 u| >= 0.093, so its absolute error is
-//      under 3e-6 relative); above, from the series
-//      -ln(1 - v) = v (1 + v/2 + v^2/3 + v^3/4 + v^4/5 + ...) with
-//      v = 1 - u = ((~w >> 9) + 1/2) 2^-23 formed exactly from the bits
-//      (truncation below v^5/6 < 2e-7 relative for v < 1/16).
-//   -ln E from lg2: absolute error a few 10^-6 over E's whole range.
-// The argmax over keys x/T + g then agrees with exact arithmetic wherever
-// the two best keys are more than ~1e-5 apart.
-__device__ __forceinline__ float gumbel(uint32_t w) {
+// Gumbel noise in base 2: log2(e) times -ln(E) of the exponential variate
+// E = -ln u, u = philox_uniform(w) = ((w >> 9) + 1/2) 2^-23, less the
+// constant log2(log2 e) (which no comparison of keys sees):
+//   gumbel2(w) = -log2(E2),  E2 = E / ln 2 = -log2 u,
+// to a few parts in 10^6:
+//   E2: for u <= 15/16 from lg2 (|log2 u| >= 0.093, so lg2's absolute error
+//       of about 2^-22 is under 3e-6 relative); above, from the series
+//       -ln(1 - v) = v (1 + v/2 + v^2/3 + v^3/4 + ...) times log2 e, with
+//       v = 1 - u exact (Sterbenz) and the truncation below v^4/5 < 4e-6
+//       relative for v <= 1/16;
+//   -log2 E2 from lg2: absolute error a few 10^-7 over E2's whole range.
+// Keys x log2(e) / T + gumbel2 then order as x / T + Gumbel does, and their
+// argmax agrees with exact arithmetic wherever the two best keys are more
+// than ~1e-5 apart.
+constexpr float kS1 = kLog2e, kS2 = kLog2e / 2, kS3 = kLog2e / 3, kS4 = kLog2e / 4;
+__device__ __forceinline__ float gumbel2(uint32_t w) {
   const float u = philox_uniform(w);
-  const float v = (float)((~w) >> 9) * 0x1p-23f + 0x1p-24f;
-  const float series = v * fmaf(v, fmaf(v, fmaf(v, fmaf(v, 0.2f, 0.25f), 1.f / 3.f), 0.5f), 1.f);
-  const float e = v < 0.0625f ? series : -kLn2 * hw_lg2(u);
-  return -kLn2 * hw_lg2(e);
+  const float v = 1.f - u;
+  const float series = v * fmaf(v, fmaf(v, fmaf(v, kS4, kS3), kS2), kS1);
+  const float e2 = v <= 0.0625f ? series : -hw_lg2(u);
+  return -hw_lg2(e2);
 }
 
 // Block-wide max or sum in a fixed tree; every thread gets the result.
@@ -133,10 +141,12 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) 
 // (max, sum of exp(x - max)) over the CTA's chunk.
 __device__ __forceinline__ float2 chunk_pair(const float (&x)[kPer], float m, float* red) {
   m = block_reduce(m, true, red);
+  // the difference first (exact near the maximum), then the base change:
+  // at a low temperature x and m are large and x log2(e) - m log2(e) would
+  // lose the difference to rounding
   float s = 0.f;
-  const float mb = m * kLog2e;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) s += hw_ex2(fmaf(x[e], kLog2e, -mb));  // 0 past the row
+  for (int e = 0; e < kPer; ++e) s += hw_ex2((x[e] - m) * kLog2e);  // 0 past the row
   return make_float2(m, block_reduce(s, false, red));
 }
 
@@ -198,63 +208,62 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
   pdl_enter();
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, lane = t & 31;
   const T* row = logits + (int64_t)r * stride;
+  // keys in base 2 (x log2(e) / T + gumbel2); the running (max, sum of
+  // exp(x / T - max)) in natural units, each difference taken before the
+  // base change (see chunk_pair)
   float bv = -INFINITY, m = -INFINITY, sum = 0.f;
   int bi = -1;
   // two batches of three groups: a batch's loads first, then its arithmetic
   constexpr int kB = kPer / 8;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-  float xs[4 * kB];
+    float xs[4 * kB];  // past the row: -inf (never wins, adds exp(-inf) = 0)
 #pragma unroll
-  for (int ii = 0; ii < kB; ++ii) {
-    const int i = half * kB + ii;
-    const int j0 = 4 * (c * (kChunk / 4) + i * kThreads + t);
-    if (kVec && j0 + 3 < vocab) {
-      if constexpr (sizeof(T) == 4) {
-        const float4 f = __ldcs(reinterpret_cast<const float4*>(row + j0));
-        xs[4 * ii] = f.x; xs[4 * ii + 1] = f.y; xs[4 * ii + 2] = f.z; xs[4 * ii + 3] = f.w;
+    for (int ii = 0; ii < kB; ++ii) {
+      const int j0 = 4 * (c * (kChunk / 4) + (half * kB + ii) * kThreads + t);
+      if (kVec && j0 + 3 < vocab) {
+        if constexpr (sizeof(T) == 4) {
+          const float4 f = __ldcs(reinterpret_cast<const float4*>(row + j0));
+          xs[4 * ii] = f.x; xs[4 * ii + 1] = f.y; xs[4 * ii + 2] = f.z; xs[4 * ii + 3] = f.w;
+        } else {
+          const uint2 u = __ldcs(reinterpret_cast<const uint2*>(row + j0));
+          xs[4 * ii] = __uint_as_float(u.x << 16);
+          xs[4 * ii + 1] = __uint_as_float(u.x & 0xffff0000u);
+          xs[4 * ii + 2] = __uint_as_float(u.y << 16);
+          xs[4 * ii + 3] = __uint_as_float(u.y & 0xffff0000u);
+        }
       } else {
-        const uint2 u = __ldcs(reinterpret_cast<const uint2*>(row + j0));
-        xs[4 * ii] = __uint_as_float(u.x << 16);
-        xs[4 * ii + 1] = __uint_as_float(u.x & 0xffff0000u);
-        xs[4 * ii + 2] = __uint_as_float(u.y << 16);
-        xs[4 * ii + 3] = __uint_as_float(u.y & 0xffff0000u);
-      }
-    } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) xs[4 * ii + e] = j0 + e < vocab ? to_f32(row[j0 + e]) : 0.f;
-    }
-  }
-#pragma unroll
-  for (int ii = 0; ii < kB; ++ii) {
-    const int i = half * kB + ii;
-    const int g = c * (kChunk / 4) + i * kThreads + t;
-    const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step),
-                                  k0, k1);
-    float x[4];
-    float gm = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = 4 * g + e;
-      x[e] = j < vocab ? xs[4 * ii + e] * inv_t : -INFINITY;
-      gm = fmaxf(gm, x[e]);
-      const float key = x[e] + gumbel(word(w, e));
-      if (j < vocab && (key > bv || bi < 0)) {
-        if (key == key) { bv = key; bi = j; }
+        for (int e = 0; e < 4; ++e)
+          xs[4 * ii + e] = j0 + e < vocab ? to_f32(row[j0 + e]) : -INFINITY;
       }
     }
-    if constexpr (kLse) {
-      if (gm > m) {
-        sum = m == -INFINITY ? 0.f : sum * hw_ex2((m - gm) * kLog2e);
-        m = gm;
-      }
-      if (m != -INFINITY) {
-        const float mb = m * kLog2e;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sum += hw_ex2(fmaf(x[e], kLog2e, -mb));
+    for (int ii = 0; ii < kB; ++ii) {
+      const int g = c * (kChunk / 4) + (half * kB + ii) * kThreads + t;
+      const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step),
+                                    k0, k1);
+      float x[4];
+      float gm = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[e] = xs[4 * ii + e] * inv_t;
+        gm = fmaxf(gm, x[e]);
+        // strictly larger: equal keys keep the lower index, NaN never wins
+        const float key = fmaf(x[e], kLog2e, gumbel2(word(w, e)));
+        if (key > bv) { bv = key; bi = 4 * g + e; }
+      }
+      if constexpr (kLse) {
+        if (gm > m) {
+          sum = m == -INFINITY ? 0.f : sum * hw_ex2((m - gm) * kLog2e);
+          m = gm;
+        }
+        if (m != -INFINITY) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sum += hw_ex2((x[e] - m) * kLog2e);
+        }
       }
     }
-  }
   }
   unsigned long long best = bi < 0 ? 0ull : order_key(bv, bi);
   best = warp_max64(best);
@@ -430,7 +439,7 @@ consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1,
     if (k < p.vocab) {
       const float xa = to_f32(za[k]);
       const float d = expf(xa * inv_t - la) - expf(to_f32(zd[k]) * inv_t - ld);
-      if (d > 0.f) best = umax64(best, order_key(logf(d) + gumbel(word(w, e)), k));
+      if (d > 0.f) best = umax64(best, order_key(log2f(d) + gumbel2(word(w, e)), k));
       bmax = umax64(bmax, order_key(xa, k));
     }
   }
