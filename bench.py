@@ -836,12 +836,15 @@ def main():
     ap.add_argument("--attn-batch", type=int, default=8,
                     help="sequences of the --kernel attn case (8: larger than L2; 1: the "
                          "round's call)")
-    ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead", "proj"], default=None,
+    ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead", "proj", "argmax",
+                                         "projround"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
                          "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
                          "the stochastic round's kernels one at a time; lmhead: the LM head "
                          "with the argmax in its epilogue against GEMM + argmax; proj: the "
-                         "attention block's projections alone")
+                         "attention block's projections alone; argmax: the vocabulary argmax "
+                         "alone; projround: the Qwen3-8B round with the projections and the "
+                         "LM head on the path")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel == "attn":
@@ -854,6 +857,19 @@ def main():
         return lm_head_kernel(args)
     if args.kernel == "proj":
         return projection_kernels(args)
+    if args.kernel == "argmax":
+        import torch
+        hbm, _ = peaks()
+        print(json.dumps({"kernel": "vocab_argmax",
+                          **argmax_leg(torch.device("cuda", 0), hbm, reps=args.steps)}))
+        return
+    if args.kernel == "projround":
+        import torch
+        hbm, _ = peaks()
+        print(json.dumps({"kernel": "projected_round",
+                          **projected_round_leg(torch.device("cuda", 0), hbm, steps=args.steps,
+                                                warmup=args.warmup)}))
+        return
 
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
