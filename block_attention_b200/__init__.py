@@ -87,6 +87,7 @@ EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_lm_head_argmax", "orthrus_lm_head_argmax_workspace",
            "orthrus_lm_head_argmax_plan",
            "orthrus_linear_tc", "orthrus_linear_tc_workspace", "orthrus_linear_tc_plan",
+           "orthrus_rope_table", "orthrus_linear_tc_qkv_rope",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
            "orthrus_swiglu", "orthrus_block_tokens")
@@ -142,8 +143,11 @@ def lib() -> ctypes.CDLL:
         L.orthrus_linear_tc_workspace.argtypes = [i32, i32, i32]
         L.orthrus_linear_tc_workspace.restype = sz
         L.orthrus_linear_tc_plan.argtypes = [i32, i32, i32, i32, vp]
-        L.orthrus_linear_tc.argtypes = [i32, vp, i32, i32, i64, vp, i32, vp, vp, i64, vp, vp, sz,
-                                        vp]
+        L.orthrus_linear_tc.argtypes = [i32, vp, i32, i32, i64, vp, i32, vp, vp, i64, vp, i64,
+                                        vp, vp, sz, vp]
+        L.orthrus_rope_table.argtypes = [vp, i32, i32, i32, c.c_double, vp, vp]
+        L.orthrus_linear_tc_qkv_rope.argtypes = [i32, vp, i32, i32, i64, vp, i32, i32, i32, vp,
+                                                 vp, vp, vp, vp, i64, vp, vp, sz, vp]
         L.orthrus_lm_head_argmax_plan.argtypes = [i32, i32, i32, i32, vp]
         L.orthrus_lm_head_argmax_workspace.argtypes = [i32]
         L.orthrus_lm_head_argmax_workspace.restype = sz
@@ -483,11 +487,64 @@ def lm_head_argmax(h, w, *, idx=None, maxval=None, err=None, workspace=None, str
     return idx
 
 
-def linear_tc(x, w, *, residual=None, out=None, err=None, workspace=None, stream=None):
+def rope_table(ctx_lens, B, blk, hd, theta, *, out=None, stream=None):
+    """float32 [B*blk, hd/2, 2] (cos, sin) of RoPE at positions ctx_lens[b] + j
+    (orthrus_rope_table)."""
+    _dev(out)
+    if not ctx_lens.is_cuda or ctx_lens.dtype != torch.int32:
+        raise ValueError("ctx_lens must be an int32 CUDA tensor")
+    if out is None:
+        out = torch.empty(B * blk, hd // 2, 2, dtype=torch.float32, device=ctx_lens.device)
+    if out.numel() != B * blk * hd or not out.is_contiguous() or out.dtype != torch.float32:
+        raise ValueError("out must be contiguous float32 with B*blk*hd elements")
+    _check("orthrus_rope_table", lib().orthrus_rope_table(
+        _ptr(ctx_lens), B, blk, hd, ctypes.c_double(theta), _ptr(out), _stream(stream)))
+    return out
+
+
+def _l2_hint(t):
+    """(pointer, bytes) of an optional L2 warm-up hint tensor."""
+    if t is None:
+        return None, 0
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("l2_next must be a contiguous CUDA tensor")
+    return _ptr(t), t.numel() * t.element_size() // 16 * 16
+
+
+def linear_tc_qkv_rope(x, w, Hq, Hkv, cos_sin, *, q, k, v, l2_next=None, err=None,
+                       workspace=None, stream=None):
+    """The QKV projection of x (bf16 [rows, K]) by w (bf16 [(Hq + 2 Hkv) * 128, K])
+    with RoPE (table `cos_sin` from rope_table) and the head split in its
+    epilogue: q [rows, Hq, 128], k / v [rows, Hkv, 128] (see orthrus.h).
+    l2_next: a tensor a later call reads, to warm L2 with (a hint)."""
+    _dev(w, cos_sin, q, k, v, err)
+    if not x.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (no CPU path)")
+    if x.dim() != 2 or w.dim() != 2 or x.stride(1) != 1 or not w.is_contiguous():
+        raise ValueError("x must be 2-D with unit column stride, w 2-D contiguous")
+    rows, K = x.shape
+    hd = 128
+    N = (Hq + 2 * Hkv) * hd
+    if tuple(w.shape) != (N, K):
+        raise ValueError("w must be [(Hq + 2 Hkv) * 128, K]")
+    for t, h in ((q, Hq), (k, Hkv), (v, Hkv)):
+        if t.numel() != rows * h * hd or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous [rows, heads, 128]")
+    buf = _ws(workspace, x.device, "linear").get(lib().orthrus_linear_tc_workspace(rows, K, N))
+    hp, hb = _l2_hint(l2_next)
+    _check("orthrus_linear_tc_qkv_rope", lib().orthrus_linear_tc_qkv_rope(
+        _dtype(x), _ptr(x), rows, K, x.stride(0), _ptr(w), Hq, Hkv, hd, _ptr(cos_sin), _ptr(q),
+        _ptr(k), _ptr(v), hp, hb, _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
+    return q, k, v
+
+
+def linear_tc(x, w, *, residual=None, out=None, l2_next=None, err=None, workspace=None,
+              stream=None):
     """bf16 [rows, N] = x @ w.T on the tensor cores (plus the residual, each
     sum rounded to bf16 first; see orthrus.h).  x bf16 [rows, K] (unit
     column stride), w bf16 [N, K] contiguous, residual/out bf16 [rows, N]
-    with unit column stride (out may be the residual)."""
+    with unit column stride (out may be the residual).  l2_next: a tensor a
+    later call reads, to warm L2 with (a hint)."""
     _dev(w, residual, out, err)
     if not x.is_cuda:
         raise ValueError("tensors must be on a CUDA device (no CPU path)")
@@ -504,7 +561,8 @@ def linear_tc(x, w, *, residual=None, out=None, err=None, workspace=None, stream
     if residual is not None and (residual.shape != (rows, N) or residual.stride() != out.stride()):
         raise ValueError("residual must be laid out like out")
     buf = _ws(workspace, x.device, "linear").get(lib().orthrus_linear_tc_workspace(rows, K, N))
+    hp, hb = _l2_hint(l2_next)
     _check("orthrus_linear_tc", lib().orthrus_linear_tc(
         _dtype(x), _ptr(x), rows, K, x.stride(0), _ptr(w), N, _ptr(residual), _ptr(out),
-        out.stride(0), _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
+        out.stride(0), hp, hb, _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
     return out

@@ -39,4 +39,23 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// RoPE (rotary position embedding) pieces shared by the stand-alone RoPE
+// kernel and the QKV projection's epilogue, so that both give identical
+// bits: the angle pos * theta^(-2i/hd) with its cosine and sine in double,
+// rounded to float; the rotation of the pair (x1, x2) = (x[i], x[i + hd/2])
+// in float with every rounding explicit (no contraction left to the
+// compiler):  x1' = x1 c - x2 s,  x2' = x2 c + x1 s.
+__device__ __forceinline__ float2 rope_cos_sin(int64_t pos, int i, int hd, double theta) {
+  const double ang = (double)pos * pow(theta, -2.0 * i / hd);
+  double sn, cn;
+  sincos(ang, &sn, &cn);
+  return make_float2((float)cn, (float)sn);
+}
+__device__ __forceinline__ float rope_first(float x1, float x2, float2 cs) {
+  return __fmaf_rn(x1, cs.x, -__fmul_rn(x2, cs.y));
+}
+__device__ __forceinline__ float rope_second(float x1, float x2, float2 cs) {
+  return __fmaf_rn(x2, cs.x, __fmul_rn(x1, cs.y));
+}
+
 }  // namespace orthrus

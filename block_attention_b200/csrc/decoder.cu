@@ -353,11 +353,9 @@ qkv_rope_kernel(const T* __restrict__ qkv, int blk, int Hq, int Hkv, int hd,
     }
     if (!table) {
       for (int i = threadIdx.x; i < half; i += kRopeThreads) {
-        const double ang = (double)pos * pow(theta, -2.0 * i / hd);
-        double sn, cn;
-        sincos(ang, &sn, &cn);
-        cs[i] = (float)cn;
-        cs[half + i] = (float)sn;
+        const float2 t = rope_cos_sin(pos, i, hd, theta);
+        cs[i] = t.x;
+        cs[half + i] = t.y;
       }
       __syncthreads();
       table = true;
@@ -370,10 +368,9 @@ qkv_rope_kernel(const T* __restrict__ qkv, int blk, int Hq, int Hkv, int hd,
         float y1[W], y2[W];
 #pragma unroll
         for (int e = 0; e < W; ++e) {
-          const float c = cs[i0 + e], s = cs[half + i0 + e];
-          const float x1 = a[u][e], x2 = c2[u][e];
-          y1[e] = x1 * c - x2 * s;
-          y2[e] = x2 * c + x1 * s;
+          const float2 t = make_float2(cs[i0 + e], cs[half + i0 + e]);
+          y1[e] = rope_first(a[u][e], c2[u][e], t);
+          y2[e] = rope_second(a[u][e], c2[u][e], t);
         }
         T* dst = h < Hq ? q + ((int64_t)r * Hq + h) * hd : k + ((int64_t)r * Hkv + h - Hq) * hd;
         if constexpr (kVec) {

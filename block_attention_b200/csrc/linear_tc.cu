@@ -24,6 +24,12 @@
 //              accumulator (128 lanes = output features, rows in columns).
 //   warps 2-5  epilogue: each thread owns one output feature (TMEM lane) and
 //              reads its row of results 32 columns at a time.
+// QKV mode (orthrus_linear_tc_qkv_rope): the tile of 128 features is one head
+// of the fused QKV output; instead of y the epilogue writes q and k rotated by
+// RoPE (the pair (i, i + 64) of a head lies in one tile: the threads of
+// features n and n ^ 64 swap their bf16 values through shared memory) and v
+// as is, with the cos/sin table of orthrus_rope_table -- the same bits as
+// orthrus_linear_tc followed by orthrus_qkv_rope.
 // Every mbarrier wait is bounded: on a timeout the kernel records
 // ORTHRUS_ETIMEOUT, stops issuing, drains what it issued and still takes its
 // ticket, so it always terminates.
@@ -31,6 +37,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -48,6 +55,7 @@ constexpr int kMaxStages = 16;
 constexpr int kRingBudget = 208 * 1024;
 constexpr int kWBox = kTileN * 128;        // bytes of one weight box
 constexpr int kNumBars = 2 * kMaxStages + 2;
+constexpr int kXchgBytes = kTileN * 33 * 4;  // QKV mode: [128][33] floats
 
 struct __align__(64) LinParams {
   CUtensorMap tm_w;  // 2D (K, N), box (64, 128)
@@ -59,6 +67,13 @@ struct __align__(64) LinParams {
   int32_t* err;
   int R, Rp, N, ldy, tiles, ksplit, ksteps, stages, stage_bytes, tmem_cols;
   int kb;  // 64-wide K steps (weight box + x box each) per stage
+  // QKV mode (rope != null): q [R, Hq, 128], k / v [R, Hkv, 128] instead of y
+  const float2* rope;  // [R][64] (cos, sin)
+  __nv_bfloat16 *q, *k, *v;
+  int Hq, Hkv;
+  // L2 warm-up hint: after its own loads each CTA prefetches its share
+  const uint8_t* l2_next;
+  int64_t l2_next_bytes;
 };
 
 struct Bars {
@@ -90,6 +105,9 @@ struct Scalars {
   unsigned* tickets;
   int32_t* err;
   int R, Rp, N, ldy, ksplit, ksteps, stages, stage_bytes, tmem_cols, kb;
+  const float2* rope;
+  __nv_bfloat16 *q, *k, *v;
+  int Hq, Hkv;
 };
 
 template <typename T> __device__ __forceinline__ T* keep(T* v) {
@@ -109,6 +127,8 @@ __device__ __forceinline__ Scalars load_scalars(const LinParams& p) {
   c.R = keep(p.R); c.Rp = keep(p.Rp); c.N = keep(p.N); c.ldy = keep(p.ldy);
   c.ksplit = keep(p.ksplit); c.ksteps = keep(p.ksteps); c.stages = keep(p.stages);
   c.stage_bytes = keep(p.stage_bytes); c.tmem_cols = keep(p.tmem_cols); c.kb = keep(p.kb);
+  c.rope = keep(p.rope); c.q = keep(p.q); c.k = keep(p.k); c.v = keep(p.v);
+  c.Hq = keep(p.Hq); c.Hkv = keep(p.Hkv);
   return c;
 }
 
@@ -139,8 +159,80 @@ __device__ __forceinline__ void store_rows(const Scalars& c, int cb, int ng, con
   }
 }
 
+// What a chunk of rows (cb .. cb + 31) of feature n needs besides its sums:
+// the residual (plain mode) or the cos/sin of its rotation pair (QKV mode),
+// all loads in flight together.
+struct ChunkIn {
+  float res[32];
+  float2 cs[32];
+};
+__device__ __forceinline__ void load_chunk_in(const Scalars& c, int cb, int n, int ng,
+                                              ChunkIn& in) {
+  if (c.rope) {
+    const int nr = min(32, c.R - cb);
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      in.cs[j] = j < nr ? c.rope[(int64_t)(cb + j) * (kTileN / 2) + (n & (kTileN / 2 - 1))]
+                        : make_float2(0.f, 0.f);
+  } else {
+    load_residual(c, cb, ng, in.res);
+  }
+}
+
+// The chunk's outputs from its fp32 sums v[j].  Plain mode: y (store_rows).
+// QKV mode: the 128 threads of the tile (named barrier 1; every one of them
+// calls this, `live` says whether its values count) swap bf16 values with
+// the feature n ^ 64 through `xchg` ([128][33] floats), rotate, and store
+// to q / k (v: as is).
+__device__ __forceinline__ void finish_chunk(const Scalars& c, int tile, int cb, int n, bool live,
+                                             const float (&v)[32], const ChunkIn& in,
+                                             float* xchg) {
+  const int ng = tile * kTileN + n;
+  if (!c.rope) {
+    if (live && ng < c.N) store_rows(c, cb, ng, v, in.res);
+    return;
+  }
+  float y[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    y[j] = bf16_round(v[j]);  // the projection's bf16 value
+    xchg[n * 33 + j] = y[j];
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int nr = min(32, c.R - cb);
+  const int pn = n ^ (kTileN / 2);
+  const bool rot = tile < c.Hq + c.Hkv;
+  __nv_bfloat16* dst;
+  int pitch;  // elements between rows
+  if (tile < c.Hq) {
+    dst = c.q + (int64_t)tile * kTileN + n;
+    pitch = c.Hq * kTileN;
+  } else if (rot) {
+    dst = c.k + (int64_t)(tile - c.Hq) * kTileN + n;
+    pitch = c.Hkv * kTileN;
+  } else {
+    dst = c.v + (int64_t)(tile - c.Hq - c.Hkv) * kTileN + n;
+    pitch = c.Hkv * kTileN;
+  }
+  float o[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float yp = xchg[pn * 33 + j];
+    o[j] = !rot ? y[j]
+           : n < kTileN / 2 ? rope_first(y[j], yp, in.cs[j]) : rope_second(yp, y[j], in.cs[j]);
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // xchg free for the next chunk
+  if (live) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nr) dst[(int64_t)(cb + j) * pitch] = __float2bfloat16_rn(o[j]);
+  }
+}
+
+template <bool kQkv>
 __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_constant__ LinParams p) {
-  const Scalars c = load_scalars(p);
+  Scalars c = load_scalars(p);
+  if (!kQkv) c.rope = nullptr;  // plain mode: the compiler drops the QKV paths
   extern __shared__ uint8_t smem_raw[];
   // 1 KB aligned for the 128-byte swizzle; offset from smem_raw itself so
   // the compiler keeps the shared address space
@@ -154,6 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 8);
+  // QKV mode's swap area: the end of the ring, idle by the time it is used
+  float* xchg = reinterpret_cast<float*>(smem + ST * SB - kXchgBytes);
 
   const int tile = blockIdx.x / c.ksplit, ks = blockIdx.x % c.ksplit;
   const int k_beg = (int)((int64_t)ks * c.ksteps / c.ksplit);
@@ -235,6 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
       // every issued load lands before the CTA can exit
       for (int u = max(0, issued - ST); u < issued; ++u)
         if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(c.err, abort_flag);
+      // this CTA's share of the next call's weights into L2 (a hint: the
+      // loads are not waited for and change no result)
+      if (p.l2_next && p.l2_next_bytes > 0) {
+        const int64_t units = p.l2_next_bytes / 16, per = (units + gridDim.x - 1) / gridDim.x;
+        const int64_t beg = (int64_t)blockIdx.x * per, end = min(units, beg + per);
+        for (int64_t u0 = beg; u0 < end; u0 += 2048)  // 32 KB a request
+          ptx::bulk_prefetch_l2(p.l2_next + u0 * 16, (uint32_t)(min(end - u0, (int64_t)2048) * 16));
+      }
     }
   } else if (warp == 1) {
     // ================================================== MMA issuer
@@ -296,11 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(d[j]);
-        if (ok && ng < c.N) {
-          float res[32];
-          load_residual(c, cb, ng, res);
-          store_rows(c, cb, ng, v, res);
-        }
+        ChunkIn in;
+        if (ok && ng < c.N) load_chunk_in(c, cb, n, ng, in);
+        finish_chunk(c, tile, cb, n, ok, v, in, xchg);
       } else {
         // this feature's partial sums of rows cb .. cb + nc - 1, contiguous
 #pragma unroll
@@ -342,17 +442,17 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
       ptx::bulk_g2s(sbase + (uint32_t)s * blk_bytes, base + (int64_t)s * kTileN * RP4, blk_bytes,
                     bars.red_full());
   }
-  // the first rows' residual comes in while the partials do
+  // the first rows' residual (or cos/sin) comes in while the partials do
   const int n = threadIdx.x, ng = n0 + n;
-  float res[32];
-  if (n < kTileN && ng < c.N) load_residual(c, 0, ng, res);
-  if (!ptx::mbar_wait(bars.red_full(), 0)) {
-    set_err(c.err, ORTHRUS_ETIMEOUT);
-  } else if (n < kTileN) {
+  ChunkIn in;
+  if (n < kTileN && ng < c.N) load_chunk_in(c, 0, n, ng, in);
+  const bool got = ptx::mbar_wait(bars.red_full(), 0);
+  if (!got) set_err(c.err, ORTHRUS_ETIMEOUT);
+  if (n < kTileN) {  // every thread of the tile: QKV mode's barriers
     const float* st = reinterpret_cast<const float*>(smem) + n * RP4;
-    if (ng < c.N) {
+    {
       for (int cb = 0; cb < c.Rp; cb += 32) {
-        if (cb > 0) load_residual(c, cb, ng, res);
+        if (cb > 0 && ng < c.N) load_chunk_in(c, cb, n, ng, in);
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -360,13 +460,13 @@ __global__ void __launch_bounds__(kThreads, 1) linear_tc_kernel(const __grid_con
           const float* src = st + (int64_t)sp * kTileN * RP4 + cb;
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
-            if (cb + j < c.Rp) {
+            if (got && cb + j < c.Rp) {
               const float4 f = *reinterpret_cast<const float4*>(src + j);
               v[j] += f.x; v[j + 1] += f.y; v[j + 2] += f.z; v[j + 3] += f.w;
             }
           }
         }
-        store_rows(c, cb, ng, v, res);
+        finish_chunk(c, tile, cb, n, got, v, in, xchg);
       }
     }
   }
@@ -419,7 +519,7 @@ struct Plan {
 // Launch shape for rows x K x N on `sms` SMs: 128-feature tiles, the K range
 // of each split over enough CTAs to fill the SMs (at most one 64-wide K step
 // less than an even share each), a ring of as many stages as fit.
-Plan plan(int rows, int K, int N, int sms, int kb) {
+Plan plan(int rows, int K, int N, int sms, int kb, bool qkv = false) {
   Plan q;
   q.Rp = (rows + 15) / 16 * 16;
   q.ksteps = K / kStepK;
@@ -434,7 +534,9 @@ Plan plan(int rows, int K, int N, int sms, int kb) {
   // no more than the ring can stage for the last CTA's sum
   q.ksplit = q.tiles >= sms ? 1 : sms / q.tiles;
   q.ksplit = min(q.ksplit, min(q.ksteps, 16));
-  q.ksplit = max(1, min(q.ksplit, q.stages * q.stage_bytes / ((q.Rp + 4) * kTileN * 4)));
+  // (QKV mode keeps the ring's last kXchgBytes for its swap area)
+  q.ksplit = max(1, min(q.ksplit, (q.stages * q.stage_bytes - (qkv ? kXchgBytes : 0)) /
+                                      ((q.Rp + 4) * kTileN * 4)));
   q.smem = q.stages * q.stage_bytes + kNumBars * 8 + 16 + 1024;
   q.tmem_cols = 32;
   while (q.tmem_cols < q.Rp) q.tmem_cols *= 2;
@@ -450,7 +552,9 @@ int choose_kb(int rows) {
   return 1;
 }
 
-Plan plan(int rows, int K, int N, int sms) { return plan(rows, K, N, sms, choose_kb(rows)); }
+Plan plan(int rows, int K, int N, int sms, bool qkv = false) {
+  return plan(rows, K, N, sms, choose_kb(rows), qkv);
+}
 
 size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
 
@@ -461,16 +565,73 @@ size_t workspace_bytes(int rows, int K, int N) {
   return round256((int64_t)q.tiles * 4) + (size_t)parts;
 }
 
+// cos/sin table of RoPE for the rows of the blocks: row r = b * blk + j at
+// position ctx_lens[b] + j, frequencies i < hd / 2 (the values the
+// stand-alone RoPE kernel computes).
+__global__ void rope_table_kernel(const int32_t* __restrict__ ctx_lens, int blk, int hd,
+                                  double theta, float2* __restrict__ table) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
+  const int r = blockIdx.x, half = hd / 2;
+  const int64_t pos = (int64_t)ctx_lens[r / blk] + r % blk;
+  for (int i = threadIdx.x; i < half; i += blockDim.x)
+    table[(int64_t)r * half + i] = rope_cos_sin(pos, i, hd, theta);
+}
+
 bool prepare() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (dev >= 0 && dev < 64 && done[dev]) return true;
-  if (cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(linear_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           227 * 1024) != cudaSuccess ||
+      cudaFuncSetAttribute(linear_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            227 * 1024) != cudaSuccess)
     return false;
   if (dev >= 0 && dev < 64) done[dev] = true;
   return true;
+}
+
+// Common tail of the entry points: plan, tensor maps, workspace, launch.
+int launch_linear(LinParams& p, const void* x, int rows, int K, int64_t ldx, const void* w,
+                  int N, bool qkv, const void* l2_next, int64_t l2_next_bytes, int32_t* err,
+                  void* workspace, size_t workspace_bytes_given, orthrus_stream_t stream) {
+  if (l2_next_bytes < 0 || (l2_next && (reinterpret_cast<uintptr_t>(l2_next) % 16 ||
+                                        l2_next_bytes % 16)))
+    return ORTHRUS_EINVAL;
+  p.l2_next = l2_next_bytes > 0 ? static_cast<const uint8_t*>(l2_next) : nullptr;
+  p.l2_next_bytes = p.l2_next ? l2_next_bytes : 0;
+  if (!workspace || workspace_bytes_given < workspace_bytes(rows, K, N) ||
+      reinterpret_cast<uintptr_t>(workspace) % 256)
+    return ORTHRUS_EWORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return ORTHRUS_ECUDA;
+  if (!prepare()) return ORTHRUS_ECUDA;
+  const Plan q = plan(rows, K, N, sms, qkv);
+  if (!encode_2d(&p.tm_w, w, K, N, (int64_t)K * 2, kTileN) ||
+      !encode_2d(&p.tm_x, x, K, rows, ldx * 2, q.Rp))
+    return ORTHRUS_ECUDA;
+  char* ws = static_cast<char*>(workspace);
+  p.tickets = reinterpret_cast<unsigned*>(ws);
+  p.part = reinterpret_cast<float*>(ws + round256((int64_t)q.tiles * 4));
+  p.err = err;
+  p.R = rows; p.Rp = q.Rp; p.N = N;
+  p.tiles = q.tiles; p.ksplit = q.ksplit; p.ksteps = q.ksteps; p.stages = q.stages;
+  p.stage_bytes = q.stage_bytes; p.tmem_cols = q.tmem_cols; p.kb = q.kb;
+
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(q.tiles * q.ksplit);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = q.smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  const cudaError_t e = qkv ? cudaLaunchKernelEx(&cfg, linear_tc_kernel<true>, p)
+                            : cudaLaunchKernelEx(&cfg, linear_tc_kernel<false>, p);
+  return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
 }
 
 }  // namespace
@@ -502,8 +663,8 @@ size_t orthrus_linear_tc_workspace(int32_t rows, int32_t K, int32_t N) {
 
 int orthrus_linear_tc(int32_t dtype, const void* x, int32_t rows, int32_t K, int64_t ldx,
                       const void* w, int32_t N, const void* residual, void* y, int64_t ldy,
-                      int32_t* err, void* workspace, size_t workspace_bytes_given,
-                      orthrus_stream_t stream) {
+                      const void* l2_next, int64_t l2_next_bytes, int32_t* err,
+                      void* workspace, size_t workspace_bytes_given, orthrus_stream_t stream) {
   if (dtype != ORTHRUS_F32 && dtype != ORTHRUS_BF16) return ORTHRUS_EINVAL;
   if (rows < 0 || K <= 0 || N <= 0 || ldx < K || ldy < N) return ORTHRUS_EINVAL;
   if (dtype != ORTHRUS_BF16) return ORTHRUS_EUNSUPPORTED;
@@ -513,39 +674,65 @@ int orthrus_linear_tc(int32_t dtype, const void* x, int32_t rows, int32_t K, int
   if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w) % 16 ||
       reinterpret_cast<uintptr_t>(y) % 2 || reinterpret_cast<uintptr_t>(residual) % 2)
     return ORTHRUS_EINVAL;
-  if (!workspace || workspace_bytes_given < workspace_bytes(rows, K, N) ||
-      reinterpret_cast<uintptr_t>(workspace) % 256)
-    return ORTHRUS_EWORKSPACE;
-  const int sms = sm_count();
-  if (sms <= 0) return ORTHRUS_ECUDA;
-  if (!prepare()) return ORTHRUS_ECUDA;
-  const Plan q = plan(rows, K, N, sms);
-  LinParams p;
-  if (!encode_2d(&p.tm_w, w, K, N, (int64_t)K * 2, kTileN) ||
-      !encode_2d(&p.tm_x, x, K, rows, ldx * 2, q.Rp))
-    return ORTHRUS_ECUDA;
-  char* ws = static_cast<char*>(workspace);
-  p.tickets = reinterpret_cast<unsigned*>(ws);
-  p.part = reinterpret_cast<float*>(ws + round256((int64_t)q.tiles * 4));
+  LinParams p = {};
   p.residual = static_cast<const __nv_bfloat16*>(residual);
   p.y = static_cast<__nv_bfloat16*>(y);
-  p.err = err;
-  p.R = rows; p.Rp = q.Rp; p.N = N; p.ldy = (int)ldy;
-  p.tiles = q.tiles; p.ksplit = q.ksplit; p.ksteps = q.ksteps; p.stages = q.stages;
-  p.stage_bytes = q.stage_bytes; p.tmem_cols = q.tmem_cols; p.kb = q.kb;
+  p.ldy = (int)ldy;
+  return launch_linear(p, x, rows, K, ldx, w, N, false, l2_next, l2_next_bytes, err, workspace,
+                       workspace_bytes_given, stream);
+}
 
+int orthrus_rope_table(const int32_t* ctx_lens, int32_t B, int32_t blk, int32_t hd, double theta,
+                       float* cos_sin, orthrus_stream_t stream) {
+  if (B < 0 || blk <= 0 || hd <= 0 || hd % 2 || !(theta > 0.0)) return ORTHRUS_EINVAL;
+  if (B == 0) return ORTHRUS_OK;
+  if (!ctx_lens || !cos_sin || reinterpret_cast<uintptr_t>(cos_sin) % 8) return ORTHRUS_EINVAL;
+  const int64_t rows = (int64_t)B * blk;
+  if (rows > 2147483647LL) return ORTHRUS_EUNSUPPORTED;
   cudaLaunchAttribute pdl;
   pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl.val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(q.tiles * q.ksplit);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = q.smem;
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3((unsigned)std::min(hd / 2, 256));
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cfg.attrs = &pdl;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, linear_tc_kernel, p) == cudaSuccess ? ORTHRUS_OK
-                                                                        : ORTHRUS_ECUDA;
+  return cudaLaunchKernelEx(&cfg, rope_table_kernel, ctx_lens, (int)blk, (int)hd, theta,
+                            reinterpret_cast<float2*>(cos_sin)) == cudaSuccess
+             ? ORTHRUS_OK
+             : ORTHRUS_ECUDA;
+}
+
+int orthrus_linear_tc_qkv_rope(int32_t dtype, const void* x, int32_t rows, int32_t K,
+                               int64_t ldx, const void* w, int32_t Hq, int32_t Hkv, int32_t hd,
+                               const float* cos_sin, void* q, void* k, void* v,
+                               const void* l2_next, int64_t l2_next_bytes, int32_t* err,
+                               void* workspace, size_t workspace_bytes_given,
+                               orthrus_stream_t stream) {
+  if (dtype != ORTHRUS_F32 && dtype != ORTHRUS_BF16) return ORTHRUS_EINVAL;
+  if (rows < 0 || K <= 0 || ldx < K || Hq <= 0 || Hkv <= 0 || hd <= 0 || hd % 2)
+    return ORTHRUS_EINVAL;
+  if (dtype != ORTHRUS_BF16 || hd != kTileN) return ORTHRUS_EUNSUPPORTED;
+  if (rows == 0) return ORTHRUS_OK;
+  if (rows > kMaxRows || K % kStepK || ldx % 8) return ORTHRUS_EUNSUPPORTED;
+  if (!x || !w || !cos_sin || !q || !k || !v) return ORTHRUS_EINVAL;
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(w) % 16 ||
+      reinterpret_cast<uintptr_t>(cos_sin) % 8 || reinterpret_cast<uintptr_t>(q) % 2 ||
+      reinterpret_cast<uintptr_t>(k) % 2 || reinterpret_cast<uintptr_t>(v) % 2)
+    return ORTHRUS_EINVAL;
+  const int64_t N = (int64_t)(Hq + 2 * Hkv) * hd;
+  if (N > 2147483647LL) return ORTHRUS_EUNSUPPORTED;
+  LinParams p = {};
+  p.rope = reinterpret_cast<const float2*>(cos_sin);
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.k = static_cast<__nv_bfloat16*>(k);
+  p.v = static_cast<__nv_bfloat16*>(v);
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.ldy = (int)N;
+  return launch_linear(p, x, rows, K, ldx, w, (int)N, true, l2_next, l2_next_bytes, err,
+                       workspace, workspace_bytes_given, stream);
 }
 
 }  // extern "C"

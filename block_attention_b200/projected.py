@@ -11,8 +11,9 @@ update):
   per view v (0 = diffusion over [anchor, MASK x (blk-1)], 1 = AR verify over
   [anchor, d0 .. d_{blk-2}]):
       x = embed[block tokens]
-      per layer l:  h = RMSNorm(x) ; qkv = h Wqkv[v, l]^T        (tensor cores)
-                    q, k, v = RoPE split of qkv at positions n .. n+blk-1
+      per layer l:  h = RMSNorm(x)
+                    q, k, v = RoPE split of h Wqkv[v, l]^T at positions
+                              n .. n+blk-1  (tensor cores, RoPE in the epilogue)
                     a = block attention over cache_l ‖ block k/v  (mask of v)
                     x = x + a Wo[v, l]^T                          (tensor cores)
       tokens_v = argmax_V RMSNorm(x) E^T                (LM head, argmax fused)
@@ -24,23 +25,35 @@ path is.  The embedding doubles as the LM head (tied).  Weights are random
 (N(0, 0.02), norm gains 1 + N(0, 0.02)) in bf16; the caches are N(0, 1).  Every
 kernel is this library's, through the C ABI, on the current stream; the round
 is captured as one CUDA graph.
+
+L2 warm-up (`prefetch`, off by default): "weights" has each QKV projection
+warm L2 with the same layer's output-projection weights (34 MB, needed one
+attention later) and each output projection with the next layer's QKV
+weights (50 MB); "kv" has each attention warm L2 with the next layer's
+cache; "both".  Measured at the Qwen3-8B shape every variant was slower
+than none (4.76 ms per round; "kv" 4.96, "weights" 5.08-5.14, "both"
+5.38): the prefetches compete with the stream on the critical path.
 """
 from __future__ import annotations
 
 import torch
 
 from . import (ATTN_EARLY_KV, BIDIR_BLOCK, CAUSAL_VERIFY, Workspace, block_attn,
-               block_tokens, consensus, embed, kv_commit, linear_tc, lm_head_argmax, rmsnorm,
-               qkv_rope)
+               block_tokens, consensus, embed, kv_commit, linear_tc, linear_tc_qkv_rope,
+               lm_head_argmax, rmsnorm, rope_table)
 
 
 class ProjectedRound:
     def __init__(self, *, layers=36, Hq=32, Hkv=8, D=128, d_model=4096, blk=32, vocab=151936,
-                 ctx=8192, seed=0, device="cuda", eps=1e-6, theta=1e6, prefetch=True):
+                 ctx=8192, seed=0, device="cuda", eps=1e-6, theta=1e6, prefetch=None):
         self.dev = torch.device(device)
         self.L, self.Hq, self.Hkv, self.D, self.d, self.blk, self.V = (
             layers, Hq, Hkv, D, d_model, blk, vocab)
-        self.ctx, self.eps, self.theta, self.prefetch = ctx, eps, theta, prefetch
+        if prefetch is True:
+            prefetch = "weights"
+        if prefetch not in (None, False, "weights", "kv", "both"):
+            raise ValueError("prefetch: None, 'weights', 'kv' or 'both'")
+        self.ctx, self.eps, self.theta, self.prefetch = ctx, eps, theta, prefetch or None
         self.cap = ctx + blk
         dev, bf = self.dev, torch.bfloat16
         g = torch.Generator(device=dev).manual_seed(seed)
@@ -66,6 +79,7 @@ class ProjectedRound:
         self.x = torch.empty(blk, d_model, dtype=bf, device=dev)
         self.h = torch.empty_like(self.x)
         self.qkv = torch.empty(blk, nqkv, dtype=bf, device=dev)
+        self.rope_cs = torch.empty(blk, D // 2, 2, dtype=torch.float32, device=dev)
         self.q = torch.empty(1, blk, Hq, D, dtype=bf, device=dev)
         self.k_blk = torch.empty(2, layers, 1, blk, Hkv, D, dtype=bf, device=dev)
         self.v_blk = torch.empty_like(self.k_blk)
@@ -84,21 +98,27 @@ class ProjectedRound:
         draft = None if v == 0 else self.tok_out[0].view(1, blk)
         block_tokens(self.anchor, draft, blk, self.mask_id, out=self.tok_in[v])
         embed(self.embed_w, self.tok_in[v].view(-1), out=self.x, err=self.err)
+        # the block's positions are the same in every layer: one cos/sin table
+        rope_table(self.ctx_lens, 1, blk, self.D, self.theta, out=self.rope_cs)
         mode = BIDIR_BLOCK if v == 0 else CAUSAL_VERIFY
         for l in range(L):
             rmsnorm(self.x, self.gain[l], self.eps, out=self.h)
-            linear_tc(self.h, self.wqkv[v, l], out=self.qkv, err=self.err,
-                      workspace=self.ws["linear"])
-            qkv_rope(self.qkv, self.ctx_lens, 1, blk, self.Hq, self.Hkv, self.D, self.theta,
-                     q=self.q, k=self.k_blk[v, l], v=self.v_blk[v, l])
+            w_pf = self.prefetch in ("weights", "both")
+            linear_tc_qkv_rope(self.h, self.wqkv[v, l], self.Hq, self.Hkv, self.rope_cs,
+                               q=self.q, k=self.k_blk[v, l], v=self.v_blk[v, l],
+                               l2_next=self.wo[v, l] if w_pf else None, err=self.err,
+                               workspace=self.ws["linear"])
             nxt = (l + 1) % L
-            # the kernel before the attention (RoPE) writes neither a cache nor
-            # the lengths: the cache may stream while it finishes
+            # the kernel before the attention (the QKV projection) writes
+            # neither a cache nor the lengths: the cache may stream while it
+            # finishes
             block_attn(self.q, self.k_blk[v, l], self.v_blk[v, l], self.k_cache[l],
                        self.v_cache[l], self.ctx_lens, mode, out=self.attn, max_ctx=self.ctx,
                        err=self.err, workspace=self.ws[f"attn{v}"], flags=ATTN_EARLY_KV,
-                       next_kv=(self.k_cache[nxt], self.v_cache[nxt]) if self.prefetch else None)
+                       next_kv=(self.k_cache[nxt], self.v_cache[nxt])
+                       if self.prefetch in ("kv", "both") else None)
             linear_tc(self.attn.view(blk, -1), self.wo[v, l], residual=self.x, out=self.x,
+                      l2_next=self.wqkv[v, l + 1] if w_pf and l + 1 < L else None,
                       err=self.err, workspace=self.ws["linear"])
         rmsnorm(self.x, self.gain_final, self.eps, out=self.h)
         lm_head_argmax(self.h, self.embed_w, idx=self.tok_out[v], err=self.err,
@@ -143,7 +163,7 @@ class ProjectedRound:
         return {"projection_weights": w, "kv_cache": kv, "lm_head": lm}
 
     def kernels_per_round(self) -> int:
-        # per view: block tokens, embed, per layer (norm, qkv, rope, attention
-        # (1 launch at the one-wave batch-1 shape), out), final norm, LM head;
-        # then consensus and commit
-        return 2 * (2 + 5 * self.L + 2) + 2
+        # per view: block tokens, embed, RoPE table, per layer (norm, QKV with
+        # RoPE, attention (1 launch at the one-wave batch-1 shape), out),
+        # final norm, LM head; then consensus and commit
+        return 2 * (3 + 4 * self.L + 2) + 2

@@ -392,6 +392,11 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
  * bounded wait inside the kernel gave up.  workspace:
  * orthrus_linear_tc_workspace(rows, K, N) bytes, 256-byte aligned, zeroed
  * once; every call leaves its ticket counters zero.  One launch.
+ * l2_next / l2_next_bytes (optional; NULL / 0 for none): a hint naming
+ * device memory a later call reads (say the next projection's weights);
+ * once its own loads are issued, each CTA prefetches its share of it into
+ * L2.  It changes no result.  Address and size multiples of 16, else
+ * ORTHRUS_EINVAL.
  * ---------------------------------------------------------------------- */
 size_t orthrus_linear_tc_workspace(int32_t rows, int32_t K, int32_t N);
 /* The launch for these sizes on a GPU with `sms` SMs (host only): out[0..8)
@@ -401,8 +406,38 @@ size_t orthrus_linear_tc_workspace(int32_t rows, int32_t K, int32_t N);
 int orthrus_linear_tc_plan(int32_t rows, int32_t K, int32_t N, int32_t sms, int32_t* out);
 int orthrus_linear_tc(int32_t dtype, const void* x, int32_t rows, int32_t K, int64_t ldx,
                       const void* w, int32_t N, const void* residual, void* y, int64_t ldy,
-                      int32_t* err, void* workspace, size_t workspace_bytes,
-                      orthrus_stream_t stream);
+                      const void* l2_next, int64_t l2_next_bytes, int32_t* err,
+                      void* workspace, size_t workspace_bytes, orthrus_stream_t stream);
+
+/* RoPE cos/sin table for the rows of B blocks of blk rows (row r = b*blk + j
+ * at absolute position ctx_lens[b] + j, read on the device):
+ *   cos_sin[(r * hd/2 + i) * 2 + 0] = cos(pos * theta^(-2i/hd)),  [.. + 1] = sin(..)
+ * for i < hd/2, the angle and its cosine and sine in double, rounded to
+ * float: the values orthrus_qkv_rope (orthrus_decoder.h) uses.  cos_sin:
+ * B*blk*hd floats, 8-byte aligned.  hd even, theta > 0.  One launch. */
+int orthrus_rope_table(const int32_t* ctx_lens, int32_t B, int32_t blk, int32_t hd, double theta,
+                       float* cos_sin, orthrus_stream_t stream);
+
+/* The QKV projection with RoPE and the head split in its epilogue (the input
+ * side of each layer's attention; explainer §二): for the rows r of x,
+ *   qkv[r, :] = bf16( sum_k x[r, k] w[n, k] ),  w [(Hq + 2 Hkv) * hd, K]
+ * as orthrus_linear_tc computes it, then
+ *   q[r, h, :] = RoPE(qkv[r, h*hd .. h*hd + hd)),          h < Hq
+ *   k[r, g, :] = RoPE(qkv[r, (Hq + g)*hd ..)),             g < Hkv
+ *   v[r, g, :] =      qkv[r, (Hq + Hkv + g)*hd ..)
+ * with the rotation of the pairs (i, i + hd/2) by cos_sin (orthrus_rope_table
+ * for the same rows) -- the same bits as orthrus_linear_tc followed by
+ * orthrus_qkv_rope, in one launch.  q [rows, Hq, hd], k and v [rows, Hkv, hd]
+ * dense bf16.  Limits: dtype ORTHRUS_BF16, hd == 128 (one 128-feature tile
+ * is one head; otherwise ORTHRUS_EUNSUPPORTED), the rest (the L2 hint
+ * included) as orthrus_linear_tc; workspace: orthrus_linear_tc_workspace(
+ * rows, K, (Hq + 2 Hkv) * hd) bytes, same rules. */
+int orthrus_linear_tc_qkv_rope(int32_t dtype, const void* x, int32_t rows, int32_t K,
+                               int64_t ldx, const void* w, int32_t Hq, int32_t Hkv, int32_t hd,
+                               const float* cos_sin, void* q, void* k, void* v,
+                               const void* l2_next, int64_t l2_next_bytes, int32_t* err,
+                               void* workspace, size_t workspace_bytes,
+                               orthrus_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 const char* orthrus_status_str(int status);

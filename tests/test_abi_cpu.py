@@ -367,9 +367,10 @@ def test_linear_tc_plan_and_rejections(L):
     vp = ctypes.c_void_p
     ws = L.orthrus_linear_tc_workspace(32, 4096, 6144)
     call = lambda dtype=1, x=256, rows=32, K=4096, ldx=4096, w=512, N=6144, y=1024, ldy=6144, \
-        wsp=2048, wsb=ws: L.orthrus_linear_tc(dtype, vp(x) if x else None, rows, K, ldx,
-                                              vp(w) if w else None, N, None, vp(y) if y else None,
-                                              ldy, None, vp(wsp) if wsp else None, wsb, None)
+        hint=0, hint_bytes=0, wsp=2048, wsb=ws: L.orthrus_linear_tc(
+            dtype, vp(x) if x else None, rows, K, ldx, vp(w) if w else None, N, None,
+            vp(y) if y else None, ldy, vp(hint) if hint else None, ctypes.c_int64(hint_bytes),
+            None, vp(wsp) if wsp else None, wsb, None)
     assert call(dtype=0) == -2           # fp32: unsupported
     assert call(dtype=5) == -1
     assert call(rows=0) == 0             # nothing to do
@@ -380,3 +381,34 @@ def test_linear_tc_plan_and_rejections(L):
     assert call(x=0) == -1 and call(w=0) == -1 and call(y=0) == -1
     assert call(x=264) == -1             # x not 16-byte aligned
     assert call(wsp=0) == -3 and call(wsb=ws - 1) == -3 and call(wsp=2056) == -3
+    # the L2 hint: 16-byte address and size, no negative size
+    assert call(hint=4104, hint_bytes=4096) == -1 and call(hint=4096, hint_bytes=100) == -1
+    assert call(hint=4096, hint_bytes=-16) == -1
+
+def test_qkv_rope_projection_and_table_rejections(L):
+    """Host-side checks of the QKV projection with RoPE in its epilogue and of
+    the RoPE table (nothing here reaches a launch)."""
+    vp = ctypes.c_void_p
+    ws = L.orthrus_linear_tc_workspace(32, 4096, 6144)
+    assert ws == L.orthrus_linear_tc_workspace(32, 4096, (32 + 2 * 8) * 128)
+    call = lambda dtype=1, x=256, rows=32, K=4096, ldx=4096, w=512, Hq=32, Hkv=8, hd=128, \
+        cs=1024, q=2048, k=4096, v=8192, wsp=16384, wsb=ws: L.orthrus_linear_tc_qkv_rope(
+            dtype, vp(x) if x else None, rows, K, ldx, vp(w) if w else None, Hq, Hkv, hd,
+            vp(cs) if cs else None, vp(q) if q else None, vp(k) if k else None,
+            vp(v) if v else None, None, ctypes.c_int64(0), None, vp(wsp) if wsp else None, wsb,
+            None)
+    assert call(dtype=0) == -2           # fp32: unsupported
+    assert call(hd=64) == -2             # a head must be one 128-feature tile
+    assert call(hd=127) == -1 and call(Hq=0) == -1 and call(Hkv=-1) == -1
+    assert call(rows=0) == 0
+    assert call(rows=129) == -2 and call(K=100, ldx=100) == -2
+    assert call(cs=0) == -1 and call(q=0) == -1 and call(k=0) == -1 and call(v=0) == -1
+    assert call(cs=1028) == -1           # the table holds float pairs: 8-byte aligned
+    assert call(x=264) == -1
+    assert call(wsp=0) == -3 and call(wsb=ws - 1) == -3
+    rt = lambda lens=256, B=1, blk=32, hd=128, theta=1e6, out=512: L.orthrus_rope_table(
+        vp(lens) if lens else None, B, blk, hd, ctypes.c_double(theta), vp(out) if out else None,
+        None)
+    assert rt(B=0) == 0
+    assert rt(lens=0) == -1 and rt(out=0) == -1 and rt(out=516) == -1
+    assert rt(hd=127) == -1 and rt(blk=0) == -1 and rt(theta=0.0) == -1 and rt(B=-1) == -1

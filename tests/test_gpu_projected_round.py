@@ -3,7 +3,9 @@
 a 1000-key context and a 16384-entry vocabulary, checked op by op against the
 float64 oracle on the GPU's own inputs: the QKV projection and the output
 projection with its residual (per row within the bf16 tolerance, the bf16
-rounding agreeing on nearly every element), the attention of both views (bf16 tolerance), the LM head's argmax
+rounding agreeing on nearly every element), the round's QKV projection with
+RoPE in its epilogue (the same bits as the projection followed by RoPE), the
+attention of both views (bf16 tolerance), the LM head's argmax
 (bit-exact wherever the top-2 gap exceeds the fp32 error scale), consensus and
 commit bit-exact; and the graph replay equals the eager round."""
 import numpy as np
@@ -36,13 +38,14 @@ def _check_projection(oracle_mod, x, w, y, residual=None):
 
 
 def test_projected_round_op_by_op(oracle_mod):
-    rnd = ProjectedRound(layers=2, ctx=1000, vocab=16384, seed=21, prefetch=True)
+    rnd = ProjectedRound(layers=2, ctx=1000, vocab=16384, seed=21, prefetch="both")
     blk, L = rnd.blk, rnd.L
     mode = {0: ba.BIDIR_BLOCK, 1: ba.CAUSAL_VERIFY}
     lens0 = rnd.ctx_base.cpu().numpy()
     kc0 = {l: _bits(rnd.k_cache[l]) for l in range(L)}
     vc0 = {l: _bits(rnd.v_cache[l]) for l in range(L)}
     rnd.ctx_lens.copy_(rnd.ctx_base)
+    table = ba.rope_table(rnd.ctx_lens, 1, blk, rnd.D, rnd.theta)
     for v in (0, 1):
         draft = None if v == 0 else rnd.tok_out[0].view(1, blk)
         ba.block_tokens(rnd.anchor, draft, blk, rnd.mask_id, out=rnd.tok_in[v])
@@ -55,6 +58,12 @@ def test_projected_round_op_by_op(oracle_mod):
             _check_projection(oracle_mod, h, rnd.wqkv[v, l], rnd.qkv)
             ba.qkv_rope(rnd.qkv, rnd.ctx_lens, 1, blk, rnd.Hq, rnd.Hkv, rnd.D, rnd.theta,
                         q=rnd.q, k=rnd.k_blk[v, l], v=rnd.v_blk[v, l])
+            fq, fk, fv = (torch.empty_like(t) for t in (rnd.q, rnd.k_blk[v, l], rnd.v_blk[v, l]))
+            ba.linear_tc_qkv_rope(h, rnd.wqkv[v, l], rnd.Hq, rnd.Hkv, table, q=fq, k=fk, v=fv,
+                                  err=rnd.err)
+            torch.cuda.synchronize()
+            assert torch.equal(fq, rnd.q) and torch.equal(fk, rnd.k_blk[v, l])
+            assert torch.equal(fv, rnd.v_blk[v, l])
             ba.block_attn(rnd.q, rnd.k_blk[v, l], rnd.v_blk[v, l], rnd.k_cache[l],
                           rnd.v_cache[l], rnd.ctx_lens, mode[v], out=rnd.attn, max_ctx=rnd.ctx,
                           err=rnd.err)

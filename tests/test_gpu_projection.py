@@ -73,3 +73,60 @@ def test_deterministic_and_workspace_left_zero():
     assert torch.equal(a, b)
     tiles = (6144 + 127) // 128
     assert int(ws.buf[:tiles * 4].count_nonzero()) == 0  # ticket counters back at zero
+
+
+@pytest.mark.parametrize("B,blk,Hq,Hkv,K", [(1, 32, 32, 8, 4096),   # the Qwen3-8B block
+                                            (3, 17, 4, 2, 640),     # ragged rows, one K split
+                                            (4, 32, 2, 1, 256),     # 128 rows: four row chunks
+                                            (2, 9, 3, 1, 64)])      # one K step: no split
+def test_qkv_rope_epilogue_equals_projection_then_rope(B, blk, Hq, Hkv, K):
+    """The QKV projection with RoPE and the head split in its epilogue gives
+    the same bits as the projection followed by the stand-alone RoPE kernel
+    (which the decoder tests check against the oracle's forward)."""
+    g = torch.Generator(device="cuda").manual_seed(B * 1000 + blk)
+    rows, hd, theta = B * blk, 128, 1e6
+    N = (Hq + 2 * Hkv) * hd
+    x = torch.randn(rows, K, generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    lens = torch.tensor([8192, 5, 77, 30000][:B], dtype=torch.int32, device="cuda")
+    table = ba.rope_table(lens, B, blk, hd, theta)
+    mk = lambda h: torch.empty(rows, h, hd, dtype=torch.bfloat16, device="cuda")
+    q, k, v = mk(Hq), mk(Hkv), mk(Hkv)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ba.linear_tc_qkv_rope(x, w, Hq, Hkv, table, q=q, k=k, v=v, err=err)
+    qkv = ba.linear_tc(x, w)
+    q2, k2, v2 = mk(Hq), mk(Hkv), mk(Hkv)
+    ba.qkv_rope(qkv, lens, B, blk, Hq, Hkv, hd, theta, q=q2, k=k2, v=v2)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(v, v2)
+    # the table holds the stand-alone kernel's angles: spot-check against float64
+    pos = (lens.cpu().numpy()[:, None] + np.arange(blk)[None]).reshape(-1)
+    ang = pos[:, None] * theta ** (-2.0 * np.arange(hd // 2) / hd)[None]
+    t = table.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(t[..., 0], np.cos(ang), atol=2e-7)
+    np.testing.assert_allclose(t[..., 1], np.sin(ang), atol=2e-7)
+
+
+def test_l2_hint_changes_nothing():
+    """The L2 warm-up hint of the projections is only a hint: with it the
+    outputs are as without it and the ticket counters return to zero."""
+    g = torch.Generator(device="cuda").manual_seed(77)
+    x = torch.randn(32, 1024, generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn(768, 1024, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    res = torch.randn(32, 768, generator=g, device="cuda").to(torch.bfloat16)
+    nxt = torch.randn(3, 1000003, generator=g, device="cuda")  # size not a multiple of the CTAs
+    ws = ba.Workspace("cuda")
+    a = ba.linear_tc(x, w, residual=res, workspace=ws)
+    b = ba.linear_tc(x, w, residual=res, l2_next=nxt, workspace=ws)
+    table = ba.rope_table(torch.tensor([100], dtype=torch.int32, device="cuda"), 1, 32, 128, 1e4)
+    mk = lambda h: torch.empty(32, h, 128, dtype=torch.bfloat16, device="cuda")
+    outs = []
+    for hint in (None, nxt):
+        q, k, v = mk(2), mk(2), mk(2)
+        ba.linear_tc_qkv_rope(x, w[:768], 2, 2, table, q=q, k=k, v=v, l2_next=hint, workspace=ws)
+        outs.append((q, k, v))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert all(torch.equal(s, t) for s, t in zip(*outs))
+    assert int(ws.buf[:(768 // 128) * 4].count_nonzero()) == 0  # ticket counters
