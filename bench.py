@@ -837,14 +837,15 @@ def main():
                     help="sequences of the --kernel attn case (8: larger than L2; 1: the "
                          "round's call)")
     ap.add_argument("--kernel", choices=["attn", "blk", "sample", "lmhead", "proj", "argmax",
-                                         "projround"], default=None,
+                                         "projround", "small"], default=None,
                     help="attn: time block attention alone on a case larger than L2 (for "
                          "profiling); blk: block-size sweep K in {4, 8, 16, 32}; sample: "
                          "the stochastic round's kernels one at a time; lmhead: the LM head "
                          "with the argmax in its epilogue against GEMM + argmax; proj: the "
                          "attention block's projections alone; argmax: the vocabulary argmax "
                          "alone; projround: the Qwen3-8B round with the projections and the "
-                         "LM head on the path")
+                         "LM head on the path; small: the tiny and Qwen3-1.7B attention "
+                         "configurations")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel == "attn":
@@ -862,6 +863,12 @@ def main():
         hbm, _ = peaks()
         print(json.dumps({"kernel": "vocab_argmax",
                           **argmax_leg(torch.device("cuda", 0), hbm, reps=args.steps)}))
+        return
+    if args.kernel == "small":
+        import torch
+        hbm, _ = peaks()
+        print(json.dumps({"kernel": "block_attn_small_configs",
+                          **small_config_legs(torch.device("cuda", 0), hbm)}))
         return
     if args.kernel == "projround":
         import torch

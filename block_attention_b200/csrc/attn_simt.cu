@@ -17,10 +17,13 @@
 //
 // Thread layout: four lanes per query row (row r = block row i * G + local
 // head), each lane holding D/4 of q and of the output accumulator; dims are
-// interleaved in float4 groups so a tile row read by a quad is one
-// conflict-free 64-byte segment.
+// interleaved in groups of four so a tile row read by a quad is one
+// contiguous segment.  K/V tiles come into shared memory by cp.async, two
+// tiles deep: the next tile's copies are in flight while the current one is
+// used (tiles past the keys are zero-filled, as before).
 #include "attn_simt.cuh"
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace orthrus {
 
@@ -37,8 +40,8 @@ attn_simt_split_kernel(const SimtParams p) {
   const int i = row_ok ? r / G : 0;
   const int h = g * G + (row_ok ? r % G : 0);
 
-  __shared__ __align__(16) float Ks[kSimtTile][D];
-  __shared__ __align__(16) float Vs[kSimtTile][D];
+  __shared__ __align__(16) T Ks[2][kSimtTile][D];
+  __shared__ __align__(16) T Vs[2][kSimtTile][D];
 
   const int n = p.ctx_lens[b];
   const bool bad = n < 0 || n > p.max_ctx;
@@ -66,23 +69,39 @@ attn_simt_split_kernel(const SimtParams p) {
   const T* vb = static_cast<const T*>(p.v_blk) + ((int64_t)b * p.blk * p.Hkv + g) * D;
   const int64_t blk_stride = (int64_t)p.Hkv * D;
 
-  for (int t0 = lo; t0 < hi; t0 += kSimtTile) {
-    __syncthreads();
-    for (int e = tid; e < kSimtTile * D / 4; e += blockDim.x) {
-      const int j = e / (D / 4), c = (e % (D / 4)) * 4;
+  // issue the 16-byte copies of the tile at t0 into buffer `buf`, as one group
+  constexpr int kVec = 16 / (int)sizeof(T);
+  auto issue = [&](int t0, int buf) {
+    for (int e = tid; e < kSimtTile * D / kVec; e += blockDim.x) {
+      const int j = e / (D / kVec), c = (e % (D / kVec)) * kVec;
       const int pos = t0 + j;
-      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
+      const T* ks = kc;
+      const T* vs = vc;
+      uint32_t bytes = 0;  // past the keys: zero-fill, nothing read
       if (pos < n) {
-        kv = load4(kc + (int64_t)pos * D + c);
-        vv = load4(vc + (int64_t)pos * D + c);
+        ks = kc + (int64_t)pos * D + c;
+        vs = vc + (int64_t)pos * D + c;
+        bytes = 16;
       } else if (pos < total) {
-        kv = load4(kb + (pos - n) * blk_stride + c);
-        vv = load4(vb + (pos - n) * blk_stride + c);
+        ks = kb + (pos - n) * blk_stride + c;
+        vs = vb + (pos - n) * blk_stride + c;
+        bytes = 16;
       }
-      *reinterpret_cast<float4*>(&Ks[j][c]) = kv;
-      *reinterpret_cast<float4*>(&Vs[j][c]) = vv;
+      ptx::cp_async16_zfill(ptx::smem_u32(&Ks[buf][j][c]), ks, bytes);
+      ptx::cp_async16_zfill(ptx::smem_u32(&Vs[buf][j][c]), vs, bytes);
     }
-    __syncthreads();
+    ptx::cp_async_commit();
+  };
+  if (lo < hi) issue(lo, 0);
+  int buf = 0;
+  for (int t0 = lo; t0 < hi; t0 += kSimtTile, buf ^= 1) {
+    if (t0 + kSimtTile < hi) {
+      issue(t0 + kSimtTile, buf ^ 1);  // its buffer was released by the last barrier
+      ptx::cp_async_wait<1>();
+    } else {
+      ptx::cp_async_wait<0>();
+    }
+    __syncthreads();  // every thread's copies of this tile have landed
 
     // Scores for every key of the tile (the quad shuffles need every lane); a row then
     // uses only its visible prefix [t0, row_end).
@@ -93,7 +112,7 @@ attn_simt_split_kernel(const SimtParams p) {
       float acc = 0.f;
 #pragma unroll
       for (int t = 0; t < kG; ++t) {
-        const float4 k4 = *reinterpret_cast<const float4*>(&Ks[j][16 * t + 4 * lane4]);
+        const float4 k4 = load4(&Ks[buf][j][16 * t + 4 * lane4]);
         acc = fmaf(q[4 * t], k4.x, acc);
         acc = fmaf(q[4 * t + 1], k4.y, acc);
         acc = fmaf(q[4 * t + 2], k4.z, acc);
@@ -120,7 +139,7 @@ attn_simt_split_kernel(const SimtParams p) {
           l += pj;
 #pragma unroll
           for (int t = 0; t < kG; ++t) {
-            const float4 v4 = *reinterpret_cast<const float4*>(&Vs[j][16 * t + 4 * lane4]);
+            const float4 v4 = load4(&Vs[buf][j][16 * t + 4 * lane4]);
             o[4 * t] = fmaf(pj, v4.x, o[4 * t]);
             o[4 * t + 1] = fmaf(pj, v4.y, o[4 * t + 1]);
             o[4 * t + 2] = fmaf(pj, v4.z, o[4 * t + 2]);
@@ -130,6 +149,7 @@ attn_simt_split_kernel(const SimtParams p) {
       }
       m = mn;
     }
+    __syncthreads();  // the buffer is free for the copies issued next iteration
   }
 
   if (!row_ok) return;

@@ -8,7 +8,7 @@
 
 namespace orthrus {
 
-constexpr int kSimtChunk = 256;  // keys per split (absolute positions)
+constexpr int kSimtChunk = 64;   // keys per split (absolute positions)
 constexpr int kSimtTile = 16;    // keys per tile (absolute positions)
 
 struct SimtParams {
