@@ -1,5 +1,5 @@
 // tc_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile
-// loads (no multicast), tcgen05 TMEM allocation / MMA / load / store, and
+// loads (each into this CTA only), tcgen05 TMEM allocation / MMA / load / store, and
 // cluster shared memory.  Formats of the shared-memory and instruction
 // descriptors follow the public PTX ISA (tcgen05 "matrix descriptors" and
 // "instruction descriptor" tables).
@@ -239,7 +239,7 @@ __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Bulk copy (TMA engine, no multicast) of `bytes` contiguous bytes from
+// Bulk copy (TMA engine, into this CTA only) of `bytes` contiguous bytes from
 // global to this CTA's shared memory, completing on `bar`.  Addresses
 // 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
