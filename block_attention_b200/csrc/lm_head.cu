@@ -11,22 +11,26 @@
 // contiguous range of vocabulary tiles of nv rows (nv chosen on the host so
 // the tiles spread evenly over the SMs: at vocabulary 151936, 176 rows when
 // four boxes per stage fit, else 208):
-//   warp 0     TMA producer: per stage kb consecutive 64-column boxes of the
-//              w slice (nv rows each, K-major, 128-byte swizzle) -- the HBM
-//              stream -- and the matching columns of h (L2-resident) into a
-//              ring of stages; more boxes per stage mean fewer handshakes per
-//              byte (4 where two such stages fit, else 2)
+//   warp 0     TMA producers: lane 0 streams per stage kb consecutive
+//              64-column boxes of the w slice (nv rows each, K-major, 128-byte
+//              swizzle) -- the HBM stream -- into the w ring; lane 1 the
+//              matching columns of h (L2-resident) into a separate, short h
+//              ring, whose slots are free again as soon as the copying warps
+//              have moved them into TMEM, so h takes little of the shared
+//              memory the w stream needs for its bytes in flight.  w never
+//              depends on the preceding kernel: its first stages are requested
+//              before the programmatic-dependency wait, h only after it
 //   warp 1     MMA issuer (one thread): per stage 4 kb MMAs of K = 16 with
 //              A = the stage's 64 kb columns of h from TMEM (128 lanes = hidden
 //              rows, zero past R) and B = the w slice from shared memory,
 //              N = nv, into one TMEM accumulator (the rest of TMEM holds the
 //              h ring)
 //   warps 2-5  per warp quadrant holding hidden rows: copy each stage's h
-//              columns from shared memory into a small TMEM ring ahead of the
+//              columns from the h ring into a small TMEM ring ahead of the
 //              MMAs, then for each finished tile scan the thread's row of D
 //              for its best (value, index), kept across the CTA's tiles; a
-//              stage's slot is free once the MMAs and the copying warps are
-//              done with it
+//              w stage is free once its MMAs are done, an h slot once it is
+//              copied
 // Operand A from TMEM leaves shared memory to the w stream: with A in shared
 // memory as well, the MMA issue rate, not HBM, bounded the kernel.
 // At the end each hidden row's CTA best goes to a 64-bit slot (value order,
@@ -54,10 +58,12 @@ constexpr int kThreads = 192;
 constexpr int kRowsMax = 128;           // hidden rows per call (UMMA M, TMEM lanes)
 constexpr int kStepK = 64;              // d elements per box (one 128-byte swizzle row)
 constexpr int kMaxStages = 12;
-constexpr int kRingBudget = 212 * 1024; // shared memory for the stage ring
+constexpr int kRingBudget = 220 * 1024; // shared memory for the w and h rings
 constexpr int kTmemCols = 512;
 constexpr int kMaxASlots = 8;
-constexpr int kNumBars = 2 * kMaxStages + 2 * kMaxASlots + 3;
+constexpr int kMaxHSlots = 4;           // h ring slots (kb boxes each)
+constexpr int kHBoxesAhead = 4;         // h boxes the h ring holds at least
+constexpr int kNumBars = 2 * kMaxStages + 2 * kMaxASlots + 2 * kMaxHSlots + 3;
 
 struct __align__(64) LmParams {
   CUtensorMap tm_w;                 // 2D (d, V), box (64, nv)
@@ -69,14 +75,17 @@ struct __align__(64) LmParams {
   int32_t* err;
   int R, V, nv, nvp, ksteps, tiles, stages, stage_bytes, w_bytes, aslots, a_col, writers, kb,
       kst, hb;  // kb boxes per stage, kst stages per tile, hb bytes of one h box
+  // w ring: stages x stage_bytes (= w_bytes, kb w boxes); h ring: hslots x
+  // h_bytes (kb h boxes)
+  int h_bytes, hslots;
 };
 
 struct Layout {
   int bars, misc, total;
 };
-__host__ __device__ inline Layout layout(int stages, int stage_bytes) {
+__host__ __device__ inline Layout layout(int stages, int stage_bytes, int h_bytes, int hslots) {
   Layout l;
-  l.bars = stages * stage_bytes;
+  l.bars = stages * stage_bytes + hslots * h_bytes;
   l.misc = l.bars + kNumBars * 8;
   l.total = l.misc + 16;
   return l;
@@ -92,6 +101,10 @@ struct Bars {
   __device__ uint32_t acc_full() const { return at(2 * kMaxStages + 2 * kMaxASlots); }
   __device__ uint32_t acc_empty() const { return at(2 * kMaxStages + 2 * kMaxASlots + 1); }
   __device__ uint32_t mma_done() const { return at(2 * kMaxStages + 2 * kMaxASlots + 2); }
+  __device__ uint32_t h_full(int j) const { return at(2 * kMaxStages + 2 * kMaxASlots + 3 + j); }
+  __device__ uint32_t h_empty(int j) const {
+    return at(2 * kMaxStages + 2 * kMaxASlots + 3 + kMaxHSlots + j);
+  }
 };
 
 __device__ __forceinline__ void record_timeout(int32_t* err, volatile int* abort_flag) {
@@ -124,7 +137,9 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned full_mask = 0xffffffffu;
   const int ST = p.stages, SB = p.stage_bytes, AS = p.aslots;
-  const Layout L = layout(ST, SB);
+  const int HS = p.hslots;
+  const Layout L = layout(ST, SB, p.h_bytes, HS);
+  const uint32_t hbase = (uint32_t)(ST * SB);  // the h ring follows the w ring
   const Bars bars{sbase + (uint32_t)L.bars};
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
@@ -141,7 +156,11 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
     *last_flag = 0;
     for (int s = 0; s < kMaxStages; ++s) {
       ptx::mbar_init(bars.full(s), 1);
-      ptx::mbar_init(bars.empty(s), 1 + (uint32_t)p.writers);  // MMA commit + copying warps
+      ptx::mbar_init(bars.empty(s), 1);  // the stage's MMA commit
+    }
+    for (int j = 0; j < kMaxHSlots; ++j) {
+      ptx::mbar_init(bars.h_full(j), 1);
+      ptx::mbar_init(bars.h_empty(j), (uint32_t)p.writers);  // every copying warp
     }
     for (int j = 0; j < kMaxASlots; ++j) {
       ptx::mbar_init(bars.a_full(j), (uint32_t)p.writers);
@@ -176,33 +195,60 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  ptx::griddep_launch_dependents();
 
-  if (warp == 0) {
-    // ================================================== TMA producer
-    if (lane == 0) {
+  if (warp == 0 && lane == 0) {
+    // ================================================== w producer
+    // the output embedding is never written by the preceding kernel: the
+    // first stages stream before the wait for it
+    auto issue_w = [&](int it) {
+      const int s = it % ST, t = t_beg + it / p.kst, k0 = (it % p.kst) * KB;
+      const uint32_t dst = sbase + (uint32_t)(s * SB);
+      ptx::mbar_expect_tx(bars.full(s), (uint32_t)SB);
+      for (int j = 0; j < KB; ++j)
+        ptx::tma_load_2d(dst + (uint32_t)(j * p.nv * 128), &p.tm_w, bars.full(s),
+                         (k0 + j) * kStepK, t * p.nv);
+    };
+    const int early = min(total, ST);
+    for (int it = 0; it < early; ++it) issue_w(it);
+    ptx::griddep_wait();
+    int it = early;
+    for (; it < total; ++it) {
+      if (*abort_flag) break;
+      if (!ptx::mbar_wait(bars.empty(it % ST), ((it / ST) & 1) ^ 1)) {
+        record_timeout(p.err, abort_flag);
+        break;
+      }
+      issue_w(it);
+    }
+    // every issued load lands before the CTA can exit
+    for (int u = max(0, it - ST); u < it; ++u)
+      if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(p.err, abort_flag);
+  } else if (warp == 0) {
+    ptx::griddep_wait();
+    if (lane == 1) {
+      // ================================================== h producer
       int it = 0;
       for (; it < total; ++it) {
         if (*abort_flag) break;
-        const int s = it % ST, t = t_beg + it / p.kst, k0 = (it % p.kst) * KB;
-        if (!ptx::mbar_wait(bars.empty(s), ((it / ST) & 1) ^ 1)) {
+        const int j = it % HS, k0 = (it % p.kst) * KB;
+        if (!ptx::mbar_wait(bars.h_empty(j), ((it / HS) & 1) ^ 1)) {
           record_timeout(p.err, abort_flag);
           break;
         }
-        const uint32_t dst = sbase + (uint32_t)(s * SB);
-        ptx::mbar_expect_tx(bars.full(s), (uint32_t)SB);
-        for (int j = 0; j < KB; ++j)
-          ptx::tma_load_2d(dst + (uint32_t)(j * p.nv * 128), &p.tm_w, bars.full(s),
-                           (k0 + j) * kStepK, t * p.nv);
-        for (int j = 0; j < KB; ++j)
-          ptx::tma_load_2d(dst + (uint32_t)(p.w_bytes + j * p.hb), &p.tm_h, bars.full(s),
-                           (k0 + j) * kStepK, 0);
+        const uint32_t dst = sbase + hbase + (uint32_t)(j * p.h_bytes);
+        ptx::mbar_expect_tx(bars.h_full(j), (uint32_t)p.h_bytes);
+        for (int b = 0; b < KB; ++b)
+          ptx::tma_load_2d(dst + (uint32_t)(b * p.hb), &p.tm_h, bars.h_full(j),
+                           (k0 + b) * kStepK, 0);
       }
-      // every issued load lands before the CTA can exit
-      for (int u = max(0, it - ST); u < it; ++u)
-        if (!ptx::mbar_wait(bars.full(u % ST), (u / ST) & 1)) record_timeout(p.err, abort_flag);
+      for (int u = max(0, it - HS); u < it; ++u)
+        if (!ptx::mbar_wait(bars.h_full(u % HS), (u / HS) & 1))
+          record_timeout(p.err, abort_flag);
     }
   } else if (warp == 1) {
     // ================================================== MMA issuer
+    ptx::griddep_wait();
     if (lane == 0) {
       const uint32_t id = ptx::idesc_bf16(kRowsMax, p.nv, false, false);
       bool ok = true;
@@ -242,8 +288,11 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
       ptx::tc_commit(bars.mma_done());
       if (!ptx::mbar_wait(bars.mma_done(), 0)) record_timeout(p.err, abort_flag);
     }
-  } else if (quad < p.writers) {
+  } else if (quad >= p.writers) {
+    ptx::griddep_wait();  // idle warp: it still takes part in the ticket's write-out
+  } else {
     // ================================================== h writer + epilogue
+    ptx::griddep_wait();
     const int r = quad * 32 + lane;  // hidden row of this thread
     const bool valid = r < p.R;
     float best_v = -INFINITY;
@@ -252,16 +301,15 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
     int it_w = 0;  // next h slice to copy (global stage index)
     for (int i = 0; ok && i < ntiles; ++i) {
       // this tile's slices, then the next tile's first ones: at most as many
-      // as both the slice ring and the stage ring hold, so that the TMEM slot
-      // and the stage of each are freed by MMAs of this tile, which do not
-      // wait on this tile's scan (one more would wait on an MMA of the next
-      // tile, which waits on that scan)
-      const int ahead = AS < ST ? AS : ST;
-      const int limit = min(min((i + 1) * p.kst + ahead, (i + 2) * p.kst), total);
+      // as the TMEM slice ring holds, so that the slot of each is freed by an
+      // MMA of this tile, which does not wait on this tile's scan (one more
+      // would wait on an MMA of the next tile, which waits on that scan).  An
+      // h slot depends on nothing but this loop: it is free once copied.
+      const int limit = min(min((i + 1) * p.kst + AS, (i + 2) * p.kst), total);
       for (; it_w < limit; ++it_w) {
-        const int a = it_w % AS, s = it_w % ST;
+        const int a = it_w % AS, j = it_w % HS;
         if (__any_sync(full_mask, *abort_flag != 0) ||
-            !__all_sync(full_mask, ptx::mbar_wait(bars.full(s), (it_w / ST) & 1)) ||
+            !__all_sync(full_mask, ptx::mbar_wait(bars.h_full(j), (it_w / HS) & 1)) ||
             !__all_sync(full_mask, ptx::mbar_wait(bars.a_empty(a), ((it_w / AS) & 1) ^ 1))) {
           ok = false;
           break;
@@ -269,7 +317,7 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
         ptx::tc_fence_after();
         for (int b = 0; b < KB; ++b) {
           // row r of box b: 128 bytes, 16-byte chunk j at (j ^ (r & 7)) (128-byte swizzle)
-          const uint8_t* hs = smem + s * SB + p.w_bytes + b * p.hb + r * 128;
+          const uint8_t* hs = smem + hbase + j * p.h_bytes + b * p.hb + r * 128;
           uint32_t x[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -283,7 +331,7 @@ lm_head_argmax_kernel(const __grid_constant__ LmParams p) {
         __syncwarp();
         if (lane == 0) {
           ptx::mbar_arrive(bars.a_full(a));
-          ptx::mbar_arrive(bars.empty(s));  // this warp is done with the stage's h rows
+          ptx::mbar_arrive(bars.h_empty(j));  // this warp is done with the slot's h rows
         }
       }
       if (!ok) break;
@@ -427,32 +475,48 @@ int choose_nv(int vocab, int sms, int max_nv) {
 }
 
 // The launch's shape for rows x d x vocab on `sms` SMs (host only): tile rows,
-// boxes per stage, the stage ring, the TMEM slice ring.
+// boxes per stage, the w ring, the h ring, the TMEM slice ring.  The h ring
+// holds at least kHBoxesAhead boxes in at least two slots (each slot's
+// refill is a round trip to L2, so fewer would pace the MMAs).  Boxes per
+// stage: the most w bytes in flight (stages x boxes) with at least two
+// stages beside the h ring, fewer boxes per stage only for more than 5% more
+// bytes in flight (a stage is one handshake); four boxes use tiles of at
+// most 176 rows so that two such stages fit.  One box per stage only where
+// the K steps leave no choice: measured at 128 rows, one box per stage with
+// 5 stages took 318 us against 234 us for two boxes with 2 stages.
 void plan(LmParams& p, int rows, int d, int vocab, int sms) {
   p.R = rows;
   p.V = vocab;
   p.ksteps = d / kStepK;
   p.writers = ceil_div(rows, 32);
   p.hb = p.writers * 32 * 128;
-  // boxes per stage: 4 if two such stages fit (tiles of at most 176 rows),
-  // else 2, else 1
   p.kb = 1;
   p.nv = choose_nv(vocab, sms, 256);
-  for (int cand = 4; cand >= 2; cand /= 2) {
-    if (p.ksteps % cand) continue;
+  p.stages = 0;
+  int64_t best = 0;
+  for (int cand = 4; cand >= 1; cand /= 2) {
+    if (p.ksteps % cand || (cand == 1 && p.ksteps % 2 == 0)) continue;
     const int nv = choose_nv(vocab, sms, cand == 4 ? 176 : 256);
-    if (kRingBudget / (cand * (nv * 128 + p.hb)) >= 2) {
+    const int hs = ceil_div(kHBoxesAhead, cand) > 2 ? ceil_div(kHBoxesAhead, cand) : 2;
+    const int ring = kRingBudget - hs * cand * p.hb;
+    int st = ring / (cand * nv * 128);
+    st = st < kMaxStages ? st : kMaxStages;
+    if (st < 2) continue;
+    const int64_t bytes = (int64_t)st * cand * nv * 128;
+    if (best == 0 || bytes * 20 > best * 21) {
+      best = bytes;
       p.kb = cand;
       p.nv = nv;
-      break;
+      p.stages = st;
+      p.hslots = hs;
     }
   }
   p.nvp = (p.nv + 31) / 32 * 32;
   p.tiles = ceil_div(vocab, p.nv);
   p.kst = p.ksteps / p.kb;
   p.w_bytes = p.kb * p.nv * 128;
-  p.stage_bytes = p.w_bytes + p.kb * p.hb;
-  p.stages = kRingBudget / p.stage_bytes < kMaxStages ? kRingBudget / p.stage_bytes : kMaxStages;
+  p.stage_bytes = p.w_bytes;
+  p.h_bytes = p.kb * p.hb;
   // TMEM: the accumulator (nv columns, 32-aligned), then the ring of h slices
   // (32 columns per box)
   p.a_col = p.nvp;
@@ -478,7 +542,7 @@ int orthrus_lm_head_argmax_plan(int32_t rows, int32_t d, int32_t vocab, int32_t 
   out[1] = p.kb;
   out[2] = p.stages;
   out[3] = p.aslots;
-  out[4] = layout(p.stages, p.stage_bytes).total + 1024;
+  out[4] = layout(p.stages, p.stage_bytes, p.h_bytes, p.hslots).total + 1024;
   out[5] = p.tiles < sms ? p.tiles : sms;
   out[6] = p.tiles;
   out[7] = kTmemCols;
@@ -520,11 +584,21 @@ int orthrus_lm_head_argmax(int32_t dtype, const void* h, int32_t rows, int32_t d
   if (!encode_2d(&p.tm_w, w, d, vocab, (int64_t)d * 2, p.nv) ||
       !encode_2d(&p.tm_h, h, d, rows, h_row_stride * 2, 32 * p.writers))
     return ORTHRUS_ECUDA;
-  const int smem = layout(p.stages, p.stage_bytes).total + 1024;
+  const int smem = layout(p.stages, p.stage_bytes, p.h_bytes, p.hslots).total + 1024;
   if (!prepare()) return ORTHRUS_ECUDA;
   const int grid = p.tiles < sms ? p.tiles : sms;
-  lm_head_argmax_kernel<<<grid, kThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, lm_head_argmax_kernel, p) == cudaSuccess ? ORTHRUS_OK
+                                                                           : ORTHRUS_ECUDA;
 }
 
 }  // extern "C"

@@ -355,7 +355,9 @@ int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stre
  * 8; vocab <= 2^30; h and w 16-byte aligned.  err (nullable) receives
  * ORTHRUS_ETIMEOUT if a bounded wait inside the kernel gave up.
  * workspace: orthrus_lm_head_argmax_workspace(rows) bytes, 16-byte aligned,
- * zeroed once; every call leaves it zero.  One launch, one CTA per SM.
+ * zeroed once; every call leaves it zero.  One launch, one CTA per SM.  w is
+ * read before the wait on the preceding kernel on the stream (it may not be
+ * written by the kernel right before this call); h only after it.
  * ---------------------------------------------------------------------- */
 size_t orthrus_lm_head_argmax_workspace(int32_t rows);
 /* The launch orthrus_lm_head_argmax would make for these sizes on a GPU with

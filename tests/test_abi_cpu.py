@@ -276,18 +276,20 @@ def test_lm_head_plan_respects_hardware_limits(L):
                     nv, kb, stages, aslots, smem, grid, tiles, tmem = list(out)
                     assert nv % 16 == 0 and 128 <= nv <= 256, (rows, d, V, nv)
                     assert kb in (1, 2, 4) and (d // 64) % kb == 0
+                    assert kb > 1 or (d // 64) % 2 == 1  # one box only for an odd K
                     assert stages >= 2 and aslots >= 1 and min(aslots, stages) >= 1
                     assert smem <= 227 * 1024, (rows, d, V, smem)
                     nvp = (nv + 31) // 32 * 32
                     assert nvp + aslots * 32 * kb <= tmem == 512
                     assert tiles * nv >= V > (tiles - 1) * nv
                     assert 1 <= grid <= min(sms, tiles)
-    # the Qwen3-8B LM head as measured: 176-row tiles, four boxes per stage for
-    # one block; 208-row tiles, two boxes for four blocks
+    # the Qwen3-8B LM head as measured: 176-row tiles, four boxes per stage and
+    # two stages for one block; 208-row tiles, two boxes per stage and three
+    # stages for four blocks (their h boxes, 16 KB each, in the separate h ring)
     assert L.orthrus_lm_head_argmax_plan(32, 4096, 151936, 148, out) == 0
     assert list(out)[:4] == [176, 4, 2, 2]
     assert L.orthrus_lm_head_argmax_plan(128, 4096, 151936, 148, out) == 0
-    assert list(out)[:4] == [208, 2, 2, 4]
+    assert list(out)[:4] == [208, 2, 3, 4]
     for bad in ((0, 4096, 100, 148), (129, 4096, 100, 148), (32, 100, 100, 148),
                 (32, 4096, 0, 148), (32, 4096, 100, 0)):
         assert L.orthrus_lm_head_argmax_plan(*bad, out) == -1

@@ -44,7 +44,9 @@ def _call_noalloc(fn, logits, idx, maxval):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_noalloc_argmax_matches_workspace_argmax_twice(dtype):
     fn = _noalloc()
-    for call, (rows, vocab) in enumerate([(32, 151936), (200, 8192)]):
+    # 151936 and 8192: one cluster per row; 300007 (19 chunks): the scratch's
+    # atomic slots and tickets
+    for call, (rows, vocab) in enumerate([(32, 151936), (200, 8192), (9, 300007)]):
         x = synth.logits(synth.rng(400 + call, len(dtype)), rows, vocab, dtype=dtype)
         if dtype == "bf16":
             t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
