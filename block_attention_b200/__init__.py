@@ -87,7 +87,7 @@ EXPORTS = ("orthrus_block_attn", "orthrus_block_attn_workspace",
            "orthrus_lm_head_argmax", "orthrus_lm_head_argmax_workspace",
            "orthrus_lm_head_argmax_plan",
            "orthrus_linear_tc", "orthrus_linear_tc_workspace", "orthrus_linear_tc_plan",
-           "orthrus_rope_table", "orthrus_linear_tc_qkv_rope",
+           "orthrus_rope_table", "orthrus_linear_tc_qkv_rope", "orthrus_selftest_bounded_wait",
            # decoder building blocks (include/orthrus_decoder.h)
            "orthrus_embed", "orthrus_rmsnorm", "orthrus_linear", "orthrus_qkv_rope",
            "orthrus_swiglu", "orthrus_block_tokens")
@@ -146,6 +146,7 @@ def lib() -> ctypes.CDLL:
         L.orthrus_linear_tc.argtypes = [i32, vp, i32, i32, i64, vp, i32, vp, vp, i64, vp, i64,
                                         vp, vp, sz, vp]
         L.orthrus_rope_table.argtypes = [vp, i32, i32, i32, c.c_double, vp, vp]
+        L.orthrus_selftest_bounded_wait.argtypes = [i32, c.c_uint32, vp, vp, vp]
         L.orthrus_linear_tc_qkv_rope.argtypes = [i32, vp, i32, i32, i64, vp, i32, i32, i32, vp,
                                                  vp, vp, vp, vp, i64, vp, vp, sz, vp]
         L.orthrus_lm_head_argmax_plan.argtypes = [i32, i32, i32, i32, vp]
@@ -536,6 +537,16 @@ def linear_tc_qkv_rope(x, w, Hq, Hkv, cos_sin, *, q, k, v, l2_next=None, err=Non
         _dtype(x), _ptr(x), rows, K, x.stride(0), _ptr(w), Hq, Hkv, hd, _ptr(cos_sin), _ptr(q),
         _ptr(k), _ptr(v), hp, hb, _ptr(err), _ptr(buf), buf.numel(), _stream(stream)))
     return q, k, v
+
+
+def selftest_bounded_wait(which, timeout_us, *, err, never=None, stream=None):
+    """Run one wait that never completes (0: an mbarrier phase, 1: the
+    generation word `never`) and let it give up after timeout_us: err (int32
+    CUDA tensor) receives ORTHRUS_ETIMEOUT (see orthrus.h)."""
+    _dev(err, never)
+    _check("orthrus_selftest_bounded_wait", lib().orthrus_selftest_bounded_wait(
+        which, timeout_us, _ptr(never), _ptr(err), _stream(stream)))
+    return err
 
 
 def linear_tc(x, w, *, residual=None, out=None, l2_next=None, err=None, workspace=None,

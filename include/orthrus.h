@@ -441,6 +441,20 @@ int orthrus_linear_tc_qkv_rope(int32_t dtype, const void* x, int32_t rows, int32
                                void* workspace, size_t workspace_bytes,
                                orthrus_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Self-test of the bounded waits (failure detection without a fault): one
+ * launch whose single wait never completes -- which = 0: an mbarrier phase
+ * nothing arrives on (the form of every TMA / MMA handshake in the kernels);
+ * which = 1: a generation word at `never` (device memory, 4-byte aligned,
+ * left unchanged by the caller meanwhile) that nothing advances (the form of
+ * the attention kernel's split-merge barrier).  After timeout_us
+ * microseconds (1 .. 10^7) the wait gives up, ORTHRUS_ETIMEOUT goes to *err
+ * (device memory) and the kernel returns; the context stays usable.  Returns
+ * ORTHRUS_EINVAL for other arguments.
+ * ---------------------------------------------------------------------- */
+int orthrus_selftest_bounded_wait(int32_t which, uint32_t timeout_us, const uint32_t* never,
+                                  int32_t* err, orthrus_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 const char* orthrus_status_str(int status);
 int orthrus_version(void);

@@ -414,3 +414,14 @@ def test_qkv_rope_projection_and_table_rejections(L):
     assert rt(B=0) == 0
     assert rt(lens=0) == -1 and rt(out=0) == -1 and rt(out=516) == -1
     assert rt(hd=127) == -1 and rt(blk=0) == -1 and rt(theta=0.0) == -1 and rt(B=-1) == -1
+
+
+def test_selftest_bounded_wait_rejections(L):
+    """Host-side checks of the bounded-wait self-test (no launch here)."""
+    vp = ctypes.c_void_p
+    st = lambda which=0, us=1000, never=256, err=512: L.orthrus_selftest_bounded_wait(
+        which, ctypes.c_uint32(us), vp(never) if never else None, vp(err) if err else None, None)
+    assert st(which=2) == -1 and st(which=-1) == -1
+    assert st(us=0) == -1 and st(us=10_000_001) == -1
+    assert st(err=0) == -1
+    assert st(which=1, never=0) == -1 and st(which=1, never=258) == -1
