@@ -684,8 +684,9 @@ def stochastic_round_leg(dev, hbm, iters=20):
     launches in one CUDA graph.  Algorithmic bytes: one read of each logit
     matrix plus the two rows of the correction.  Timed twice: 20 rounds back
     to back (the logits stay L2-resident, as right after the LM head writes
-    them), and single rounds after an L2 flush (HBM reads; the fraction of
-    peak refers to these)."""
+    them), and rounds that each follow an L2 flush (HBM reads; the fraction
+    of peak refers to these): a graph of `iters` x (flush, round) less a
+    graph of `iters` flushes, so no host launch gap enters the figure."""
     import torch
     import block_attention_b200 as ba
     w = WORKLOAD
@@ -708,34 +709,34 @@ def stochastic_round_leg(dev, hbm, iters=20):
     for k in range(3):
         step(k)
     torch.cuda.synchronize()
-    graph, one = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    graph, cold_g, flush_g = (torch.cuda.CUDAGraph() for _ in range(3))
     with torch.cuda.graph(graph):
         for k in range(iters):
             step(k)
-    with torch.cuda.graph(one):
-        step(0)
-    graph.replay()
-    one.replay()
+    with torch.cuda.graph(cold_g):
+        for k in range(iters):
+            flush.fill_(k & 0xFF)
+            step(k)
+    with torch.cuda.graph(flush_g):
+        for k in range(iters):
+            flush.fill_(k & 0xFF)
+    for g_ in (graph, cold_g, flush_g):
+        g_.replay()
     torch.cuda.synchronize()
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    e0, e1 = ev(), ev()
-    e0.record()
-    graph.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    hot = e0.elapsed_time(e1) * 1e3 / iters
-    cold = []
-    for k in range(10):
-        flush.fill_(k & 0xFF)
+
+    def timed(g_):
         e0, e1 = ev(), ev()
         e0.record()
-        one.replay()
+        g_.replay()
         e1.record()
         torch.cuda.synchronize()
-        cold.append(e0.elapsed_time(e1) * 1e3)
-    cold = sorted(cold)[len(cold) // 2]
+        return e0.elapsed_time(e1) * 1e3
+
+    hot = timed(graph) / iters
+    cold = sorted((timed(cold_g) - timed(flush_g)) / iters for _ in range(3))[1]
     nbytes = 2 * rows * V * 4 + 2 * V * 4
-    del graph, one
+    del graph, cold_g, flush_g
     return {"workload": f"stochastic consensus, B=1 block 32, vocab {V}, fp32 logits, T = 1",
             "kernels_per_round": 3, "bytes_per_round": nbytes,
             "us_per_round_l2_resident": hot, "us_per_round_cold": cold,
