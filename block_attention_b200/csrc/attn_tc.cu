@@ -452,13 +452,15 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       int nv = nv_tile;
       if (blk_tile && p.mask_mode == ORTHRUS_CAUSAL_VERIFY) nv = min(i_blk + 1, p.blk);
       const uint32_t s_addr = lane_addr + X * kTile;
-      // S(u) is read from TMEM twice, 64 columns at a time -- once for the row
-      // maximum, once for the exponentials -- so that no more than 64 of its
-      // values are live in registers; masked keys -> -inf (exactly 0 in P)
+      // S(u) is read from TMEM 64 columns at a time, so that no more than 64
+      // of its values are live in registers: both halves for the row
+      // maximum, then the exponentials of the second half, still in
+      // registers, and of the first half, read again (three loads, not
+      // four); masked keys -> -inf (exactly 0 in P)
       float mt[2] = {-INFINITY, -INFINITY};
+      uint32_t sv[2][32];  // after the maximum: the second half, masked
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t sv[2][32];
         ptx::tmem_ld32(s_addr + 64 * half, sv[0]);
         ptx::tmem_ld32(s_addr + 64 * half + 32, sv[1]);
         ptx::tmem_wait_ld();
@@ -492,16 +494,17 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       uint8_t* prow = smem + kPOff + X * kPBytes + r * 128;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sv[2][32];
-        ptx::tmem_ld32(s_addr + 64 * half, sv[0]);
-        ptx::tmem_ld32(s_addr + 64 * half + 32, sv[1]);
-        ptx::tmem_wait_ld();
-        if (half == 1) {  // S(u) is read: its TMEM buffer may take S(u + 2)
+      for (int hh = 0; hh < 2; ++hh) {
+        const int half = 1 - hh;
+        if (hh == 1) {
+          ptx::tmem_ld32(s_addr, sv[0]);
+          ptx::tmem_ld32(s_addr + 32, sv[1]);
+          ptx::tmem_wait_ld();
+          // S(u) is read: its TMEM buffer may take S(u + 2)
           ptx::tc_fence_before();
           ptx::mbar_arrive(bars.s_free(X));
+          if (nv < kTile) mask_keys(sv, 0, nv);
         }
-        if (nv < kTile) mask_keys(sv, 64 * half, nv);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {  // 8 keys: 64 half + 8 ch .. + 7
           uint32_t w4[4];
