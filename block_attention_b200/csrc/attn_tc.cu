@@ -12,43 +12,45 @@
 // (128 FLOP per KV byte at the Qwen3-8B shape -- beyond CUDA cores, so the
 // QK^T and PV products run on the tensor pipe).
 //
-// attn_tc_kernel, grid (S splits, Hkv, B), one CTA per SM.  The keys
+// attn_tc_kernel, grid (Hkv, B, S splits), one CTA per SM.  The keys
 // cache[0, n) of a (sequence, kv-head) are cut into 128-key tiles, followed by
-// one tile holding the blk block rows; the tiles are dealt out contiguously
-// over the S splits.  Per CTA (10 warps):
+// one tile holding the blk block rows; the T tiles are dealt out contiguously
+// over the S splits, the first T mod S splits taking one tile more.  The
+// splits vary slowest in the grid, so the CTAs launched last -- on the SMs the
+// preceding kernel frees last -- are the high splits, the ones with fewer
+// tiles.  Per CTA (10 warps):
 //   warp 0      TMA producers: lane 0 streams K tiles, lane 1 V tiles, through
-//               a 3-stage ring (32 KB of K + 32 KB of V per stage); a K slot
+//               a 2-stage ring (32 KB of K + 32 KB of V per stage); a K slot
 //               is refilled as soon as its S = Q K^T product has read it, a V
 //               slot once its P V product has
 //   warp 1      MMA issuer (one thread): S(u) = Q K(u)^T (M=128, N=128 per
 //               instruction, Q and K from shared memory) into TMEM buffer
-//               u & 1, and O_(u & 1) += P(u) V(u) with P(u) read from TMEM;
-//               once P(u) is ready the 8 instructions of P(u) V(u) go out,
-//               then the 8 of S(u + 2), into the buffer P(u) occupied (one
-//               thread's MMAs run in order, so P(u) has been read by then)
+//               u & 1; S(u + 2) goes out as soon as softmax(u) has read S(u),
+//               ahead of O_(u & 1) += P(u) V(u) (P(u) from shared memory)
 //   warps 2..9  softmax, two warpgroups taking turns: warps 2-5 the even
-//               tiles, warps 6-9 the odd ones, one query row per thread.  A
-//               softmax warp per SM sub-partition is latency-bound (its
-//               exponentials and bf16 conversions wait on each other); two
-//               overlap.  Each warpgroup keeps its own running max and sum
-//               and its own O accumulator with lazy rescaling (O is rescaled
-//               only when a row's running maximum grows by more than 2^8) and
-//               writes P over the S buffer it has just read, as bf16 pairs.
-//               At the end they swap (max, sum) and each writes half of the
-//               combined unnormalised O, with the row max and sum, to the
-//               workspace.
+//               tiles, warps 6-9 the odd ones, one query row per thread, so
+//               that one warpgroup's exponentials overlap the other's.  Each
+//               keeps its own running max and sum and its own O accumulator
+//               with lazy rescaling (O is rescaled only when a row's running
+//               maximum grows by more than 2^8).  S is read from TMEM 64
+//               columns at a time (three loads per tile: both halves for the
+//               maximum, the second kept into the exponentials); P goes to the
+//               warpgroup's shared-memory buffer as bf16, in the MMA's K-major
+//               128-byte-swizzled layout.  At the end the two swap (max, sum)
+//               and each writes half of the combined unnormalised O, with the
+//               row max and sum, to the workspace.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O_0 [256,256+D) O_1 [256+D,
-// 256+2D); P(u) over the first 64 columns of S(u)'s buffer.
+// 256+2D).
 // 128-key S tiles: a tcgen05.mma with N = 64 costs the issuing thread as much
 // as one with N = 128, so the wider tile halves the MMA issue time per key.
 //
-// Split merge.  Each split writes its unnormalised O (fp32), row max and row
-// sum to an L2-resident workspace, grouped by the query rows one merging CTA
-// owns, so that the owner fetches a split's share with one bulk copy.  When
-// the grid fits one wave (every CTA resident at once, the batch-1 decoding
-// case) the merge runs inside the same launch: a sense-reversing barrier per
-// (sequence, kv-head) -- count in, the last CTA resets the count and
-// advances the generation the others wait on (bounded) -- then every CTA
+// Split merge.  Each split writes its unnormalised O (bf16), row max and row
+// sum (fp32) to an L2-resident workspace, grouped by the query rows one
+// merging CTA owns, so that the owner fetches a split's share with one bulk
+// copy.  When the grid fits one wave (every CTA resident at once, the batch-1
+// decoding case) the merge runs inside the same launch: a sense-reversing
+// barrier per (sequence, kv-head) -- count in, the last CTA resets the count
+// and advances the generation the others wait on (bounded) -- then every CTA
 // stages its row group of all S partials by bulk copies and merges them in
 // split order (the result does not depend on timing) into bf16 output.
 // Larger grids, whose CTAs cannot all be resident, end instead and a second
@@ -184,7 +186,7 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int g = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
   const int S = p.S;
   const unsigned full_mask = 0xffffffffu;
 
@@ -246,8 +248,9 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
     const bool bad = n < 0 || n > p.max_ctx;
     Tc = bad ? 0 : ceil_div(n, kTile);
     const int T = bad ? 0 : Tc + 1;
-    t0 = (int)(((int64_t)split * T) / S);
-    U = (int)(((int64_t)(split + 1) * T) / S) - t0;
+    const int base = T / S, extra = T % S;  // the first `extra` splits take base + 1
+    t0 = split * base + min(split, extra);
+    U = base + (split < extra ? 1 : 0);
   };
   // K (is_v false) or V half of tile t into ring slot u % kStages
   auto issue = [&](bool is_v, int u, int t, int Tc) {
@@ -895,7 +898,7 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl.val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, a.Hkv, a.B);
+  cfg.gridDim = dim3(a.Hkv, a.B, S);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;

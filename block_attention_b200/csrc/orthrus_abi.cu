@@ -106,9 +106,9 @@ int orthrus_block_attn_plan(const orthrus_attn_args* a, int32_t sms, int32_t* ou
   const int S = tc_plan_splits(*a, sms);
   const int tiles = (a->max_ctx + 127) / 128 + 1;  // 128-key cache tiles + the block tile
   out[0] = S;
-  out[1] = S;
-  out[2] = a->Hkv;
-  out[3] = a->B;
+  out[1] = a->Hkv;
+  out[2] = a->B;
+  out[3] = S;
   out[4] = tc_threads();
   out[5] = tc_smem_bytes();
   out[6] = (tiles + S - 1) / S;

@@ -157,7 +157,7 @@ int orthrus_block_attn_launches(const orthrus_attn_args* a);
  * only; pointers in `a` are not read).  The keys of each (sequence, kv-head)
  * -- cache[0, max_ctx) in 128-key tiles, then one tile of block rows -- are
  * dealt over S splits, one CTA each; the splits' partial results are merged
- * in split order.  out[0..8) = S, grid x, y, z (S, Hkv, B), threads per CTA,
+ * in split order.  out[0..8) = S, grid x, y, z (Hkv, B, S), threads per CTA,
  * dynamic shared memory bytes, most tiles one split streams, and 1 if the
  * merge runs inside the one launch (the grid fits one wave of one CTA per SM:
  * B * Hkv * S <= sms and B * Hkv <= 256) or 0 if a second, PDL-chained

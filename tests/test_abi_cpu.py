@@ -324,7 +324,7 @@ def test_tensor_core_attention_plan(L):
                         heads = B * Hkv
                         assert 1 <= S <= min(24, tiles), key
                         assert 2048 + heads * S * part <= ws, key  # fits the sized buffer
-                        assert (gx, gy, gz) == (S, Hkv, B), key
+                        assert (gx, gy, gz) == (Hkv, B, S), key
                         assert most == -(-tiles // S), key
                         assert most <= 64 or S == 24, key
                         if heads < sms:  # a small batch fills the SMs as far as it can
@@ -341,7 +341,7 @@ def test_tensor_core_attention_plan(L):
     # the Qwen3-8B round shape on 148 SMs: 18 splits per kv-head, 144 CTAs,
     # at most 4 of the 65 tiles each, merged inside the launch
     assert L.orthrus_block_attn_plan(ctypes.byref(a), 148, out) == 0
-    assert list(out)[:4] == [18, 18, 8, 1] and out[6] == 4 and out[7] == 1
+    assert list(out)[:4] == [18, 8, 1, 18] and out[6] == 4 and out[7] == 1
 
 
 def test_linear_tc_plan_and_rejections(L):
