@@ -54,7 +54,12 @@
 // stages its row group of all S partials by bulk copies and merges them in
 // split order (the result does not depend on timing) into bf16 output.
 // Larger grids, whose CTAs cannot all be resident, end instead and a second
-// kernel (attn_tc_combine, PDL-chained) merges the same way.
+// kernel (attn_tc_combine, PDL-chained) merges the same way.  In such a grid
+// over 2..32 sequences the CTAs take their (sequence, split, kv-head) in
+// order of decreasing context length rather than by grid position: the
+// hardware starts CTAs in launch order as SMs come free, so the longest
+// splits start first and the short ones fill the tail (longest processing
+// time first list scheduling).
 //
 // With ORTHRUS_ATTN_EARLY_KV the kernel reads ctx_lens and starts
 // streaming its first K/V tiles before waiting on the preceding kernel; Q and
@@ -137,6 +142,7 @@ struct __align__(64) TcParams {
   const __nv_bfloat16* next_v;
   float* part;         // [B][Hkv] x S split partials (workspace after the counters)
   int R;               // query rows per partial group = rows one merging CTA owns
+  int order;           // launch order sorted by context length (B in [2, 32], unfused)
   unsigned* counters;  // [B * Hkv] arrival counters of the in-kernel merge (kept at zero)
   int B, Hq, Hkv, blk, cap, max_ctx, mask_mode, G, S, early;
   float scale_log2;
@@ -186,7 +192,7 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
+  int g = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
   const int S = p.S;
   const unsigned full_mask = 0xffffffffu;
 
@@ -237,6 +243,40 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   ptx::griddep_launch_dependents();
+
+  // Longest sequences first, for grids of more than one wave: CTAs start in
+  // launch order, so launch position `lin` takes entry `lin` of the list of
+  // (sequence, split, kv-head) sorted by decreasing context length (kv-head
+  // fastest, ties by sequence index).  The long splits start first and the
+  // short ones fill the tail.  Warp 0 keeps the lengths it ranked (`seen`):
+  // under ORTHRUS_ATTN_EARLY_KV they were read before the dependency wait,
+  // and a change under the kernel is caught after it.
+  int seen = 0;
+  if (!kFused && p.order) {
+    if (!p.early) ptx::griddep_wait();  // the lengths may come from the preceding kernel
+    int* map = reinterpret_cast<int*>(smem + kPOff);  // P is written only after the MMAs
+    if (warp == 0) {
+      seen = lane < p.B ? p.ctx_lens[lane] : 0;
+      const int key = lane >= p.B ? -2 : (seen < 0 || seen > p.max_ctx ? -1 : seen);
+      int rank = 0;
+      for (int i = 0; i < p.B; ++i) {
+        const int ki = __shfl_sync(full_mask, key, i);
+        rank += (ki > key || (ki == key && i < lane)) ? 1 : 0;
+      }
+      const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+      const unsigned hit = __ballot_sync(full_mask, lane < p.B && rank == lin / (p.Hkv * S));
+      if (lane == 0) {
+        map[0] = __ffs(hit) - 1;
+        map[1] = (lin / p.Hkv) % S;
+        map[2] = lin % p.Hkv;
+      }
+    }
+    __syncthreads();
+    b = map[0];
+    split = map[1];
+    g = map[2];
+    __syncthreads();
+  }
 
   const uint32_t q_s = sbase;
   auto k_s = [&](int stage) { return sbase + kRingOff + stage * kStageBytes; };
@@ -310,7 +350,10 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   if (bad && split == 0 && g == 0 && threadIdx.x == 0) set_err(p.err, ORTHRUS_ECAPACITY);
   int Tc, t0, U;
   geometry(n, Tc, t0, U);
-  if (warp == 0 && lane == 0 && early_issued > 0 && early_n != n) {
+  // with the sorted launch order, any length read early must hold
+  const bool moved = !kFused && p.order && p.early && warp == 0 &&
+                     __any_sync(full_mask, lane < p.B && p.ctx_lens[lane] != seen);
+  if (warp == 0 && lane == 0 && ((early_issued > 0 && early_n != n) || moved)) {
     // the EARLY_KV contract was broken (the length changed under us): drain
     // the early loads and produce nothing for this split
     for (int u = 0; u < early_issued; ++u)
@@ -892,6 +935,7 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   p.max_ctx = a.max_ctx; p.mask_mode = a.mask_mode; p.G = G; p.S = S;
   p.R = fused ? ceil_div(G * a.blk, S) : kGroupRows;
   p.early = (a.flags & ORTHRUS_ATTN_EARLY_KV) ? 1 : 0;
+  p.order = !fused && a.B >= 2 && a.B <= 32;
   p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
 
   cudaLaunchAttribute pdl;

@@ -78,6 +78,30 @@ def test_qwen3_8b_layer_full(oracle_mod, mode):
     check(inp, mode, "bf16", oracle_mod=oracle_mod)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_multi_wave_grid_sorted_by_length(oracle_mod, mode):
+    """A bf16 grid of more than one wave (here 20 sequences x 8 kv-heads x 2
+    splits = 320 CTAs, merged by the second kernel) starts its CTAs
+    longest-sequence first.  Every (sequence, kv-head, split) is still
+    computed exactly once: the output matches the oracle, and the
+    ORTHRUS_ATTN_EARLY_KV launch (lengths read before the dependency wait)
+    gives the same bits."""
+    lens = [5, 900, 0, 3000, 129, 2500, 77, 1800, 640, 1, 3333, 256, 1500, 12, 2048, 700,
+            999, 9000, 31, 1024]
+    inp = synth.attn_inputs(len(lens), 16, 8, 128, 16, lens, max(lens) + 20, "bf16", seed=120)
+    ref = oracle_mod.block_attn(inp["q"], inp["k_blk"], inp["v_blk"], inp["k_cache"],
+                                inp["v_cache"], inp["ctx_lens"], mode)
+    t = {k: to_dev(v) for k, v in inp.items()}
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = [ba.block_attn(t["q"], t["k_blk"], t["v_blk"], t["k_cache"], t["v_cache"],
+                          t["ctx_lens"], mode, err=err, flags=f) for f in (0, ba.ATTN_EARLY_KV)]
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(outs[0], outs[1])
+    e = rel_err_rows(to_host(outs[0]), ref)
+    assert e.max() <= TOL["bf16"], (e.max(), np.unravel_index(e.argmax(), e.shape))
+
+
 def test_ragged_batch_sampled_sequences(oracle_mod):
     """16 sequences, contexts ~ U{1024..32768}; the GPU runs the whole batch,
     the oracle checks three of them (first, longest, shortest)."""
