@@ -301,20 +301,49 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
 // Grid (chunks, rows); element e of thread t is c * kChunk + e * kThreads + t
 // (coalesced).  The row's last CTA merges the chunk pairs.  Workspace:
 // tickets [rows] then the pairs [rows][chunks].
-template <typename T>
+template <typename T, bool kVec>
 __device__ __forceinline__ float load_chunk(const T* row, int c, int vocab, float inv_t,
                                             float (&x)[kPer]) {
   float m = -INFINITY;
+  if constexpr (kVec) {
+    // groups of four consecutive logits, one 16-byte (f32) or 8-byte (bf16)
+    // load each, as the sampler reads them; every load in flight first
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    const int k = c * kChunk + e * kThreads + threadIdx.x;
-    x[e] = k < vocab ? to_f32(row[k]) * inv_t : -INFINITY;
-    m = fmaxf(m, x[e]);
+    for (int e4 = 0; e4 < kPer / 4; ++e4) {
+      const int k = c * kChunk + (e4 * kThreads + threadIdx.x) * 4;
+      if (k + 3 < vocab) {
+        if constexpr (sizeof(T) == 4) {
+          const float4 f = __ldcs(reinterpret_cast<const float4*>(row + k));
+          x[4 * e4] = f.x; x[4 * e4 + 1] = f.y; x[4 * e4 + 2] = f.z; x[4 * e4 + 3] = f.w;
+        } else {
+          const uint2 u = __ldcs(reinterpret_cast<const uint2*>(row + k));
+          x[4 * e4] = __uint_as_float(u.x << 16);
+          x[4 * e4 + 1] = __uint_as_float(u.x & 0xffff0000u);
+          x[4 * e4 + 2] = __uint_as_float(u.y << 16);
+          x[4 * e4 + 3] = __uint_as_float(u.y & 0xffff0000u);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[4 * e4 + e] = k + e < vocab ? to_f32(row[k + e]) : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      x[e] *= inv_t;
+      m = fmaxf(m, x[e]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int k = c * kChunk + e * kThreads + threadIdx.x;
+      x[e] = k < vocab ? to_f32(row[k]) * inv_t : -INFINITY;
+      m = fmaxf(m, x[e]);
+    }
   }
   return m;
 }
 
-template <typename T>
+template <typename T, bool kVec>
 __global__ void __launch_bounds__(kThreads)
 token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
                      const int32_t* __restrict__ idx, float inv_t, int nchunks,
@@ -326,7 +355,7 @@ token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x;
   const T* row = logits + (int64_t)r * stride;
   float x[kPer];
-  const float2 pr = chunk_pair(x, load_chunk(row, c, vocab, inv_t, x), red);
+  const float2 pr = chunk_pair(x, load_chunk<T, kVec>(row, c, vocab, inv_t, x), red);
   if (t == 0) {
     pairs[(int64_t)r * nchunks + c] = pr;
     __threadfence();
@@ -363,7 +392,7 @@ struct SeqSlot {
   unsigned long long key_res, key_max;
 };
 
-template <typename T>
+template <typename T, bool kVec>
 __global__ void __launch_bounds__(kThreads, 6)
 consensus_verify_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, float inv_t,
                         int nchunks, SeqSlot* seq, unsigned* row_tickets, float2* pairs) {
@@ -373,7 +402,7 @@ consensus_verify_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, f
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, blk = p.blk, b = r / blk;
   const T* row = static_cast<const T*>(p.logits_ar) + (int64_t)r * p.row_stride;
   float x[kPer];
-  const float2 pr = chunk_pair(x, load_chunk(row, c, p.vocab, inv_t, x), red);
+  const float2 pr = chunk_pair(x, load_chunk<T, kVec>(row, c, p.vocab, inv_t, x), red);
   if (t == 0) {
     pairs[(int64_t)r * nchunks + c] = pr;
     __threadfence();
@@ -467,6 +496,13 @@ consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1,
 }
 
 size_t round256(int64_t n) { return (size_t)((n + 255) / 256 * 256); }
+
+// One 16-byte (f32) or 8-byte (bf16) load per group of four logits: the
+// base aligned to a group and every row starting on a group boundary.
+bool vec_rows(const void* logits, int64_t row_stride, int32_t dtype) {
+  const size_t gbytes = dtype == ORTHRUS_F32 ? 16 : 8;
+  return reinterpret_cast<uintptr_t>(logits) % gbytes == 0 && row_stride % 4 == 0;
+}
 constexpr int32_t kMaxVocab = 1 << 30;
 
 }  // namespace
@@ -563,13 +599,17 @@ int orthrus_token_logprob(int32_t dtype, const void* logits, int32_t rows, int32
   const float inv_t = 1.f / temperature;
   auto st = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid(nchunks, rows);
-  if (dtype == ORTHRUS_F32)
-    return status(launch_pdl(token_logprob_kernel<float>, grid, st,
-                             static_cast<const float*>(logits), vocab, row_stride, idx, inv_t,
-                             nchunks, tickets, pairs, logprob, lse));
-  return status(launch_pdl(token_logprob_kernel<__nv_bfloat16>, grid, st,
-                           static_cast<const __nv_bfloat16*>(logits), vocab, row_stride, idx,
-                           inv_t, nchunks, tickets, pairs, logprob, lse));
+  const bool vec = vec_rows(logits, row_stride, dtype);
+#define ORTHRUS_LOGPROB(T, V)                                                                  \
+  return status(launch_pdl(token_logprob_kernel<T, V>, grid, st, static_cast<const T*>(logits), \
+                           vocab, row_stride, idx, inv_t, nchunks, tickets, pairs, logprob, lse))
+  if (dtype == ORTHRUS_F32) {
+    if (vec) ORTHRUS_LOGPROB(float, true);
+    ORTHRUS_LOGPROB(float, false);
+  }
+  if (vec) ORTHRUS_LOGPROB(__nv_bfloat16, true);
+  ORTHRUS_LOGPROB(__nv_bfloat16, false);
+#undef ORTHRUS_LOGPROB
 }
 
 size_t orthrus_consensus_sample_workspace(int32_t B, int32_t blk, int32_t vocab) {
@@ -606,15 +646,20 @@ int orthrus_consensus_sample(const orthrus_sample_args* a, orthrus_stream_t stre
   const int nres = ceil_div(a->vocab, kResChunk);
   const dim3 g1(nchunks, (unsigned)rows), g2(nres, a->B);
   const orthrus_sample_args args = *a;
+  const bool vec = vec_rows(a->logits_ar, a->row_stride, a->dtype);
   cudaError_t e;
   if (a->dtype == ORTHRUS_F32) {
-    e = launch_pdl(consensus_verify_kernel<float>, g1, st, args, k0, k1, inv_t, nchunks, seq,
-                   row_tickets, pairs);
+    e = vec ? launch_pdl(consensus_verify_kernel<float, true>, g1, st, args, k0, k1, inv_t,
+                         nchunks, seq, row_tickets, pairs)
+            : launch_pdl(consensus_verify_kernel<float, false>, g1, st, args, k0, k1, inv_t,
+                         nchunks, seq, row_tickets, pairs);
     if (e == cudaSuccess)
       e = launch_pdl(consensus_residual_kernel<float>, g2, st, args, k0, k1, inv_t, nres, seq);
   } else {
-    e = launch_pdl(consensus_verify_kernel<__nv_bfloat16>, g1, st, args, k0, k1, inv_t,
-                   nchunks, seq, row_tickets, pairs);
+    e = vec ? launch_pdl(consensus_verify_kernel<__nv_bfloat16, true>, g1, st, args, k0, k1,
+                         inv_t, nchunks, seq, row_tickets, pairs)
+            : launch_pdl(consensus_verify_kernel<__nv_bfloat16, false>, g1, st, args, k0, k1,
+                         inv_t, nchunks, seq, row_tickets, pairs);
     if (e == cudaSuccess)
       e = launch_pdl(consensus_residual_kernel<__nv_bfloat16>, g2, st, args, k0, k1, inv_t,
                      nres, seq);
