@@ -679,9 +679,12 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
     __threadfence();  // this CTA's partial is visible before it is counted
     int ok = 1;
     if (atomicAdd(cnt, 1u) == (unsigned)S - 1u) {
-      atomicExch(cnt, 0u);  // every split has arrived: ready for the next call
+      // every split has arrived: release the others first (the fence orders
+      // the partials acquired through the count before the generation), then
+      // ready the count for the next call, which starts after this one ends
       __threadfence();
       atomicAdd(gen, 1u);
+      atomicExch(cnt, 0u);
     } else {
       const uint64_t t0 = ptx::globaltimer();
       while (ptx::ld_acquire_gpu(gen) == gen0) {
@@ -732,7 +735,15 @@ __device__ __forceinline__ void merge_rows(const TcParams& p, int b, int g, int 
     set_err(p.err, ORTHRUS_ETIMEOUT);
     return;
   }
-  for (int it = tid; it < nr * kChunks; it += nthreads) {
+  // One item per (row, 16-byte chunk).  With threads to spare and enough
+  // splits to share, two threads take an item, one the even splits and one
+  // the odd (lanes 2k and 2k + 1: nthreads is even), and the even one adds
+  // the odd one's sums to its own.
+  const int items = nr * kChunks;
+  const bool pair = 2 * items <= nthreads && S >= 8;
+  const int per = pair ? 2 : 1;
+  for (int it2 = tid; it2 < items * per; it2 += nthreads) {
+    const int it = it2 / per, half = it2 % per;
     const int c8 = it / nr, rl = it % nr, r = r0 + rl;
     float M = -INFINITY;
     for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, st4[s2 * gf4 + kChunks * R + rl].x);
@@ -740,7 +751,7 @@ __device__ __forceinline__ void merge_rows(const TcParams& p, int b, int g, int 
     float L = 0.f, acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    for (int s2 = 0; s2 < S; ++s2) {
+    for (int s2 = half; s2 < S; s2 += per) {
       const float4 ml = st4[s2 * gf4 + kChunks * R + rl];
       const uint4 o = reinterpret_cast<const uint4*>(st4)[s2 * gf4 + c8 * R + rl];
       const float w = ptx::ex2(ml.x - M);  // 0 for an empty split
@@ -751,6 +762,14 @@ __device__ __forceinline__ void merge_rows(const TcParams& p, int b, int g, int 
         acc[2 * e] = fmaf(w, __uint_as_float(ow[e] << 16), acc[2 * e]);
         acc[2 * e + 1] = fmaf(w, __uint_as_float(ow[e] & 0xffff0000u), acc[2 * e + 1]);
       }
+    }
+    if (pair) {
+      // both lanes of the pair are here: same item, same M
+      const unsigned pm = 3u << ((threadIdx.x & 31) & ~1);
+      L += __shfl_xor_sync(pm, L, 1);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(pm, acc[e], 1);
+      if (half) continue;
     }
     const float inv = 1.f / L;
     const int i = r / p.G, h = g * p.G + r % p.G;
