@@ -205,16 +205,28 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
   __shared__ float red[kWarps + 1];
   __shared__ unsigned long long wbest[kWarps];
   __shared__ bool last;
-  pdl_enter();
   const int c = blockIdx.x, r = blockIdx.y, t = threadIdx.x, lane = t & 31;
+  // two batches of three groups: a batch's loads first, then its arithmetic
+  constexpr int kB = kPer / 8;
+  // the first batch's noise depends only on (row, index, step): drawn before
+  // the wait, while the preceding kernel (the one writing the logits) ends
+  ptx::griddep_launch_dependents();
+  float gn0[4 * kB];
+#pragma unroll
+  for (int ii = 0; ii < kB; ++ii) {
+    const int g = c * (kChunk / 4) + ii * kThreads + t;
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step),
+                                  k0, k1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) gn0[4 * ii + e] = gumbel2(word(w, e));
+  }
+  ptx::griddep_wait();
   const T* row = logits + (int64_t)r * stride;
   // keys in base 2 (x log2(e) / T + gumbel2); the running (max, sum of
   // exp(x / T - max)) in natural units, each difference taken before the
   // base change (see chunk_pair)
   float bv = -INFINITY, m = -INFINITY, sum = 0.f;
   int bi = -1;
-  // two batches of three groups: a batch's loads first, then its arithmetic
-  constexpr int kB = kPer / 8;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     float xs[4 * kB];  // past the row: -inf (never wins, adds exp(-inf) = 0)
@@ -241,8 +253,9 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
 #pragma unroll
     for (int ii = 0; ii < kB; ++ii) {
       const int g = c * (kChunk / 4) + (half * kB + ii) * kThreads + t;
-      const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step),
-                                    k0, k1);
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (half == 1)
+        w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)r, kPurposeDraft, step), k0, k1);
       float x[4];
       float gm = -INFINITY;
 #pragma unroll
@@ -250,7 +263,7 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
         x[e] = xs[4 * ii + e] * inv_t;
         gm = fmaxf(gm, x[e]);
         // strictly larger: equal keys keep the lower index, NaN never wins
-        const float key = fmaf(x[e], kLog2e, gumbel2(word(w, e)));
+        const float key = fmaf(x[e], kLog2e, half == 0 ? gn0[4 * ii + e] : gumbel2(word(w, e)));
         if (key > bv) { bv = key; bi = 4 * g + e; }
       }
       if constexpr (kLse) {
@@ -450,8 +463,17 @@ __global__ void __launch_bounds__(kThreads)
 consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, float inv_t,
                           int nchunks, SeqSlot* seq) {
   __shared__ unsigned long long wres[kWarps], wmax[kWarps];
-  pdl_enter();
   const int c = blockIdx.x, b = blockIdx.y, t = threadIdx.x, blk = p.blk;
+  // the noise depends on the vocabulary index, not on which row is
+  // corrected: drawn while the log p pass finishes, before the wait
+  ptx::griddep_launch_dependents();
+  const int g = c * (kResChunk / 4) + t;
+  const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)b, kPurposeResidual, p.step),
+                                k0, k1);
+  float gn[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) gn[e] = gumbel2(word(w, e));
+  ptx::griddep_wait();
   const int L = p.accept_len[b];
   if (L >= blk) return;  // every draft accepted: no correction
   const int r = b * blk + L;
@@ -459,16 +481,13 @@ consensus_residual_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1,
   const T* zd = static_cast<const T*>(p.logits_diff) + (int64_t)r * p.row_stride;
   const float la = p.lse_ar[r], ld = p.lse_diff[r];
   unsigned long long best = 0ull, bmax = 0ull;
-  const int g = c * (kResChunk / 4) + t;
-  const uint4 w = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)b, kPurposeResidual, p.step),
-                                k0, k1);
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int k = 4 * g + e;
     if (k < p.vocab) {
       const float xa = to_f32(za[k]);
       const float d = expf(xa * inv_t - la) - expf(to_f32(zd[k]) * inv_t - ld);
-      if (d > 0.f) best = umax64(best, order_key(log2f(d) + gumbel2(word(w, e)), k));
+      if (d > 0.f) best = umax64(best, order_key(log2f(d) + gn[e], k));
       bmax = umax64(bmax, order_key(xa, k));
     }
   }
