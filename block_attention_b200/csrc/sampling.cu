@@ -388,10 +388,10 @@ token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
 
 // ------------------------------------------------------ stochastic consensus
 // Launch 1, grid (chunks, B*blk) over the AR logits: log p_j(d_j) and the
-// row's log-sum-exp as in token_logprob_kernel; the CTA that merges a
-// sequence's last row (per-sequence ticket) then tests the acceptances of
-// the sequence in one warp: log u_j < log p_j(d_j) - log q_j(d_j), left to
-// right, and writes every output except the correction.
+// row's log-sum-exp as in token_logprob_kernel, and the row's acceptance
+// test log u_j < log p_j(d_j) - log q_j(d_j); the CTA that merges a
+// sequence's last row (per-sequence count) takes the first rejection, left
+// to right, and writes every output except the correction.
 // Launch 2, grid (kResChunk-element chunks, B): one group of four per thread,
 // so the two rows' work spreads over about one wave; Gumbel-max over the
 // rejected row's residual max(0, p - q) (the AR row's argmax as the
@@ -401,8 +401,11 @@ token_logprob_kernel(const T* __restrict__ logits, int vocab, int64_t stride,
 constexpr int kResChunk = kThreads * 4;
 
 struct SeqSlot {
-  uint32_t rows_done, ticket;
+  // rows verified (high word) and the rejected positions (low word, bit j
+  // for row j: rows are distinct, so adding a row's bit is or-ing it)
+  unsigned long long verified;
   unsigned long long key_res, key_max;
+  uint32_t ticket, pad;
 };
 
 template <typename T, bool kVec>
@@ -426,25 +429,25 @@ consensus_verify_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, f
   __threadfence();
   const int lane = t;
   const float l = merge_pairs(pairs + (int64_t)r * nchunks, nchunks, lane);
-  int seq_last = 0;
+  // the row's own acceptance test, folded with the row count into one
+  // atomic: the warp whose row completes the sequence reads the first
+  // rejection from the folded bits (no other row's values are read back)
+  unsigned long long st = 0ull;
   if (lane == 0) {
     row_tickets[r] = 0u;
-    const int d = p.draft[r];
+    const int d = p.draft[r], j = r - b * blk;
+    const float lp = (d >= 0 && d < p.vocab) ? to_f32(row[d]) * inv_t - l : qnan();
     p.lse_ar[r] = l;
-    p.logp[r] = (d >= 0 && d < p.vocab) ? to_f32(row[d]) * inv_t - l : qnan();
-    __threadfence();
-    seq_last = atomicAdd(&seq[b].rows_done, 1u) == (unsigned)blk - 1u;
-  }
-  if (!__shfl_sync(0xffffffffu, seq_last, 0)) return;
-  __threadfence();
-  bool acc = true;
-  if (lane < blk) {
-    const int rj = b * blk + lane;
-    const uint4 w = philox4x32_10(make_uint4((uint32_t)lane, (uint32_t)b, kPurposeAccept, p.step),
+    p.logp[r] = lp;
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)j, (uint32_t)b, kPurposeAccept, p.step),
                                   k0, k1);
-    acc = logf(philox_uniform(w.x)) < __ldcg(&p.logp[rj]) - p.logq[rj];  // NaN: reject
+    const bool acc = logf(philox_uniform(w.x)) < lp - p.logq[r];  // NaN: reject
+    const unsigned long long add = (1ull << 32) | (acc ? 0ull : 1ull << j);
+    st = atomicAdd(&seq[b].verified, add) + add;
   }
-  const unsigned miss = __ballot_sync(0xffffffffu, !acc);
+  st = __shfl_sync(0xffffffffu, st, 0);
+  if ((unsigned)(st >> 32) != (unsigned)blk) return;
+  const unsigned miss = (unsigned)st;
   const int L = miss ? __ffs(miss) - 1 : blk;
   if (lane < blk) {
     const int d = p.draft[(int64_t)b * blk + lane];
@@ -452,7 +455,7 @@ consensus_verify_kernel(const orthrus_sample_args p, uint32_t k0, uint32_t k1, f
     if (L == blk && lane == blk - 1 && p.next_anchor) p.next_anchor[b] = d;
   }
   if (lane == 0) {
-    seq[b].rows_done = 0u;
+    seq[b].verified = 0ull;
     p.accept_len[b] = L;
     p.n_emit[b] = min(L + 1, blk);
   }
