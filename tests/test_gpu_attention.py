@@ -164,6 +164,31 @@ def test_device_length_over_bound_sets_error_word(oracle_mod, dtype):
     assert np.all(got[1] == 7.0)  # skipped sequence left untouched
 
 
+def test_multi_wave_grid_with_lengths_over_bound(oracle_mod):
+    """The length-sorted launch order of a multi-wave grid ranks sequences
+    whose length is out of bounds last; they report ORTHRUS_ECAPACITY and
+    are left untouched, the others match the oracle (20 sequences x 8
+    kv-heads: 160 CTAs, more than one wave)."""
+    lens = [5, 900, 0, 3000, 129, 2500, 77, 1800, 640, 1, 3333, 256, 1500, 12, 2048, 700,
+            999, 4000, 31, 1024]
+    inp = synth.attn_inputs(len(lens), 16, 8, 128, 16, lens, 4100, "bf16", seed=121)
+    bad = [3, 17]
+    lens_dev = np.array(lens, np.int32)
+    lens_dev[bad] = [3500, 4050]  # over max_ctx = 3400
+    inp_dev = dict(inp, ctx_lens=lens_dev)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((len(lens), 16, 16, 128), 7.0, device="cuda", dtype=torch.bfloat16)
+    run_gpu(inp_dev, 0, max_ctx=3400, err=err, out=out)
+    assert int(err.item()) == -4  # ORTHRUS_ECAPACITY
+    got = to_host(out)
+    good = [i for i in range(len(lens)) if i not in bad]
+    sub = {k: v[good] for k, v in inp.items()}
+    ref = oracle_mod.block_attn(sub["q"], sub["k_blk"], sub["v_blk"], sub["k_cache"],
+                                sub["v_cache"], sub["ctx_lens"], 0)
+    assert rel_err_rows(got[good], ref).max() <= TOL["bf16"]
+    assert np.all(got[bad] == 7.0)
+
+
 def test_one_workspace_reused_across_shapes(oracle_mod):
     """One bf16 workspace serves calls of different shapes in any order: the
     merge's arrival counts (the buffer's first 1024 bytes; the generations
