@@ -48,11 +48,13 @@
 // sum (fp32) to an L2-resident workspace, grouped by the query rows one
 // merging CTA owns, so that the owner fetches a split's share with one bulk
 // copy.  When the grid fits one wave (every CTA resident at once, the batch-1
-// decoding case) the merge runs inside the same launch: a sense-reversing
-// barrier per (sequence, kv-head) -- count in, the last CTA resets the count
-// and advances the generation the others wait on (bounded) -- then every CTA
-// stages its row group of all S partials by bulk copies and merges them in
-// split order (the result does not depend on timing) into bf16 output.
+// decoding case) the merge runs inside the same launch: a barrier per
+// (sequence, kv-head) on one (generation, count) word -- each CTA adds its
+// arrival without waiting for the atomic, the merging CTAs wait (bounded)
+// for the count of their generation to reach S, and split 0 then starts the
+// next generation -- then every merging CTA stages its row group of all S
+// partials by bulk copies and merges them in split order (the result does
+// not depend on timing) into bf16 output.
 // Larger grids, whose CTAs cannot all be resident, end instead and a second
 // kernel (attn_tc_combine, PDL-chained) merges the same way.  In such a grid
 // over 2..32 sequences the CTAs take their (sequence, split, kv-head) in
@@ -97,7 +99,7 @@ static_assert(kOCol + 2 * 128 <= kTmemCols, "TMEM columns at D = 128");
 constexpr float kLazyThresh = 8.f;  // log2 units
 constexpr int kMaxSplits = 24;      // the merge keeps every split's loads in registers
 constexpr int kCounterBytes = 2048;  // workspace head: merge counters, never partials
-constexpr int kMaxFusedHeads = kCounterBytes / 8;  // an arrival count and a generation each
+constexpr int kMaxFusedHeads = kCounterBytes / 8;  // one 64-bit (generation, count) word each
 constexpr int kGroupRows = 8;        // rows per CTA of the separate combine kernel
 constexpr int kCombineThreads = 256;
 
@@ -143,7 +145,7 @@ struct __align__(64) TcParams {
   float* part;         // [B][Hkv] x S split partials (workspace after the counters)
   int R;               // query rows per partial group = rows one merging CTA owns
   int order;           // launch order sorted by context length (B in [2, 32], unfused)
-  unsigned* counters;  // [B * Hkv] arrival counters of the in-kernel merge (kept at zero)
+  unsigned long long* counters;  // [B * Hkv] in-kernel merge: generation << 32 | arrivals
   int B, Hq, Hkv, blk, cap, max_ctx, mask_mode, G, S, early;
   float scale_log2;
 };
@@ -346,7 +348,7 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   // change before this CTA has arrived, and the previous call has completed
   unsigned gen0 = 0;
   if (kFused && threadIdx.x == 0)
-    gen0 = ptx::ld_acquire_gpu(p.counters + kMaxFusedHeads + (b * p.Hkv + g));
+    gen0 = (unsigned)(ptx::ld_acquire_gpu_u64(p.counters + (b * p.Hkv + g)) >> 32);
   if (bad && split == 0 && g == 0 && threadIdx.x == 0) set_err(p.err, ORTHRUS_ECAPACITY);
   int Tc, t0, U;
   geometry(n, Tc, t0, U);
@@ -665,38 +667,38 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
   if (!kFused) return;  // the combine kernel merges the splits
 
   // ---- split merge inside the launch (every CTA of the grid is resident at
-  // once: the host takes this path only when the grid fits one wave).  A
-  // sense-reversing barrier per (sequence, kv-head): each CTA notes the
-  // generation, publishes its partial and counts itself in; the last to
-  // arrive resets the count and advances the generation, which releases the
-  // others.  Then CTA `split` merges query rows [split * R, split * R + R)
-  // in split order and writes them.  No atomics follow the merge.
+  // once: the host takes this path only when the grid fits one wave).  One
+  // 64-bit word per (sequence, kv-head): generation << 32 | arrivals.  Each
+  // CTA publishes its partial and adds one arrival (fire and forget, after a
+  // fence); the CTAs that merge wait until the count reaches S within their
+  // generation.  Split 0, having seen it, moves to the next generation and
+  // returns the count to zero in one atomic -- a CTA that looks after that
+  // sees the new generation and goes on too.  Then CTA `split` merges query
+  // rows [split * R, split * R + R) in split order and writes them; the
+  // splits that own no rows leave once counted.
+  const bool merger = split * p.R < rows;
   volatile int* go = abort_flag + 1;
   if (threadIdx.x == 0) {
-    const int hidx = b * p.Hkv + g;
-    unsigned* cnt = p.counters + hidx;
-    unsigned* gen = p.counters + kMaxFusedHeads + hidx;
+    unsigned long long* word = p.counters + (b * p.Hkv + g);
     __threadfence();  // this CTA's partial is visible before it is counted
+    atomicAdd(word, 1ull);
     int ok = 1;
-    if (atomicAdd(cnt, 1u) == (unsigned)S - 1u) {
-      // every split has arrived: release the others first (the fence orders
-      // the partials acquired through the count before the generation), then
-      // ready the count for the next call, which starts after this one ends
-      __threadfence();
-      atomicAdd(gen, 1u);
-      atomicExch(cnt, 0u);
-    } else {
+    if (merger) {
       const uint64_t t0 = ptx::globaltimer();
-      while (ptx::ld_acquire_gpu(gen) == gen0) {
+      for (;;) {
+        const unsigned long long w = ptx::ld_acquire_gpu_u64(word);
+        if ((unsigned)(w >> 32) != gen0 || (unsigned)w == (unsigned)S) break;
         if (ptx::globaltimer() - t0 > 1000000000ull) {
           set_err(p.err, ORTHRUS_ETIMEOUT);
           ok = 0;
           break;
         }
       }
+      if (ok && split == 0) atomicAdd(word, (1ull << 32) - (unsigned long long)S);
     }
     *go = ok;
   }
+  if (!merger) return;
   __syncthreads();
   if (*go && !bad)
     merge_rows<kD>(p, b, g, split, threadIdx.x, kThreads, smem + kRingOff, bars.merge_full());
@@ -948,7 +950,7 @@ int tc_launch(const orthrus_attn_args& a, cudaStream_t st) {
   if (!p.next_k || !p.next_v) p.next_k = p.next_v = nullptr;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = a.err;
-  p.counters = static_cast<unsigned*>(a.workspace);
+  p.counters = static_cast<unsigned long long*>(a.workspace);
   p.part = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + kCounterBytes);
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.blk = a.blk; p.cap = a.cap;
   p.max_ctx = a.max_ctx; p.mask_mode = a.mask_mode; p.G = G; p.S = S;

@@ -133,10 +133,12 @@ typedef struct orthrus_attn_args {
 /* Workspace of orthrus_block_attn: the per-split partial results of the
  * split-KV reduction (unnormalised O plus row max and row sum), written and
  * read back within the call.  The BF16 tensor-core path also keeps, in the
- * buffer's first 2048 bytes, the counters of its in-launch merge:
- * zero the buffer once (cudaMemset 0); every call leaves the counters at
- * zero, so one buffer serves any later FP32 and BF16 calls on one stream
- * whose sizes fit it (zero it again after a call that reported an error).
+ * buffer's first 2048 bytes, the state of its in-launch merge (a 64-bit
+ * generation and arrival count per (sequence, kv-head)): zero the buffer
+ * once (cudaMemset 0); every call leaves each count at zero and moves the
+ * generations it used on by one, so one buffer serves any later FP32 and
+ * BF16 calls on one stream whose sizes fit it (zero it again after a call
+ * that reported an error).
  * A BF16 call whose grid fits one wave (see orthrus_block_attn_plan) counts
  * on all of its CTAs being resident together: do not run it concurrently
  * with kernels (other streams) that could hold SMs until it ends -- the

@@ -190,14 +190,17 @@ def test_multi_wave_grid_with_lengths_over_bound(oracle_mod):
 
 
 def test_one_workspace_reused_across_shapes(oracle_mod):
-    """One bf16 workspace serves calls of different shapes in any order: the
-    merge's arrival counts (the buffer's first 1024 bytes; the generations
-    follow, and no partial is ever written there) are back at zero after
-    every call."""
+    """One bf16 workspace serves calls of different shapes in any order.  The
+    in-launch merge keeps one 64-bit word per (sequence, kv-head) in the
+    buffer's first 2048 bytes (these shapes all fit one wave): the arrival
+    count (low half) is back at zero after every call and the generation
+    (high half) of every head the call covers has moved on by exactly one;
+    no partial is ever written there."""
     ws = ba.Workspace("cuda")
     shapes = [(2, 32, 8, 128, 32, [3000, 500]), (1, 4, 1, 64, 32, [100]),
               (1, 16, 8, 128, 32, [2048]), (1, 8, 8, 128, 4, [0]),
               (3, 32, 8, 128, 32, [900, 10, 4000]), (1, 16, 8, 128, 32, [2048])]
+    gens = np.zeros(256, np.int64)
     for k, (B, Hq, Hkv, D, blk, lens) in enumerate(shapes):
         inp = synth.attn_inputs(B, Hq, Hkv, D, blk, lens, max(lens) + 8, "bf16", seed=300 + k)
         t = {kk: to_dev(v) for kk, v in inp.items()}
@@ -209,7 +212,10 @@ def test_one_workspace_reused_across_shapes(oracle_mod):
                                         inp["v_cache"], inp["ctx_lens"], mode)
             e = rel_err_rows(to_host(out), ref)
             assert e.max() <= TOL["bf16"], (k, mode, e.max())
-            assert int(ws.buf[:1024].count_nonzero()) == 0, (k, mode)
+            words = ws.buf[:2048].cpu().numpy().view(np.uint64)
+            assert not (words & 0xFFFFFFFF).any(), (k, mode)  # counts back at zero
+            gens[:B * Hkv] += 1
+            assert np.array_equal((words >> 32).astype(np.int64), gens), (k, mode)
 
 
 @pytest.mark.parametrize("mode", [0, 1])
