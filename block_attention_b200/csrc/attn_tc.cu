@@ -705,11 +705,11 @@ attn_tc_kernel(const __grid_constant__ TcParams p) {
 }
 
 // Merge the S split partials of query-row group q (rows [q R, q R + R)) of
-// (sequence b, kv-head g) and write bf16 output.  One thread stages every
-// split's block of the group into shared memory with bulk copies (one each,
-// all in flight at once, completing on `bar`); then one item per (row,
-// 16-byte chunk) merges the splits in index order, so the result does not
-// depend on timing.  `stage` holds S * (D/4 + 1) * R float4s.  Every thread
+// (sequence b, kv-head g) and write bf16 output.  The first warp stages
+// every split's block of the group into shared memory with bulk copies (lane
+// s the split s, all in flight at once, completing on `bar`); then one item
+// per (row, 16-byte chunk) merges the splits in index order, so the result
+// does not depend on timing.  `stage` holds S * (D/4 + 1) * R float4s.  Every thread
 // of the CTA calls this with the same q (the barrier inside is CTA-wide).
 template <int kD>
 __device__ __forceinline__ void merge_rows(const TcParams& p, int b, int g, int q, int tid,
@@ -723,15 +723,19 @@ __device__ __forceinline__ void merge_rows(const TcParams& p, int b, int g, int 
   float4* st4 = reinterpret_cast<float4*>(stage);
   const float4* base = reinterpret_cast<const float4*>(
       p.part + (int64_t)(b * p.Hkv + g) * S * part_floats<kD>());
-  if (tid == 0) {
-    // the partials were written by other CTAs' generic stores, acquired by
-    // this thread; the bulk copies read them through the async proxy
-    ptx::fence_proxy_async_global();
-    ptx::mbar_expect_tx(bar, (uint32_t)(S * gf4 * 16));
-    for (int s2 = 0; s2 < S; ++s2)
+  if (tid < 32) {
+    // lane s copies split s's block (the copies go out together); the
+    // partials were written by other CTAs' generic stores, acquired through
+    // the CTA's barrier after thread 0's acquire, and the bulk copies read
+    // them through the async proxy
+    if (tid == 0) ptx::mbar_expect_tx(bar, (uint32_t)(S * gf4 * 16));
+    __syncwarp();
+    for (int s2 = tid; s2 < S; s2 += 32) {
+      ptx::fence_proxy_async_global();
       ptx::bulk_g2s(ptx::smem_u32(st4 + s2 * gf4),
                     base + (int64_t)s2 * (part_floats<kD>() / 4) + (int64_t)q * gf4,
                     (uint32_t)(gf4 * 16), bar);
+    }
   }
   if (!ptx::mbar_wait(bar, 0)) {
     set_err(p.err, ORTHRUS_ETIMEOUT);
