@@ -121,6 +121,22 @@ def test_ragged_batch_sampled_sequences(oracle_mod):
             assert e.max() <= TOL["bf16"], (b, mode, e.max())
 
 
+@pytest.mark.parametrize("B,Hkv", [(32, 8), (40, 4)])
+def test_many_sequences_multi_wave(oracle_mod, B, Hkv):
+    """More kv-head rows than SMs (one split each, two launches): 32
+    sequences take the length-sorted launch order, 40 the grid order; every
+    sequence matches the oracle in both views."""
+    lens = [int(x) for x in np.random.default_rng(B).integers(0, 600, B)]
+    lens[3] = 0
+    inp = synth.attn_inputs(B, 2 * Hkv, Hkv, 128, 8, lens, max(lens) + 10, "bf16", seed=130 + B)
+    for mode in (0, 1):
+        ref = oracle_mod.block_attn(inp["q"], inp["k_blk"], inp["v_blk"], inp["k_cache"],
+                                    inp["v_cache"], inp["ctx_lens"], mode)
+        got = to_host(run_gpu(inp, mode))
+        e = rel_err_rows(got, ref)
+        assert e.max() <= TOL["bf16"], (mode, e.max(), np.unravel_index(e.argmax(), e.shape))
+
+
 def test_f32_causal_row_equals_single_token_decode_bitwise():
     """Verify row i over (cache n, block) == one-row decode at n+i over
     (cache n+i, block of 1), bit for bit, across split and tile boundaries."""
