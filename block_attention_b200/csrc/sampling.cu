@@ -311,9 +311,12 @@ vocab_sample_kernel(const T* __restrict__ logits, int vocab, int64_t stride, flo
 }
 
 // ------------------------------------------------------------ log-prob at T
-// Grid (chunks, rows); element e of thread t is c * kChunk + e * kThreads + t
-// (coalesced).  The row's last CTA merges the chunk pairs.  Workspace:
-// tickets [rows] then the pairs [rows][chunks].
+// Grid (chunks, rows); chunk c holds elements [c kChunk, (c + 1) kChunk) of
+// the row.  With kVec thread t reads groups of four, elements c kChunk +
+// 4 (g kThreads + t) + 0..3 for g < kPer / 4 (one 16- or 8-byte load each);
+// otherwise element e is c kChunk + e kThreads + t.  Both coalesce.  The
+// row's last CTA merges the chunk pairs.  Workspace: tickets [rows] then the
+// pairs [rows][chunks].
 template <typename T, bool kVec>
 __device__ __forceinline__ float load_chunk(const T* row, int c, int vocab, float inv_t,
                                             float (&x)[kPer]) {
