@@ -97,7 +97,7 @@ constexpr int kTmemCols = 512;      // S0 [0,128) S1 [128,256) O_0 [256,256+D) O
 constexpr int kOCol = 256;
 static_assert(kOCol + 2 * 128 <= kTmemCols, "TMEM columns at D = 128");
 constexpr float kLazyThresh = 8.f;  // log2 units
-constexpr int kMaxSplits = 24;      // the merge keeps every split's loads in registers
+constexpr int kMaxSplits = 24;      // bounds the partials (kPartRows) and the merge's staging
 constexpr int kCounterBytes = 2048;  // workspace head: merge counters, never partials
 constexpr int kMaxFusedHeads = kCounterBytes / 8;  // one 64-bit (generation, count) word each
 constexpr int kGroupRows = 8;        // rows per CTA of the separate combine kernel
