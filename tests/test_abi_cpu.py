@@ -343,6 +343,11 @@ def test_tensor_core_attention_plan(L):
     # at most 4 of the 65 tiles each, merged inside the launch
     assert L.orthrus_block_attn_plan(ctypes.byref(a), 148, out) == 0
     assert list(out)[:4] == [18, 8, 1, 18] and out[6] == 4 and out[7] == 1
+    # the Qwen3-1.7B layer (ctx 2048, 17 tiles): 8 splits of two or three
+    # tiles rather than 17 of one, merged inside the launch
+    a = _args(dtype=1, B=1, Hq=16, Hkv=8, D=128, blk=32, max_ctx=2048, cap=2080, scale=0.1)
+    assert L.orthrus_block_attn_plan(ctypes.byref(a), 148, out) == 0
+    assert list(out)[:4] == [8, 8, 1, 8] and out[6] == 3 and out[7] == 1
 
 
 def test_linear_tc_plan_and_rejections(L):
