@@ -79,6 +79,35 @@ def max_over_ranks(values, device):
     return [float(x) for x in t.tolist()]
 
 
+def bind_host_to_gpu(dev_index):
+    """Run this process on the CPUs nearest the GPU (NVML's affinity for the
+    GPU's PCI address), so that pinned host buffers allocated afterwards sit
+    on the GPU's NUMA node and host-device copies do not cross the socket
+    interconnect.  A setting of this process only (nothing of the GPU is
+    changed).  Returns (previous CPU set, description), or (None, None)
+    where the affinity cannot be read."""
+    try:
+        import pynvml
+        import torch
+        prop = torch.cuda.get_device_properties(dev_index)
+        bus = f"{prop.pci_domain_id:08x}:{prop.pci_bus_id:02x}:{prop.pci_device_id:02x}.0"
+        pynvml.nvmlInit()
+        try:
+            handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            words = pynvml.nvmlDeviceGetCpuAffinity(handle, ((os.cpu_count() or 64) + 63) // 64)
+        finally:
+            pynvml.nvmlShutdown()
+        before = os.sched_getaffinity(0)
+        near = {64 * i + b for i, w in enumerate(words) for b in range(64) if (w >> b) & 1}
+        near &= before
+        if not near or near == before:
+            return None, None
+        os.sched_setaffinity(0, near)
+        return before, f"{len(near)} of {len(before)} cpus, the GPU's NUMA node"
+    except Exception:
+        return None, None
+
+
 def whole_job_rate(world, steps, ms):
     """Units per second completed by all ranks together: every rank runs
     `steps` units of its own (weak scaling), in at most `ms` milliseconds."""
@@ -965,6 +994,7 @@ def main():
     # Two input sets: round i+1's inputs are copied in on a second stream
     # while round i runs on the other set; every round's copy, graph and
     # result read-back are inside the timed region.
+    cpus_before, host_cpus = bind_host_to_gpu(local)
     h_in, h_out = rnd.pinned_inputs(), rnd.pinned_outputs()
     rnd.add_input_set()
     comp, copy = torch.cuda.current_stream(dev), torch.cuda.Stream(device=dev)
@@ -1007,6 +1037,8 @@ def main():
     rnd.use_set(0)
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
     e2e_rounds = whole_job_rate(world, args.steps, e2e_ms)
+    if cpus_before:
+        os.sched_setaffinity(0, cpus_before)  # the CPU legs below use every core
     assert np.array_equal(h_out["n_emit"].numpy(), expect_ne)
     check_probe("end-to-end rounds")
 
@@ -1074,7 +1106,7 @@ def main():
         "round_hbm_gbs": sum(rb.values()) / (total_ms / args.steps * 1e-3) / 1e9,
         "step_ms_median": statistics.median(step_ms),
         "e2e": {"value": e2e_rounds, "unit": "rounds/s", "h2d_bytes_per_step": bi,
-                "d2h_bytes_per_step": bo},
+                "d2h_bytes_per_step": bo, "host_cpus": host_cpus or "unbound"},
         "gpu_launches": gpu_launches,
         "clocks": clk,
         "cpu_baseline": cpu,
